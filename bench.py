@@ -1,0 +1,427 @@
+"""Benchmark of the blockwise 4-bit quantization hot path on B200.
+
+One step = one pass of every hot-path operation over the Llama-2-7B-shaped
+decoder layer (q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008):
+  1. load-time quantize of L distinct layer copies (bf16 ~ N(0, 0.02) ->
+     NF4 blocksize 64 with double quantization of the absmax);
+  2. fused dequant-GEMV of every layer copy at decode batch M = 1, 4, 16
+     (fp16 activations ~ N(0, 1), fp32 accumulate, fp16 out), one grouped
+     launch per layer;
+  3. dequantize of every layer copy to bf16;
+  4. W4A16 tcgen05 GEMM of every layer copy at prefill M = 512 (bf16).
+The L = 4 copies (~2 GB of inputs) rotate, so every kernel reads data that
+was last touched more than the 126 MB L2 ago.  `value` is the headline
+metric: GEMV effective HBM TB/s = algorithmic bytes (packed weights + block
+state + activations + outputs) / device time of the GEMV launches; quantize
+GB/s (input bytes / time) and every kernel's roofline are reported beside it.
+
+Multi-GPU: the path does not shard (a single-GPU format and kernels); with
+--gpus N every rank runs an independent replica (weak scaling) and the
+whole-job value is the sum of bytes over the max time across ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "4-bit GEMV effective HBM TB/s (7B shapes, batch 1-16); quantize GB/s"
+UNIT = "TB/s"
+WORKLOAD = "llama2-7b-layer-nf4-b64-dq"
+DECODE_M = (1, 4, 16)
+PREFILL_M = 512
+N_COPIES = 4
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def layer_state_bytes(shapes, blocksize=64):
+    """Resident NF4 + double-quant bytes of one layer (codes, int8 absmax
+    codes, fp32 second-level scales, fp32 mean)."""
+    tot = 0
+    for _, N, K in shapes:
+        n = N * K
+        nb = -(-n // blocksize)
+        tot += (n + 1) // 2 + nb + 4 * (-(-nb // 256)) + 4
+    return tot
+
+
+def gemv_bytes(shapes, M):
+    return layer_state_bytes(shapes) + sum(2 * M * K + 2 * M * N for _, N, K in shapes)
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ------------------------------------------------------------- CPU oracle ---
+def oracle_sample(rows_per_matrix=16, seed=0):
+    """Time the oracle on a bounded sample of the same workload: NF4 + DQ
+    quantize of one 4096x4096 bf16 matrix, and the GEMV reference (dequantize
+    + binary64 matmul) of the first `rows_per_matrix` rows of every matrix of
+    the layer at M = 1, 4, 16.  Returns (TB/s of GEMV algorithmic bytes,
+    quantize GB/s, threads, description, seconds)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    threads = oracle.set_threads(os.cpu_count() or 1)
+    t0 = time.perf_counter()
+    W = wl.gaussian((4096, 4096), 0.02, torch.bfloat16, seed)
+    wb = W.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    tq = time.perf_counter()
+    oracle.quantize(wb, True, 64, oracle.QT_NF4, True)
+    tq = time.perf_counter() - tq
+    q_gbs = wb.size * 2 / tq / 1e9
+    sub_bytes = 0
+    tg = 0.0
+    for i, (_, N, K) in enumerate(wl.LAYER_7B):
+        Wr = wl.gaussian((rows_per_matrix, K), 0.02, torch.bfloat16, seed + 1 + i)
+        st = oracle.quantize(Wr.view(torch.int16).numpy().view(np.uint16).reshape(-1), True, 64,
+                             oracle.QT_NF4, True)
+        for M in DECODE_M:
+            A = wl.activation(M, K, torch.float16, seed + 50 + i)
+            ab = A.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+            t = time.perf_counter()
+            oracle.gemv_reference(ab, False, st, rows_per_matrix, K)
+            tg += time.perf_counter() - t
+            sub_bytes += layer_state_bytes([("s", rows_per_matrix, K)]) + 2 * M * K + 2 * M * rows_per_matrix
+    desc = (f"oracle on host cores: NF4+DQ quantize of one 4096x4096 bf16 matrix, and the GEMV "
+            f"reference (dequantize + fp64 matmul) of the first {rows_per_matrix} rows of each "
+            f"of the 7 layer matrices at M=1,4,16; bytes scaled per row")
+    return sub_bytes / tg / 1e12, q_gbs, threads, desc, time.perf_counter() - t0
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    vals, qs = [], []
+    for i in range(warm + steps):
+        tb, qg, thr, desc, secs = oracle_sample(rows_per_matrix=8, seed=i)
+        if i >= warm:
+            vals.append(tb)
+            qs.append(qg)
+    v = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": steps, "warmup": warm, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "decode_M": list(DECODE_M), "sample": "8 rows per matrix"},
+            "quantize_gbs": statistics.mean(qs),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm --
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from bit_blockwise_weight_absmax_b200 import q4
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    shapes = wl.LAYER_7B
+    peaks = _peaks()
+    L = N_COPIES
+
+    # ---- inputs resident in HBM before timing (seeded, generated on device)
+    Ws = [[wl.gaussian((N, K), 0.02, torch.bfloat16, 1000 * l + i + 17 * rank, dev)
+           for i, (_, N, K) in enumerate(shapes)] for l in range(L)]
+    A_dec = {M: [wl.activation(M, K, torch.float16, 7000 + 10 * M + i, dev) for i, (_, N, K) in enumerate(shapes)]
+             for M in DECODE_M}
+    A_pre = [wl.activation(PREFILL_M, K, torch.bfloat16, 9000 + i, dev) for i, (_, N, K) in enumerate(shapes)]
+    states = [[q4.quantize(w, 64, "nf4", True) for w in layer] for layer in Ws]
+    y_dec = {M: [[torch.empty(M, N, dtype=torch.float16, device=dev) for _, N, K in shapes]
+                 for _ in range(L)] for M in DECODE_M}
+    deq_out = [torch.empty(N, K, dtype=torch.bfloat16, device=dev) for _, N, K in shapes]
+    y_pre = [torch.empty(PREFILL_M, N, dtype=torch.bfloat16, device=dev) for _, N, K in shapes]
+    torch.cuda.synchronize()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    n_params = sum(N * K for _, N, K in shapes)
+
+    # Every phase is one CUDA graph of library launches (captured once after
+    # an eager warm-up), so no host-side marshalling falls inside a timed
+    # interval; graphs replay back to back on one stream.
+    def ph_quantize():
+        for l in range(L):
+            for w, st in zip(Ws[l], states[l]):
+                q4.quantize(w, 64, "nf4", True, out=st)
+
+    def ph_gemv(M):
+        for l in range(L):
+            q4.gemv_grouped(A_dec[M], states[l], outs=y_dec[M][l])
+
+    def ph_dequantize():
+        for l in range(L):
+            for st, o in zip(states[l], deq_out):
+                q4.dequantize(st, torch.bfloat16, out=o)
+
+    def ph_gemm():
+        for l in range(L):
+            q4.gemm_grouped(A_pre, states[l], outs=y_pre)
+
+    fns = {"quantize": ph_quantize}
+    for M in DECODE_M:
+        fns[f"gemv_m{M}"] = (lambda M=M: ph_gemv(M))
+    fns["dequantize"] = ph_dequantize
+    fns["gemm"] = ph_gemm
+    phases = list(fns)
+    launches = {"quantize": L * len(shapes) * 2, "dequantize": L * len(shapes), "gemm": L}
+    for M in DECODE_M:
+        launches[f"gemv_m{M}"] = L
+    launches_per_step = sum(launches.values())
+    for f in fns.values():
+        f()
+    torch.cuda.synchronize()
+    graphs = {}
+    for name, f in fns.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            f()
+        graphs[name] = g
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step(rec):
+        for name in phases:
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            graphs[name].replay()
+            e1.record(stream)
+            rec[name].append((e0, e1))
+
+    for _ in range(args.warmup):
+        step({p: [] for p in phases})
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    rec = {p: [] for p in phases}
+    t_start, t_end = ev(), ev()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(rec)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+
+    total_ms = t_start.elapsed_time(t_end)
+    ph_ms = {p: sum(a.elapsed_time(b) for a, b in rec[p]) for p in phases}
+    gemv_B = {M: gemv_bytes(shapes, M) * L * args.steps for M in DECODE_M}
+    gemv_ms = sum(ph_ms[f"gemv_m{M}"] for M in DECODE_M)
+    q_in_bytes = 2 * n_params * L * args.steps
+    state_b = layer_state_bytes(shapes)
+    q_alg_bytes = (2 * n_params + state_b) * L * args.steps
+    deq_alg_bytes = (state_b + 2 * n_params) * L * args.steps
+    gemm_flops = 2 * PREFILL_M * n_params * L * args.steps
+
+    # max over ranks of the device times; value = all ranks' bytes / that time
+    import torch as _t
+    vec = _t.tensor([total_ms, gemv_ms] + [ph_ms[p] for p in phases], dtype=_t.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vec, op=dist.ReduceOp.MAX)
+    total_ms, gemv_ms = vec[0].item(), vec[1].item()
+    ph_ms = {p: vec[2 + i].item() for i, p in enumerate(phases)}
+
+    value = world * sum(gemv_B.values()) / (gemv_ms / 1e3) / 1e12
+    per_m = {f"M={M}": {"tb_s": gemv_B[M] / (ph_ms[f"gemv_m{M}"] / 1e3) / 1e12,
+                        "us_per_layer": ph_ms[f"gemv_m{M}"] * 1e3 / (L * args.steps),
+                        "bytes_per_layer": gemv_bytes(shapes, M)} for M in DECODE_M}
+    hbm = peaks["hbm_gbs"]
+    quant_gbs = q_in_bytes / (ph_ms["quantize"] / 1e3) / 1e9
+    rooflines = {
+        "quantize": {"bound": "hbm", "achieved": q_alg_bytes / (ph_ms["quantize"] / 1e3) / 1e9,
+                     "peak": hbm, "unit": "GB/s"},
+        "gemv": {"bound": "hbm", "achieved": sum(gemv_B.values()) / (gemv_ms / 1e3) / 1e9, "peak": hbm,
+                 "unit": "GB/s"},
+        "dequantize": {"bound": "hbm", "achieved": deq_alg_bytes / (ph_ms["dequantize"] / 1e3) / 1e9,
+                       "peak": hbm, "unit": "GB/s"},
+        "gemm": {"bound": "tensor", "achieved": gemm_flops / (ph_ms["gemm"] / 1e3) / 1e12,
+                 "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s"},
+    }
+    for r in rooflines.values():
+        r["frac"] = r["achieved"] / r["peak"]
+    dominant = max(["quantize", "dequantize", "gemm"] + ["gemv"],
+                   key=lambda k: gemv_ms if k == "gemv" else ph_ms[k])
+    dom = dict(rooflines[dominant])
+    dom["kernel"] = dominant
+    dom["launch_us"] = (gemv_ms if dominant == "gemv" else ph_ms[dominant]) * 1e3 / (
+        args.steps * (L * len(DECODE_M) if dominant == "gemv" else launches[dominant]))
+    dom["traffic"] = None
+    dom["peak_source"] = f"{peaks['source']} ({'bf16_tflops_sustained' if dom['bound'] == 'tensor' else 'hbm_gbs'})"
+
+    # ---- end to end through the public API: pinned host activations in,
+    # results back to host, weights resident (quantized at load time)
+    e2e = None
+    if not args.no_e2e:
+        host_A = {M: [a.cpu().pin_memory() for a in A_dec[M]] for M in DECODE_M}
+        host_Y = {M: [torch.empty(M, N, dtype=torch.float16).pin_memory() for _, N, K in shapes]
+                  for M in DECODE_M}
+        dev_A = {M: [torch.empty_like(a) for a in A_dec[M]] for M in DECODE_M}
+        h2d = sum(a.numel() * 2 for M in DECODE_M for a in A_dec[M]) * L
+        d2h = sum(M * N * 2 for M in DECODE_M for _, N, K in shapes) * L
+
+        def e2e_step():
+            for M in DECODE_M:
+                for l in range(L):
+                    for da, ha in zip(dev_A[M], host_A[M]):
+                        da.copy_(ha, non_blocking=True)
+                    ys = q4.gemv_grouped(dev_A[M], states[l], outs=y_dec[M][l], stream=stream)
+                    for hy, y in zip(host_Y[M], ys):
+                        hy.copy_(y, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        e0, e1 = ev(), ev()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        v = _t.tensor([e2e_ms], dtype=_t.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(v, op=dist.ReduceOp.MAX)
+        e2e_ms = v.item()
+        e2e = {"value": world * sum(gemv_B.values()) / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "what": "q4.gemv_grouped at M=1,4,16 over the resident layer copies, activations "
+                       "copied from pinned host memory and outputs read back every call"}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        tb, qg, thr, desc, secs = oracle_sample(rows_per_matrix=16)
+        cpu = {"value": tb, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc,
+               "quantize_gbs": qg, "seconds": round(secs, 1)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic (seeded Gaussian weights of 7B-layer shapes; no checkpoint)",
+            "config": {"workload": WORKLOAD, "decode_M": list(DECODE_M), "prefill_M": PREFILL_M,
+                       "layer_copies": L, "blocksize": 64, "double_quant": True,
+                       "l2": f"{L} rotating layer copies (~{L * 2 * n_params / 1e9:.1f} GB bf16 + "
+                             f"{L * state_b / 1e6:.0f} MB packed) > 126 MB L2",
+                       "parallelism": f"replicas x{world}"},
+            "quantize_gbs": quant_gbs,
+            "gemv_per_m": per_m,
+            "phase_ms_per_step": {p: ph_ms[p] / args.steps for p in phases},
+            "roofline": dom,
+            "rooflines": rooflines,
+            "gpu_launches": launches_per_step * args.steps,
+            "launches_per_step": launches,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="q4", choices=["q4", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,26 @@
+// k_gemm.cu -- launcher of the tcgen05 W4A16 GEMM kernel.
+#include <algorithm>
+
+#include "q4_internal.h"
+
+namespace q4 {
+namespace {
+template <int DA>
+int go(const GemmParams &p, int sms, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(gemm_kernel<DA>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
+        cudaSuccess)
+      return Q4_ERR_CUDA;
+    attr = true;
+  }
+  const int grid = (int)std::min<int64_t>(p.total_tiles, (int64_t)sms);
+  gemm_kernel<DA><<<grid, kGemmThreads, kGemmSmem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+}  // namespace
+
+int run_gemm(int da, const GemmParams &p, int sms, cudaStream_t st) {
+  return da == Q4_F16 ? go<Q4_F16>(p, sms, st) : go<Q4_BF16>(p, sms, st);
+}
+}  // namespace q4

@@ -1,0 +1,495 @@
+// q4_api.cu -- the C ABI of include/q4.h (libq4.so).
+//
+// Host side only: argument validation, launch planning, TMA descriptors and
+// status codes.  Every step of the computation runs in the sm_100a kernels of
+// the other translation units; the host never touches tensor data and never
+// allocates device memory.
+#include <cuda.h>
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "q4_internal.h"
+
+namespace q4 {
+__device__ int g_status = 0;
+}
+
+using namespace q4;
+
+namespace {
+
+// The 16 NF4 levels exactly as printed on n4n.ai, "What is 4-bit
+// quantization and why does it matter?", code block "Conceptual NF4
+// dequantization", read as binary32.
+const float kNF4Levels[16] = {-1.0f,  -0.696f, -0.525f, -0.395f, -0.284f, -0.185f,
+                              -0.091f, 0.0f,    0.079f,  0.161f,  0.246f,  0.338f,
+                              0.441f,  0.562f,  0.720f,  1.0f};
+
+// Decision thresholds of nearest-level coding: t_i is the smallest binary32 x
+// whose nearest level is L_{i+1} or above.  At an exact midpoint the level of
+// smaller magnitude wins (the pages give no tie rule).
+void derive_thresholds(float t[15]) {
+  for (int i = 0; i < 15; ++i) {
+    const double lo = kNF4Levels[i], hi = kNF4Levels[i + 1];
+    const double m = (lo + hi) * 0.5;  // exact in binary64
+    const bool tie_goes_up = fabs(hi) < fabs(lo);
+    float f = (float)m;
+    if (tie_goes_up) {
+      if ((double)f < m) f = nextafterf(f, INFINITY);
+    } else {
+      if ((double)f <= m) f = nextafterf(f, INFINITY);
+    }
+    t[i] = f;
+  }
+}
+
+// Bin table of the quantize kernel: the bin of x is the low 5 bits of
+// fmaf(x, 15, 12582927) (round(15x) + 15); each bin may hold one threshold.
+bool build_bin_table(Nf4BinTable *tab) {
+  float t[15];
+  derive_thresholds(t);
+  int bin_of[15];
+  for (int i = 0; i < 15; ++i) {
+    const float v = fmaf(t[i], 15.0f, 12582927.0f);
+    uint32_t u;
+    memcpy(&u, &v, 4);
+    bin_of[i] = (int)(u & 31u);
+  }
+  for (int j = 0; j < 32; ++j) {
+    tab->thr[j] = INFINITY;
+    tab->base[j] = 0;
+    int hits = 0;
+    for (int i = 0; i < 15; ++i) {
+      if (bin_of[i] < j) tab->base[j]++;
+      if (bin_of[i] == j) {
+        tab->thr[j] = t[i];
+        hits++;
+      }
+    }
+    if (hits > 1) return false;
+  }
+  return true;
+}
+
+struct DeviceInfo {
+  int ok = Q4_ERR_NO_DEVICE;
+  int sms = 0;
+  int *status = nullptr;  // device address of q4::g_status
+};
+
+DeviceInfo device_info() {
+  static DeviceInfo cache[64];
+  static bool filled[64] = {};
+  static std::mutex mu;
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess || count == 0) {
+    cudaGetLastError();
+    return DeviceInfo{};
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceInfo{Q4_ERR_CUDA, 0, nullptr};
+  std::lock_guard<std::mutex> lk(mu);
+  if (filled[dev]) return cache[dev];
+  DeviceInfo d;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  d.ok = (major == 10 && minor == 0) ? Q4_OK : Q4_ERR_ARCH;
+  if (d.ok == Q4_OK) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, q4::g_status) != cudaSuccess) {
+      cudaGetLastError();
+      d.ok = Q4_ERR_CUDA;
+    }
+    d.status = reinterpret_cast<int *>(ptr);
+  }
+  cache[dev] = d;
+  filled[dev] = true;
+  return d;
+}
+
+inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+inline bool valid_bs(int b) { return b == 32 || b == 64 || b == 128 || b == 256; }
+inline bool valid_in_dtype(int d) { return d == Q4_F16 || d == Q4_BF16; }
+inline bool valid_out_dtype(int d) { return d == Q4_F16 || d == Q4_BF16 || d == Q4_F32; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int check_state(const q4_state *s) {
+  if (!s || !s->packed) return Q4_ERR_ARG;
+  if (s->qtype < 0 || s->qtype > 2 || !valid_bs(s->blocksize)) return Q4_ERR_ARG;
+  if (s->double_quant) {
+    if (s->qtype != Q4_NF4 || !s->absmax_q || !s->absmax_scale || !s->absmax_mean) return Q4_ERR_ARG;
+  } else if (!s->absmax) {
+    return Q4_ERR_ARG;
+  }
+  if (s->qtype == Q4_INT4_ASYM && !s->zero) return Q4_ERR_ARG;
+  if (s->n < 1 || s->rows < 1 || s->cols < 1 || s->rows * s->cols != s->n) return Q4_ERR_SHAPE;
+  if (!aligned16(s->packed)) return Q4_ERR_ALIGN;
+  return Q4_OK;
+}
+
+// ---- GEMV planning: rows per unit (16 * r), n8 tiles, k per unit ---------------
+constexpr int kGemvUnitK = 1024;
+struct GemvPlan {
+  int nt, r;
+};
+GemvPlan gemv_plan(int64_t M) {
+  if (M <= 8) return {1, 1};
+  if (M <= 16) return {2, 2};
+  return {4, 2};
+}
+size_t gemv_ws_for(const q4_state *s, int64_t M, int64_t *n_tiles, int64_t *n_splits) {
+  const GemvPlan pl = gemv_plan(M);
+  *n_tiles = ceil_div(s->rows, 16 * pl.r);
+  *n_splits = ceil_div(s->cols / s->blocksize, kGemvUnitK / s->blocksize);
+  if (*n_splits <= 1) return 0;
+  return align256((size_t)s->rows * (size_t)M * 4) + align256((size_t)*n_tiles * 4);
+}
+
+// ---- TMA descriptors ----------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `esize`-byte elements, box {bx, by}.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t rows, int64_t cols,
+              int esize, int bx, int by, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(cols * esize)};
+  const cuuint32_t box[2] = {(cuuint32_t)bx, (cuuint32_t)by};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// =============================================================================
+extern "C" {
+
+const char *q4_strerror(int code) {
+  switch (code) {
+    case Q4_OK: return "ok";
+    case Q4_ERR_ARG: return "invalid argument";
+    case Q4_ERR_SHAPE: return "invalid shape";
+    case Q4_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case Q4_ERR_NO_DEVICE: return "no CUDA device (there is no CPU fallback)";
+    case Q4_ERR_ARCH: return "device is not sm_100 (B200)";
+    case Q4_ERR_CUDA: return "CUDA runtime error";
+    case Q4_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown error";
+}
+
+int q4_nf4_levels(float out[16]) {
+  if (!out) return Q4_ERR_ARG;
+  memcpy(out, kNF4Levels, sizeof(kNF4Levels));
+  return Q4_OK;
+}
+
+int q4_nf4_thresholds(float out[15]) {
+  if (!out) return Q4_ERR_ARG;
+  derive_thresholds(out);
+  return Q4_OK;
+}
+
+int q4_check_device(void) { return device_info().ok; }
+
+int q4_state_sizes(int32_t qtype, int64_t n, int32_t blocksize, int32_t double_quant,
+                   size_t sizes_out[6]) {
+  if (!sizes_out || qtype < 0 || qtype > 2 || !valid_bs(blocksize) ||
+      (double_quant != 0 && double_quant != 1) || (double_quant && qtype != Q4_NF4))
+    return Q4_ERR_ARG;
+  if (n < 1) return Q4_ERR_SHAPE;
+  const int64_t nb = ceil_div(n, blocksize);
+  sizes_out[0] = (size_t)((n + 1) / 2);
+  sizes_out[1] = (size_t)nb * 4;
+  sizes_out[2] = qtype == Q4_INT4_ASYM ? (size_t)((nb + 1) / 2) : 0;
+  sizes_out[3] = double_quant ? (size_t)nb : 0;
+  sizes_out[4] = double_quant ? (size_t)ceil_div(nb, Q4_DQ_GROUP) * 4 : 0;
+  sizes_out[5] = double_quant ? 4 : 0;
+  return Q4_OK;
+}
+
+int q4_quantize_workspace_size(int32_t qtype, int64_t n, int32_t blocksize, int32_t double_quant,
+                               size_t *bytes) {
+  size_t sz[6];
+  const int rc = q4_state_sizes(qtype, n, blocksize, double_quant, sz);
+  if (rc != Q4_OK) return rc;
+  if (!bytes) return Q4_ERR_ARG;
+  *bytes = double_quant ? (size_t)(kMaxRunPartials * 8 + 256) : 0;
+  return Q4_OK;
+}
+
+int q4_quantize(const void *W, int32_t w_dtype, int64_t rows, int64_t cols, int32_t blocksize,
+                int32_t qtype, int32_t double_quant, q4_state *out, void *workspace,
+                size_t workspace_bytes, void *stream) {
+  if (!W || !out || !valid_in_dtype(w_dtype)) return Q4_ERR_ARG;
+  if (rows < 1 || cols < 1) return Q4_ERR_SHAPE;
+  const int64_t n = rows * cols;
+  size_t sz[6];
+  int rc = q4_state_sizes(qtype, n, blocksize, double_quant, sz);
+  if (rc != Q4_OK) return rc;
+  if (!out->packed || !out->absmax || (qtype == Q4_INT4_ASYM && !out->zero)) return Q4_ERR_ARG;
+  if (double_quant && (!out->absmax_q || !out->absmax_scale || !out->absmax_mean)) return Q4_ERR_ARG;
+  if (!aligned16(W) || !aligned16(out->packed) || ((uintptr_t)out->absmax & 3u)) return Q4_ERR_ALIGN;
+  size_t need = 0;
+  q4_quantize_workspace_size(qtype, n, blocksize, double_quant, &need);
+  if (need && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+
+  static Nf4BinTable tab;
+  static bool tab_ok = false;
+  static std::once_flag once;
+  std::call_once(once, [] { tab_ok = build_bin_table(&tab); });
+  if (!tab_ok) return Q4_ERR_ARG;
+
+  out->qtype = qtype;
+  out->src_dtype = w_dtype;
+  out->n = n;
+  out->rows = rows;
+  out->cols = cols;
+  out->blocksize = blocksize;
+  out->double_quant = double_quant;
+  out->dq_group = Q4_DQ_GROUP;
+  out->reserved = 0;
+  if (!double_quant) out->absmax_q = nullptr, out->absmax_scale = nullptr, out->absmax_mean = nullptr;
+  if (qtype != Q4_INT4_ASYM) out->zero = nullptr;
+
+  const int64_t nb = ceil_div(n, blocksize);
+  const int64_t n_chunks = ceil_div(nb, kChunkBlocks);
+  int64_t run = 1;
+  while (ceil_div(n_chunks, run) > kMaxRunPartials) run <<= 1;
+  const int grid = (int)ceil_div(n_chunks, run);
+
+  QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.W = reinterpret_cast<const uint16_t *>(W);
+  p.n = n;
+  p.nb = nb;
+  p.n_chunks = n_chunks;
+  p.run = run;
+  p.packed = out->packed;
+  p.absmax = out->absmax;
+  p.zero = out->zero;
+  if (double_quant) {
+    p.partials = reinterpret_cast<double *>(workspace);
+    p.counter = reinterpret_cast<unsigned *>((char *)workspace + kMaxRunPartials * 8);
+    p.absmax_mean = out->absmax_mean;
+  }
+  p.status = di.status;
+  p.tab = tab;
+  cudaStream_t st = (cudaStream_t)stream;
+  rc = run_quantize(w_dtype, qtype, blocksize, double_quant != 0, p, grid, st);
+  if (rc != Q4_OK) return rc;
+  if (double_quant) rc = run_double_quant(out->absmax, nb, out->absmax_mean, out->absmax_q, out->absmax_scale, st);
+  return rc;
+}
+
+int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream) {
+  int rc = check_state(Wq);
+  if (rc != Q4_OK) return rc;
+  if (!out || !valid_in_dtype(out_dtype)) return Q4_ERR_ARG;
+  if (!aligned16(out)) return Q4_ERR_ALIGN;
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+  DequantParams p;
+  p.packed = Wq->packed;
+  p.absmax = Wq->absmax;
+  p.zero = Wq->zero;
+  p.absmax_q = Wq->absmax_q;
+  p.absmax_scale = Wq->absmax_scale;
+  p.absmax_mean = Wq->absmax_mean;
+  p.n = Wq->n;
+  p.out = out;
+  memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+  const int64_t groups = ceil_div(Wq->n, 16);
+  const int grid = (int)std::min<int64_t>(ceil_div(groups, 256), (int64_t)di.sms * 8);
+  return run_dequantize(Wq->qtype, out_dtype, Wq->blocksize, Wq->double_quant != 0, p, grid,
+                        (cudaStream_t)stream);
+}
+
+int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {
+  if (!bytes || !Wq || count < 1 || count > kMaxGroup) return Q4_ERR_ARG;
+  if (M < 1 || M > 32) return Q4_ERR_SHAPE;
+  size_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    if (!Wq[i]) return Q4_ERR_ARG;
+    if (!valid_bs(Wq[i]->blocksize) || Wq[i]->cols % Wq[i]->blocksize) return Q4_ERR_SHAPE;
+    int64_t t, s;
+    total += gemv_ws_for(Wq[i], M, &t, &s);
+  }
+  *bytes = total;
+  return Q4_OK;
+}
+
+int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
+                    void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+  if (count < 1 || count > kMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
+  if (M < 1 || M > 32) return Q4_ERR_SHAPE;
+  GemvParams p;
+  memset(&p, 0, sizeof(p));
+  p.count = count;
+  p.M = (int)M;
+  p.y_dtype = y_dtype;
+  if (!Wq[0]) return Q4_ERR_ARG;
+  const int bs = Wq[0]->blocksize;
+  const int dq = Wq[0]->double_quant;
+  int64_t units = 0;
+  size_t ws_off = 0;
+  for (int i = 0; i < count; ++i) {
+    const q4_state *s = Wq[i];
+    int rc = check_state(s);
+    if (rc != Q4_OK) return rc;
+    if (s->qtype != Q4_NF4 || s->blocksize != bs || s->double_quant != dq) return Q4_ERR_ARG;
+    if (s->cols % bs || s->rows > INT32_MAX || s->cols > INT32_MAX) return Q4_ERR_SHAPE;
+    if (!A[i] || !Y[i]) return Q4_ERR_ARG;
+    if (!aligned16(A[i])) return Q4_ERR_ALIGN;
+    int64_t n_tiles, n_splits;
+    const size_t need = gemv_ws_for(s, M, &n_tiles, &n_splits);
+    GemvMat &m = p.mat[i];
+    m.packed = s->packed;
+    m.absmax = s->absmax;
+    m.absmax_q = s->absmax_q;
+    m.absmax_scale = s->absmax_scale;
+    m.absmax_mean = s->absmax_mean;
+    m.A = reinterpret_cast<const uint16_t *>(A[i]);
+    m.Y = Y[i];
+    m.N = (int32_t)s->rows;
+    m.K = (int32_t)s->cols;
+    m.n_tiles = (int32_t)n_tiles;
+    m.n_splits = (int32_t)n_splits;
+    m.unit_begin = units;
+    units += n_tiles * n_splits;
+    if (need) {
+      if (!workspace || ws_off + need > workspace_bytes) return Q4_ERR_WORKSPACE;
+      m.acc = reinterpret_cast<float *>((char *)workspace + ws_off);
+      m.cnt = reinterpret_cast<unsigned *>((char *)workspace + ws_off +
+                                           align256((size_t)s->rows * (size_t)M * 4));
+      ws_off += need;
+    }
+  }
+  p.dq = dq;
+  p.total_units = units;
+  memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+  const GemvPlan pl = gemv_plan(M);
+  return run_gemv(a_dtype, pl.nt, pl.r, bs, p, di.sms, (cudaStream_t)stream);
+}
+
+int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
+            int32_t y_dtype, void *workspace, size_t workspace_bytes, void *stream) {
+  const void *a[1] = {A};
+  const q4_state *w[1] = {Wq};
+  void *y[1] = {Y};
+  return q4_gemv_grouped(1, a, w, y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
+}
+
+int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
+                    void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream) {
+  if (count < 1 || count > kMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
+  if (y_dtype != Q4_F32 && y_dtype != a_dtype) return Q4_ERR_ARG;
+  if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;
+  const DeviceInfo di = device_info();
+  static thread_local GemmParams p;  // host staging of the kernel parameters (~5 KB)
+  memset(&p, 0, sizeof(p));
+  int rc = Q4_OK;
+  int64_t tiles = 0;
+  int dq = -1;
+  for (int i = 0; i < count && rc == Q4_OK; ++i) {
+    const q4_state *s = Wq[i];
+    rc = check_state(s);
+    if (rc != Q4_OK) break;
+    if (s->qtype != Q4_NF4 || s->blocksize != 64) { rc = Q4_ERR_ARG; break; }
+    if (dq < 0) dq = s->double_quant;
+    if (s->double_quant != dq) { rc = Q4_ERR_ARG; break; }
+    if (s->cols % 64 || s->rows % 16 || s->rows > INT32_MAX || s->cols > INT32_MAX) { rc = Q4_ERR_SHAPE; break; }
+    if (!A[i] || !Y[i]) { rc = Q4_ERR_ARG; break; }
+    if (!aligned16(A[i]) || !aligned16(Y[i])) { rc = Q4_ERR_ALIGN; break; }
+    if (di.ok != Q4_OK) { rc = di.ok; break; }
+    GemmMat &m = p.mat[i];
+    const CUtensorMapDataType adt = a_dtype == Q4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&m.tmA, adt, A[i], M, s->cols, 2, kGemmBK, kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&m.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1, kGemmBK / 2,
+                  kGemmBN, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+      rc = Q4_ERR_CUDA;
+      break;
+    }
+    m.absmax_q = s->absmax_q;
+    m.absmax_scale = s->absmax_scale;
+    m.absmax_mean = s->absmax_mean;
+    m.absmax = s->absmax;
+    m.Y = Y[i];
+    m.M = (int32_t)M;
+    m.N = (int32_t)s->rows;
+    m.K = (int32_t)s->cols;
+    m.tiles_m = (int32_t)ceil_div(M, kGemmBM);
+    m.tiles_n = (int32_t)ceil_div(s->rows, kGemmBN);
+    m.tile_begin = tiles;
+    tiles += (int64_t)m.tiles_m * m.tiles_n;
+  }
+  if (rc == Q4_OK) {
+    p.count = count;
+    p.y_dtype = y_dtype;
+    p.dq = dq;
+    p.total_tiles = tiles;
+    p.status = di.status;
+    memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+    rc = run_gemm(a_dtype, p, di.sms, (cudaStream_t)stream);
+  }
+  return rc;
+}
+
+int q4_gemm(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
+            int32_t y_dtype, void *stream) {
+  const void *a[1] = {A};
+  const q4_state *w[1] = {Wq};
+  void *y[1] = {Y};
+  return q4_gemm_grouped(1, a, w, y, M, a_dtype, y_dtype, stream);
+}
+
+int q4_device_status(int32_t *status) {
+  if (!status) return Q4_ERR_ARG;
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+  int v = 0;
+  if (cudaMemcpy(&v, di.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return Q4_ERR_CUDA;
+  *status = v;
+  return Q4_OK;
+}
+
+int q4_clear_device_status(void) {
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+  if (cudaMemset(di.status, 0, sizeof(int)) != cudaSuccess) return Q4_ERR_CUDA;
+  return Q4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// q4_common.cuh -- shared device helpers for the sm_100a kernels of libq4.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/q4.h"
+
+namespace q4 {
+
+// Sticky status word (Q4_STATUS_* bits): kernels receive its device address.
+__device__ __forceinline__ void raise_status(int *status, int bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// ---- 16-bit loads/conversions ------------------------------------------------
+template <int DT> struct Dt;
+template <> struct Dt<Q4_F16> {
+  using T = __half;
+  using T2 = __half2;
+  static __device__ __forceinline__ float to_f(uint16_t b) {
+    return __half2float(__ushort_as_half(b));
+  }
+  static __device__ __forceinline__ uint16_t from_f(float f) {
+    return __half_as_ushort(__float2half_rn(f));
+  }
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+  }
+};
+template <> struct Dt<Q4_BF16> {
+  using T = __nv_bfloat16;
+  using T2 = __nv_bfloat162;
+  static __device__ __forceinline__ float to_f(uint16_t b) {
+    return __uint_as_float(((uint32_t)b) << 16);
+  }
+  static __device__ __forceinline__ uint16_t from_f(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+  }
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+  }
+};
+
+// Lower / upper 16-bit float of a 32-bit word as binary32.
+template <int DT> __device__ __forceinline__ float lo16(uint32_t w) {
+  return Dt<DT>::to_f((uint16_t)(w & 0xFFFFu));
+}
+template <int DT> __device__ __forceinline__ float hi16(uint32_t w) {
+  return Dt<DT>::to_f((uint16_t)(w >> 16));
+}
+
+// Streaming 128-bit global load that does not allocate in L1.
+__device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint2 ldg_stream_v2(const void *p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
+// Correctly rounded binary32 quotient a / b from y = RN(1/b) with one
+// correction step (Markstein's theorem: q = RN(a*y) is within one ulp of a/b,
+// the residual r = a - b*q is exact under FMA, and RN(q + r*y) = RN(a/b);
+// the residual must not underflow: with the divisor in [2^-90, 2^125] the
+// result is exact whenever |a/b| >= 2^-6 and otherwise stays below 2^-5 in
+// magnitude, which decides every NF4 code and every INT4 rint the same way;
+// callers use __fdiv_rn outside that divisor range).
+__device__ __forceinline__ float div_markstein(float a, float b, float y) {
+  float q = __fmul_rn(a, y);
+  float r = __fmaf_rn(-q, b, a);
+  return __fmaf_rn(r, y, q);
+}
+
+__device__ __forceinline__ bool markstein_ok(float b) {
+  float ab = fabsf(b);
+  return ab >= 8.0779356e-28f /* 2^-90 */ && ab <= 4.2535296e37f /* 2^125 */;
+}
+
+}  // namespace q4

@@ -1,0 +1,21 @@
+// q4_internal.h -- host-side launcher entry points shared by the translation
+// units of libq4.so (not part of the public C ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "q4_common.cuh"
+#include "quantize.cuh"
+#include "dequantize.cuh"
+#include "gemv.cuh"
+#include "gemm.cuh"
+
+namespace q4 {
+int run_quantize(int dt, int qt, int bs, bool dq, const QuantParams &p, int grid, cudaStream_t st);
+int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t *absmax_q,
+                     float *absmax_scale, cudaStream_t st);
+int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int grid,
+                   cudaStream_t st);
+int run_gemv(int da, int nt, int r, int bs, const GemvParams &p, int sms, cudaStream_t st);
+int run_gemm(int da, const GemmParams &p, int sms, cudaStream_t st);
+}  // namespace q4

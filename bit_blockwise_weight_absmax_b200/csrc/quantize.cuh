@@ -1,0 +1,328 @@
+// quantize.cuh -- blockwise 4-bit quantization kernels (sm_100a).
+//
+// Defines (learn.pranaymahendrakar.com, "Loading a model in 4-bit", section
+// "Block-wise quantisation, stated exactly"): contiguous blocks of B over the
+// flattened row-major weights; per block c = max|w|; every weight is divided
+// by c and mapped to the nearest of the 16 levels (NF4 levels from n4n.ai,
+// "What is 4-bit quantization and why does it matter?", code block
+// "Conceptual NF4 dequantization"); two codes per byte, low nibble first.
+// INT4 symmetric (n4n.ai "INT4 symmetric": -8..7, s = max|w|/7) and INT4
+// asymmetric (robotsatlas.com "INT4", "How it works"/"Components": [0,15]
+// with an integer zero-point) share the kernel.  Double quantization of the
+// absmax ("blocks of 256, to 8 bits") is a second kernel.
+//
+// Design: one streaming pass over W.  A thread owns 8 consecutive elements
+// (one 128-bit load); B/8 adjacent lanes own one block and reduce its absmax
+// with xor shuffles.  A CTA (256 threads) walks 256-block chunks (the
+// double-quant groups); each CTA owns a contiguous, power-of-two-aligned run
+// of chunks so that the fp64 pairwise sum of the block absmax values used for
+// the double-quant mean is formed in the exact order of the definition (an
+// aligned binary tree) without atomics: lanes -> chunk (shared memory tree)
+// -> CTA run (streaming pairwise stack) -> the last CTA to finish combines the
+// per-CTA partial sums and writes the mean.
+#pragma once
+#include "q4_common.cuh"
+
+namespace q4 {
+
+constexpr int kQThreads = 256;
+constexpr int kChunkBlocks = Q4_DQ_GROUP;  // 256 blocks per chunk
+constexpr int kMaxRunPartials = 2048;      // per-CTA partial sums combined by the last CTA
+
+// NF4 coding table: x (the exact binary32 quotient w / c) falls in bin
+// j = round(15 x) + 15 computed as the low 5 bits of fmaf(x, 15, 2^23*1.5 + 15);
+// each bin holds at most one decision threshold t, so
+// code = base[j] + (x >= thr[j]) with thr = +inf for bins without one.
+struct Nf4BinTable {
+  float thr[32];
+  int base[32];
+};
+
+__device__ __forceinline__ uint32_t nf4_bin(float x) {
+  return __float_as_uint(__fmaf_rn(x, 15.0f, 12582927.0f)) & 31u;
+}
+
+struct QuantParams {
+  const uint16_t *W;
+  int64_t n, nb;
+  int64_t n_chunks;       // ceil(nb / 256)
+  int64_t run;            // chunks per CTA (power of two)
+  uint8_t *packed;
+  float *absmax;
+  uint8_t *zero;
+  double *partials;       // [gridDim.x] fp64 pairwise sums (double quant)
+  unsigned *counter;      // arrival counter (double quant), left at 0
+  float *absmax_mean;     // mean output (double quant)
+  int *status;            // sticky status word
+  Nf4BinTable tab;
+};
+
+// Absolute value of eight 16-bit floats as a max over (bits & 0x7fff): the
+// order of magnitudes of IEEE 16-bit floats is the integer order of these
+// patterns, and NaN / Inf sort above every finite value.
+__device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
+  uint32_t a = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+  uint32_t b = __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu);
+  uint32_t m = __vmaxu2(a, b);
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+template <int DT, int QT, int B, bool DQ>
+__global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
+  constexpr int LPB = B / 8;                     // lanes per block
+  constexpr int ELEMS_IT = kQThreads * 8;        // elements per CTA iteration
+  constexpr int IT_PER_CHUNK = kChunkBlocks * B / ELEMS_IT;  // = B / 8
+  constexpr int BLK_IT = ELEMS_IT / B;           // blocks per CTA iteration
+  constexpr int BATCH = IT_PER_CHUNK < 8 ? IT_PER_CHUNK : 8;
+
+  __shared__ float2 s_tab[32 * 32];              // lane-private copies of the bin table
+  __shared__ double s_blk[kChunkBlocks];         // block absmax of the current chunk
+  __shared__ uint8_t s_zero[BLK_IT];             // INT4_ASYM zero-points of one iteration
+  __shared__ double s_stack[24];                 // streaming pairwise stack (thread 0)
+  __shared__ int s_last;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  if (QT == Q4_NF4) {
+    for (int i = tid; i < 32 * 32; i += kQThreads) {
+      int e = i >> 5;
+      s_tab[i] = make_float2(p.tab.thr[e], __int_as_float(p.tab.base[e]));
+    }
+  }
+  __syncthreads();
+
+  int nonfinite = 0;
+  int depth = 0;  // stack depth (thread 0)
+  const int64_t c0 = (int64_t)blockIdx.x * p.run;
+  const int64_t c1 = min(c0 + p.run, p.n_chunks);
+
+  for (int64_t chunk = c0; chunk < c1; ++chunk) {
+    const int64_t chunk_e0 = chunk * (int64_t)kChunkBlocks * B;
+    for (int it0 = 0; it0 < IT_PER_CHUNK; it0 += BATCH) {
+      uint4 v[BATCH];
+#pragma unroll
+      for (int b = 0; b < BATCH; ++b) {
+        const int64_t e0 = chunk_e0 + (int64_t)(it0 + b) * ELEMS_IT + tid * 8;
+        if (e0 + 8 <= p.n) {
+          v[b] = ldg_stream_v4(p.W + e0);
+        } else {
+          uint16_t t[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) t[j] = (e0 + j < p.n) ? p.W[e0 + j] : (uint16_t)0;
+          v[b] = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
+                            t[6] | (t[7] << 16));
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < BATCH; ++b) {
+        const int it = it0 + b;
+        const int64_t e0 = chunk_e0 + (int64_t)it * ELEMS_IT + tid * 8;
+        const int64_t blk = e0 / B;
+        const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+        float f[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          f[2 * j] = lo16<DT>(w[j]);
+          f[2 * j + 1] = hi16<DT>(w[j]);
+        }
+        uint32_t codes = 0;
+        float scale;
+        if (QT == Q4_NF4 || QT == Q4_INT4_SYM) {
+          uint32_t m = absmax_bits8(v[b]);
+#pragma unroll
+          for (int o = LPB / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+          const float c = Dt<DT>::to_f((uint16_t)m);
+          if (!(c <= 3.4028235e38f)) nonfinite = 1;
+          if (QT == Q4_NF4) {
+            scale = c;
+            const bool fast = markstein_ok(c);
+            const float y = fast ? __frcp_rn(c) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float x = fast ? div_markstein(f[j], c, y) : (c == 0.0f ? 0.0f : __fdiv_rn(f[j], c));
+              const float2 e = s_tab[nf4_bin(x) * 32 + lane];
+              const int code = __float_as_int(e.y) + (x >= e.x ? 1 : 0);
+              codes |= (uint32_t)code << (4 * j);
+            }
+          } else {
+            const float s = __fdiv_rn(c, 7.0f);
+            scale = s;
+            const bool fast = markstein_ok(s);
+            const float y = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              int q = 0;
+              if (s != 0.0f) {
+                float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
+                q = min(max(__float2int_rn(x), -8), 7);
+              }
+              codes |= (uint32_t)(q & 15) << (4 * j);
+            }
+          }
+        } else {  // Q4_INT4_ASYM
+          float mn = 0.0f, mx = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            mn = fminf(mn, f[j]);
+            mx = fmaxf(mx, f[j]);
+          }
+          uint32_t m = absmax_bits8(v[b]);
+#pragma unroll
+          for (int o = LPB / 2; o >= 1; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+          }
+          if (!(Dt<DT>::to_f((uint16_t)m) <= 3.4028235e38f)) nonfinite = 1;
+          const float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+          scale = s;
+          int z = 0;
+          if (s != 0.0f) z = min(max(__float2int_rn(__fdiv_rn(-mn, s)), 0), 15);
+          const bool fast = markstein_ok(s);
+          const float y = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            int q = 0;
+            if (s != 0.0f) {
+              float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
+              q = min(max(__float2int_rn(x) + z, 0), 15);
+            }
+            codes |= (uint32_t)q << (4 * j);
+          }
+          if ((tid % LPB) == 0) s_zero[(tid * 8) / B] = (uint8_t)z;
+        }
+        // ---- stores
+        if (e0 + 8 <= p.n) {
+          *reinterpret_cast<uint32_t *>(p.packed + e0 / 2) = codes;
+        } else if (e0 < p.n) {
+          const int valid = (int)(p.n - e0);
+          for (int j = 0; j < 4; ++j) {
+            if (2 * j < valid) {
+              uint32_t byte = (codes >> (8 * j)) & 0xFFu;
+              if (2 * j + 1 >= valid) byte &= 0x0Fu;  // odd n: high nibble is padding
+              p.packed[e0 / 2 + j] = (uint8_t)byte;
+            }
+          }
+        }
+        if ((tid % LPB) == 0) {
+          if (blk < p.nb) p.absmax[blk] = scale;
+          if (DQ) s_blk[it * BLK_IT + (tid * 8) / B] = (blk < p.nb) ? (double)scale : 0.0;
+        }
+        if (QT == Q4_INT4_ASYM) {
+          __syncthreads();
+          if (tid < BLK_IT / 2) {
+            const int64_t b0 = (chunk_e0 + (int64_t)it * ELEMS_IT) / B + 2 * tid;
+            if (b0 < p.nb) p.zero[b0 / 2] = (uint8_t)(s_zero[2 * tid] | (s_zero[2 * tid + 1] << 4));
+          }
+          __syncthreads();
+        }
+      }
+    }
+    if (DQ) {
+      // Pairwise fp64 sum of the chunk's 256 block values in tree order:
+      // lane l reduces blocks 8l..8l+7 as ((0+1)+(2+3))+((4+5)+(6+7)), then
+      // xor shuffles at distance 1, 2, 4, 8, 16 pair adjacent subtrees.
+      __syncthreads();
+      if (tid < 32) {
+        const double *q = s_blk + 8 * tid;
+        double s = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) s = s + __shfl_xor_sync(0xffffffffu, s, o);
+        if (tid == 0) {
+          // streaming pairwise stack over the CTA's run of chunks: merging
+          // equal-size neighbours reproduces the aligned binary tree
+          s_stack[depth++] = s;
+          for (int64_t k = chunk - c0 + 1; (k & 1) == 0; k >>= 1) {
+            s_stack[depth - 2] = s_stack[depth - 2] + s_stack[depth - 1];
+            --depth;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  if (nonfinite) raise_status(p.status, Q4_STATUS_NONFINITE);
+
+  if (DQ) {
+    if (tid == 0) {
+      // pad the run with zero chunks up to its power-of-two length
+      for (int64_t k = c1 - c0; k < p.run; ++k) {
+        s_stack[depth++] = 0.0;
+        for (int64_t kk = k + 1; (kk & 1) == 0; kk >>= 1) {
+          s_stack[depth - 2] = s_stack[depth - 2] + s_stack[depth - 1];
+          --depth;
+        }
+      }
+      p.partials[blockIdx.x] = (c1 > c0 || p.run > 0) ? s_stack[0] : 0.0;
+      __threadfence();
+      const unsigned ticket = atomicAdd(p.counter, 1u);
+      s_last = (ticket == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (s_last) {
+      // the last CTA: pairwise tree over the per-CTA partials (aligned
+      // subtrees of `run` chunks), level by level, odd last carried up
+      __threadfence();
+      __shared__ double s_red[kMaxRunPartials];
+      int len = gridDim.x;
+      for (int i = tid; i < len; i += kQThreads) s_red[i] = __ldcg(p.partials + i);
+      __syncthreads();
+      while (len > 1) {
+        const int half = len >> 1;
+        double t[kMaxRunPartials / kQThreads / 2 + 1];
+        int cnt = 0;
+        for (int i = tid; i < half; i += kQThreads) t[cnt++] = s_red[2 * i] + s_red[2 * i + 1];
+        double carry = s_red[len - 1];
+        __syncthreads();
+        cnt = 0;
+        for (int i = tid; i < half; i += kQThreads) s_red[i] = t[cnt++];
+        if ((len & 1) && tid == 0) s_red[half] = carry;
+        __syncthreads();
+        len = half + (len & 1);
+      }
+      if (tid == 0) {
+        const double S = s_red[0];
+        p.absmax_mean[0] = __double2float_rn(__ddiv_rn(S, (double)p.nb));
+        *p.counter = 0u;  // leave the workspace zeroed for the next call
+      }
+    }
+  }
+}
+
+// Second-level quantization of the block absmax, one warp per group of 256:
+// m2 = max|c - mu|, s2 = m2 / 127, q2 = clamp(rint((c - mu) / s2), -128, 127).
+static __global__ void __launch_bounds__(256) double_quant_kernel(const float *__restrict__ absmax,
+                                                           int64_t nb,
+                                                           const float *__restrict__ mean,
+                                                           int8_t *__restrict__ absmax_q,
+                                                           float *__restrict__ absmax_scale) {
+  const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int64_t ng = (nb + Q4_DQ_GROUP - 1) / Q4_DQ_GROUP;
+  if (g >= ng) return;
+  const float mu = __ldg(mean);
+  float d[8];
+  float m2 = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t b = g * Q4_DQ_GROUP + lane * 8 + j;
+    d[j] = (b < nb) ? __fsub_rn(__ldg(absmax + b), mu) : 0.0f;
+    if (b < nb) m2 = fmaxf(m2, fabsf(d[j]));
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+  const float s2 = __fdiv_rn(m2, 127.0f);
+  if (lane == 0) absmax_scale[g] = s2;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t b = g * Q4_DQ_GROUP + lane * 8 + j;
+    if (b < nb) {
+      int q2 = 0;
+      if (s2 != 0.0f) q2 = min(max(__float2int_rn(__fdiv_rn(d[j], s2)), -128), 127);
+      absmax_q[b] = (int8_t)q2;
+    }
+  }
+}
+
+}  // namespace q4

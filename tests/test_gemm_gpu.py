@@ -1,0 +1,81 @@
+"""GPU parity of the tcgen05 W4A16 GEMM against the oracle (C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import assert_matmul_close, bits, oracle_state
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q4():
+    from bit_blockwise_weight_absmax_b200 import build
+    build.build()
+    from bit_blockwise_weight_absmax_b200 import q4 as m
+    m.clear_device_status()
+    return m
+
+
+def _case(q4, oracle, M, N, K, a_dtype=torch.bfloat16, dq=True, seed=0, out_dtype=None, rows=None):
+    g = torch.Generator().manual_seed(seed)
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).to(a_dtype)
+    st = q4.quantize(W.cuda(), 64, "nf4", dq)
+    ost = oracle_state(oracle, W, 64, 0, dq)
+    y = q4.gemm(A.cuda(), st, out_dtype)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    if rows is None:
+        ref = oracle.gemv_reference(bits(A), a_dtype == torch.bfloat16, ost, N, K)
+        return y, ref
+    w16 = oracle.dequantize(ost, a_dtype == torch.bfloat16).reshape(N, K)[rows]
+    ref = oracle.matmul(bits(A), a_dtype == torch.bfloat16, w16, a_dtype == torch.bfloat16, M,
+                        len(rows), K)
+    return y[:, torch.from_numpy(rows).cuda()], ref
+
+
+def test_gemm_one_tile(q4, oracle):
+    y, ref = _case(q4, oracle, 256, 256, 64)
+    assert_matmul_close(y, ref)
+
+
+def test_gemm_fp32_out_tight(q4, oracle):
+    """fp32 output: the only difference from the binary64 reference is the
+    fp32 accumulation order, far below the tolerance."""
+    y, ref = _case(q4, oracle, 256, 512, 1024, out_dtype=torch.float32, seed=1)
+    fro, mx = assert_matmul_close(y, ref)
+    assert fro < 1e-5
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 64), (100, 512, 256), (300, 272, 1088),
+                                   (513, 768, 4096)])
+def test_gemm_ragged(q4, oracle, M, N, K):
+    y, ref = _case(q4, oracle, M, N, K, seed=M + N)
+    assert_matmul_close(y, ref)
+
+
+@pytest.mark.parametrize("a_dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("dq", [False, True])
+def test_gemm_dtypes(q4, oracle, a_dtype, dq):
+    y, ref = _case(q4, oracle, 384, 512, 512, a_dtype=a_dtype, dq=dq, seed=3)
+    assert_matmul_close(y, ref)
+
+
+def test_gemm_prefill_7b_layer_m512(q4, oracle):
+    """Prefill config: the 7B layer shapes, NF4 double-quant weights, bf16
+    activations at M = 512, one grouped launch; sampled output columns."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    Ws = wl.layer_weights(wl.LAYER_7B, 0.02, seed=300)
+    sts = [q4.quantize(W.cuda(), 64, "nf4", True) for W in Ws]
+    osts = [oracle_state(oracle, W, 64, 0, True) for W in Ws]
+    rng = np.random.default_rng(1)
+    M = 512
+    As = [wl.activation(M, K, torch.bfloat16, seed=400 + i) for i, (_, N, K) in enumerate(wl.LAYER_7B)]
+    ys = q4.gemm_grouped([a.cuda() for a in As], sts)
+    torch.cuda.synchronize()
+    for (name, N, K), a, y, ost in zip(wl.LAYER_7B, As, ys, osts):
+        rows = np.sort(rng.choice(N, 128, replace=False))
+        w16 = oracle.dequantize(ost, True).reshape(N, K)[rows]
+        ref = oracle.matmul(bits(a), True, w16, True, M, len(rows), K)
+        assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)

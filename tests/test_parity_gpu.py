@@ -1,0 +1,225 @@
+"""GPU parity: quantize / dequantize bit-exact, GEMV within tolerance, against
+the CPU oracle on identical seeded inputs, called through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import (assert_matmul_close, assert_state_equal, bits, is_bf16, oracle_state)
+
+pytestmark = pytest.mark.gpu
+
+QT = {"nf4": 0, "int4_sym": 1, "int4_asym": 2}
+
+
+@pytest.fixture(scope="module")
+def q4():
+    from bit_blockwise_weight_absmax_b200 import build
+    build.build()
+    from bit_blockwise_weight_absmax_b200 import q4 as m
+    assert torch.cuda.is_available()
+    m.clear_device_status()
+    return m
+
+
+def dev(t):
+    return t.to("cuda")
+
+
+# ------------------------------------------------------------- quantize -----
+
+def test_tiny_nf4_config(q4, oracle):
+    """fp16 W[256,512] ~ N(0,0.02), seed 0, NF4 blocksize 64, no double quant;
+    quantize -> pack -> dequantize bit-exact; GEMV with x[512] ~ N(0,1)."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    W = wl.tiny_weight(0)
+    x = wl.tiny_activation(1)
+    st = q4.quantize(dev(W), 64, "nf4", False)
+    ost = oracle_state(oracle, W, 64, 0, False)
+    assert_state_equal(st, ost)
+    d = q4.dequantize(st)
+    assert np.array_equal(bits(d), oracle.dequantize(ost, False))
+    y = q4.gemv(dev(x), st)
+    ref = oracle.gemv_reference(bits(x), False, ost, 256, 512)
+    assert_matmul_close(y, ref)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+
+
+@pytest.mark.parametrize("qtype,bs,dq", [("nf4", 64, True), ("int4_sym", 128, False),
+                                         ("int4_asym", 128, False)])
+def test_scheme_config_4096_outliers(q4, oracle, qtype, bs, dq):
+    """bf16 W[4096,4096] ~ N(0,0.02) with 0.1% x20 outliers; the three schemes."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    W = wl.outlier_weight(4096, 4096, seed=0)
+    st = q4.quantize(dev(W), bs, qtype, dq)
+    ost = oracle_state(oracle, W, bs, QT[qtype], dq)
+    assert_state_equal(st, ost)
+    for out_dt in (torch.bfloat16, torch.float16):
+        d = q4.dequantize(st, out_dt)
+        assert np.array_equal(bits(d), oracle.dequantize(ost, out_dt == torch.bfloat16))
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("qtype", ["nf4", "int4_sym", "int4_asym"])
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+def test_quantize_ragged_shapes(q4, oracle, dtype, qtype, bs):
+    """Several tiles plus ragged tails: n not a multiple of the block or of a
+    256-block chunk, odd n, a single element, and wide-range values."""
+    g = torch.Generator().manual_seed(bs * 7 + QT[qtype])
+    shapes = [(1, 1), (3, 5), (17, 33), (7, 1001), (257, 300), (96, 4096 + 64)]
+    for rows, cols in shapes:
+        W = (torch.randn(rows, cols, generator=g) *
+             torch.exp(torch.randn(rows, cols, generator=g) * 2)).to(dtype)
+        W[0, 0] = 0.0
+        dq = qtype == "nf4"
+        for use_dq in ([False, True] if dq else [False]):
+            st = q4.quantize(dev(W), bs, qtype, use_dq)
+            ost = oracle_state(oracle, W, bs, QT[qtype], use_dq)
+            assert_state_equal(st, ost)
+            d = q4.dequantize(st, dtype)
+            assert np.array_equal(bits(d), oracle.dequantize(ost, is_bf16(W)))
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_nearest_coding_exhaustive_16bit_on_gpu(q4, oracle, dtype):
+    """Every finite 16-bit value w paired with block maxima c from a spread of
+    magnitudes (blocks [w, c] of size 2... as 32-blocks padded with zeros):
+    codes bit-exact with the oracle."""
+    allbits = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(dtype)
+    vals = allbits[torch.isfinite(allbits.float())]
+    for c in [1.0, 0.7, 3.0e-3, 1234.5, 6.0e-5]:
+        cc = torch.tensor(c, dtype=torch.float32).to(dtype)
+        v = vals[vals.float().abs() <= cc.float()]
+        blocks = torch.zeros(v.numel(), 32, dtype=dtype)
+        blocks[:, 0] = v
+        blocks[:, 1] = cc
+        st = q4.quantize(dev(blocks), 32, "nf4", False)
+        ost = oracle_state(oracle, blocks, 32, 0, False)
+        assert_state_equal(st, ost)
+        st = q4.quantize(dev(blocks), 32, "int4_sym", False)
+        assert_state_equal(st, oracle_state(oracle, blocks, 32, 1, False))
+
+
+def test_nonfinite_input_sets_status(q4):
+    W = torch.randn(64, 64).half()
+    W[3, 5] = float("inf")
+    q4.clear_device_status()
+    q4.quantize(dev(W), 64, "nf4", False)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() & 1
+    q4.clear_device_status()
+    assert q4.last_device_status() == 0
+
+
+def test_double_quant_mean_many_chunks(q4, oracle):
+    """More 256-block chunks than one CTA run: the pairwise mean crosses CTAs."""
+    W = torch.randn(4099, 8192, generator=torch.Generator().manual_seed(2)).mul(0.015).bfloat16()
+    st = q4.quantize(dev(W), 64, "nf4", True)
+    assert_state_equal(st, oracle_state(oracle, W, 64, 0, True))
+    st2 = q4.quantize(dev(W), 64, "nf4", True)  # the workspace was left clean
+    assert torch.equal(st.absmax_mean, st2.absmax_mean) and torch.equal(st.absmax_q, st2.absmax_q)
+
+
+def test_host_rejects_bad_arguments(q4):
+    W = dev(torch.randn(64, 64).half())
+    with pytest.raises(q4.Q4Error):
+        q4.quantize(W, 48)
+    with pytest.raises(q4.Q4Error):
+        q4.quantize(W, 64, "int4_sym", True)
+    with pytest.raises(q4.Q4Error):
+        base = dev(torch.randn(64 * 64 + 8).half())
+        q4.quantize(base[1:64 * 64 + 1].view(64, 64), 64)  # not 16-byte aligned
+    st = q4.quantize(W, 64)
+    with pytest.raises(q4.Q4Error):
+        q4.gemv(dev(torch.randn(33, 64).half()), st)    # M > 32
+
+
+# ------------------------------------------------------------------ GEMV -----
+
+def _gemv_case(q4, oracle, N, K, M, a_dtype, dq, bs=64, seed=0, out_dtype=None):
+    g = torch.Generator().manual_seed(seed)
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).to(a_dtype)
+    st = q4.quantize(dev(W), bs, "nf4", dq)
+    ost = oracle_state(oracle, W, bs, 0, dq)
+    y = q4.gemv(dev(A), st, out_dtype)
+    ref = oracle.gemv_reference(bits(A), a_dtype == torch.bfloat16, ost, N, K)
+    return y, ref
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 7, 8, 9, 16, 17, 31, 32])
+def test_gemv_batch_sizes(q4, oracle, M):
+    y, ref = _gemv_case(q4, oracle, 512, 2048 + 64, M, torch.float16, True, seed=M)
+    assert_matmul_close(y, ref)
+
+
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+@pytest.mark.parametrize("a_dtype", [torch.float16, torch.bfloat16])
+def test_gemv_blocksizes_dtypes(q4, oracle, bs, a_dtype):
+    for M in (1, 16):
+        y, ref = _gemv_case(q4, oracle, 272, 3072, M, a_dtype, bs == 64, bs=bs, seed=bs + M)
+        assert_matmul_close(y, ref)
+
+
+def test_gemv_fp32_output_tight(q4, oracle):
+    """fp32 output against the unrounded reference: the fused path's own error
+    (fp16 codebook values, fp32 accumulation) stays far below the tolerance."""
+    y, ref = _gemv_case(q4, oracle, 1024, 4096, 4, torch.float16, True, out_dtype=torch.float32)
+    fro, mx = assert_matmul_close(y, ref)
+    assert fro < 5e-4
+
+
+def test_gemv_exact_small_integers(q4, oracle):
+    """A in {-1,0,1}, power-of-two block maxima, K = 64: the fp32 result is
+    exact, so Y equals the reference exactly."""
+    g = torch.Generator().manual_seed(4)
+    N, K = 64, 64
+    L = torch.tensor(oracle.nf4_levels())
+    codes = torch.randint(0, 16, (N, K), generator=g)
+    scale = 2.0 ** torch.randint(-3, 3, (N, 1), generator=g).float()
+    W = (L[codes] * scale)
+    W[:, 0] = scale[:, 0]  # the block absmax is the power of two
+    W = W.half()
+    A = torch.randint(-1, 2, (3, K), generator=g).half()
+    st = q4.quantize(dev(W), 64, "nf4", False)
+    ost = oracle_state(oracle, W, 64, 0, False)
+    assert_state_equal(st, ost)
+    y = q4.gemv(dev(A), st, torch.float32)
+    ref = oracle.gemv_reference(bits(A), False, ost, N, K)
+    assert np.array_equal(y.cpu().double().numpy(), ref)
+
+
+def test_gemv_grouped_7b_layer(q4, oracle):
+    """Llama-2-7B-shaped decode layer (q/k/v/o 4096x4096, gate/up 11008x4096,
+    down 4096x11008), bf16 weights ~ N(0,0.02) -> NF4 blocksize 64 with double
+    quant, fp16 activations at M = 1, 4, 16, one grouped launch; checked on
+    sampled output rows of every matrix."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    Ws = wl.layer_weights(wl.LAYER_7B, 0.02, seed=100)
+    sts = [q4.quantize(dev(W), 64, "nf4", True) for W in Ws]
+    osts = [oracle_state(oracle, W, 64, 0, True) for W in Ws]
+    for st, ost in zip(sts, osts):
+        assert_state_equal(st, ost)
+    rng = np.random.default_rng(0)
+    for M in (1, 4, 16):
+        As = [wl.activation(M, K, torch.float16, seed=200 + M + i) for i, (_, N, K) in enumerate(wl.LAYER_7B)]
+        ys = q4.gemv_grouped([dev(a) for a in As], sts)
+        for (name, N, K), a, y, ost in zip(wl.LAYER_7B, As, ys, osts):
+            rows = np.sort(rng.choice(N, 384, replace=False))
+            w16 = oracle.dequantize(ost, False).reshape(N, K)[rows]
+            ref = oracle.matmul(bits(a), False, w16, False, M, len(rows), K)
+            assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+
+
+def test_gemv_repeat_calls_agree(q4, oracle):
+    """The split-K workspace is left zeroed: a second call gives the same
+    result (up to the order of the fp32 partial-sum additions)."""
+    g = torch.Generator().manual_seed(6)
+    W = dev(torch.randn(4096, 11008, generator=g).mul(0.02).bfloat16())
+    st = q4.quantize(W, 64, "nf4", True)
+    A = dev(torch.randn(16, 11008, generator=g).half())
+    y1 = q4.gemv(A, st)
+    y2 = q4.gemv(A, st)
+    torch.cuda.synchronize()
+    d = (y1.float() - y2.float()).abs().max().item()
+    assert d <= 1e-3 * y1.float().abs().max().item()
