@@ -188,7 +188,7 @@ def run_gpu(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     shapes = wl.LAYER_7B
     peaks = _peaks()
-    L = N_COPIES
+    L = args.copies
 
     # ---- inputs resident in HBM before timing (seeded, generated on device)
     Ws = [[wl.gaussian((N, K), 0.02, torch.bfloat16, 1000 * l + i + 17 * rank, dev)
@@ -237,6 +237,14 @@ def run_gpu(args, rank, world, local_rank):
     for M in DECODE_M:
         launches[f"gemv_m{M}"] = L
     launches_per_step = sum(launches.values())
+    if args.profile:
+        # a short eager run of one phase for a profiler capture (no timing)
+        for _ in range(1 + args.steps):
+            fns[args.profile]()
+        torch.cuda.synchronize()
+        if rank == 0:
+            print(json.dumps({"profile": args.profile, "launches": launches[args.profile] * (1 + args.steps)}))
+        return
     for f in fns.values():
         f()
     torch.cuda.synchronize()
@@ -401,6 +409,11 @@ def main():
     ap.add_argument("--impl", default="q4", choices=["q4", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", default=None,
+                    help="run one phase eagerly (quantize, gemv_m1, gemv_m4, gemv_m16, dequantize, "
+                         "gemm) --steps+1 times for a profiler capture; prints no metric")
+    ap.add_argument("--copies", type=int, default=N_COPIES,
+                    help="distinct layer copies that rotate through the step")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -119,23 +119,28 @@ __device__ __forceinline__ void store_y(void *Y, int ydt, int64_t idx, float v) 
 
 template <int DA, int NT, int R, int B, int UB, int PF>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(GemvParams p) {
-  constexpr int SPLIT = (DA == Q4_BF16) ? 2 : 1;  // bf16: codebook as hi + lo parts
   constexpr int STEPS = B / 16;                  // MMA k-steps per block
   constexpr int ROWS = 16 * R;                   // rows per unit
-  extern __shared__ uint32_t s_lut[];            // [SPLIT][256][32]
+  extern __shared__ uint32_t s_lut[];            // [256][32] (fp16 pairs or float2)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
 
-  // byte -> (level(lo nibble), level(hi nibble)) as a 16-bit pair
-  for (int i = tid; i < 256 * 32; i += blockDim.x) {
-    const int b = i >> 5;
-    const float l0 = p.levels[b & 15], l1 = p.levels[b >> 4];
-    const uint32_t hi = Dt<DA>::pack2(l0, l1);
-    s_lut[i] = hi;
-    if (SPLIT == 2) {
-      const float r0 = __fsub_rn(l0, lo16<DA>(hi)), r1 = __fsub_rn(l1, hi16<DA>(hi));
-      s_lut[256 * 32 + i] = Dt<DA>::pack2(r0, r1);
+  if constexpr (DA == Q4_BF16) {
+    // bf16 activations: the reference dequantizes to bf16 first, so the MMA
+    // must see the exact w^ = bf16(c~ * level); the LUT holds binary32 level
+    // pairs and the scale is applied per weight before the rounding.
+    float2 *lut2 = reinterpret_cast<float2 *>(s_lut);
+    for (int i = tid; i < 256 * 32; i += blockDim.x) {
+      const int b = i >> 5;
+      lut2[i] = make_float2(p.levels[b & 15], p.levels[b >> 4]);
+    }
+  } else {
+    // fp16 activations: byte -> (level(lo nibble), level(hi nibble)) as an
+    // fp16 pair; the block scale multiplies the fp32 partial afterwards.
+    for (int i = tid; i < 256 * 32; i += blockDim.x) {
+      const int b = i >> 5;
+      s_lut[i] = Dt<DA>::pack2(p.levels[b & 15], p.levels[b >> 4]);
     }
   }
   __syncthreads();
@@ -216,20 +221,39 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(GemvParams p) {
             for (int v = 0; v < B / 8; ++v) act[nt][v] = 0;
           }
         }
-        float part[R][NT][4];
+        if constexpr (DA == Q4_BF16) {
+          const float2 *lut2 = reinterpret_cast<const float2 *>(s_lut) + lane;
 #pragma unroll
-        for (int rt = 0; rt < R; ++rt)
+          for (int s = 0; s < STEPS; ++s) {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
+            for (int rt = 0; rt < R; ++rt) {
+              const float c0 = cur.sc[rt][0], c1 = cur.sc[rt][1];
+              const float2 e0 = lut2[cur.row[rt][0].byte(2 * s) * 32];
+              const float2 e1 = lut2[cur.row[rt][1].byte(2 * s) * 32];
+              const float2 e2 = lut2[cur.row[rt][0].byte(2 * s + 1) * 32];
+              const float2 e3 = lut2[cur.row[rt][1].byte(2 * s + 1) * 32];
+              uint32_t a[4];
+              a[0] = Dt<DA>::pack2(__fmul_rn(c0, e0.x), __fmul_rn(c0, e0.y));
+              a[1] = Dt<DA>::pack2(__fmul_rn(c1, e1.x), __fmul_rn(c1, e1.y));
+              a[2] = Dt<DA>::pack2(__fmul_rn(c0, e2.x), __fmul_rn(c0, e2.y));
+              a[3] = Dt<DA>::pack2(__fmul_rn(c1, e3.x), __fmul_rn(c1, e3.y));
 #pragma unroll
-            for (int j = 0; j < 4; ++j) part[rt][nt][j] = 0.0f;
+              for (int nt = 0; nt < NT; ++nt) Mma<DA>::run(acc[rt][nt], a, act[nt][2 * s], act[nt][2 * s + 1]);
+            }
+          }
+        } else {
+          float part[R][NT][4];
 #pragma unroll
-        for (int s = 0; s < STEPS; ++s) {
+          for (int rt = 0; rt < R; ++rt)
 #pragma unroll
-          for (int rt = 0; rt < R; ++rt) {
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int sp = 0; sp < SPLIT; ++sp) {
-              const uint32_t *lut = s_lut + sp * 256 * 32 + lane;
+              for (int j = 0; j < 4; ++j) part[rt][nt][j] = 0.0f;
+#pragma unroll
+          for (int s = 0; s < STEPS; ++s) {
+#pragma unroll
+            for (int rt = 0; rt < R; ++rt) {
+              const uint32_t *lut = s_lut + lane;
               uint32_t a[4];
               a[0] = lut[cur.row[rt][0].byte(2 * s) * 32];
               a[1] = lut[cur.row[rt][1].byte(2 * s) * 32];
@@ -239,16 +263,16 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(GemvParams p) {
               for (int nt = 0; nt < NT; ++nt) Mma<DA>::run(part[rt][nt], a, act[nt][2 * s], act[nt][2 * s + 1]);
             }
           }
+#pragma unroll
+          for (int rt = 0; rt < R; ++rt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              acc[rt][nt][0] = fmaf(cur.sc[rt][0], part[rt][nt][0], acc[rt][nt][0]);
+              acc[rt][nt][1] = fmaf(cur.sc[rt][0], part[rt][nt][1], acc[rt][nt][1]);
+              acc[rt][nt][2] = fmaf(cur.sc[rt][1], part[rt][nt][2], acc[rt][nt][2]);
+              acc[rt][nt][3] = fmaf(cur.sc[rt][1], part[rt][nt][3], acc[rt][nt][3]);
+            }
         }
-#pragma unroll
-        for (int rt = 0; rt < R; ++rt)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[rt][nt][0] = fmaf(cur.sc[rt][0], part[rt][nt][0], acc[rt][nt][0]);
-            acc[rt][nt][1] = fmaf(cur.sc[rt][0], part[rt][nt][1], acc[rt][nt][1]);
-            acc[rt][nt][2] = fmaf(cur.sc[rt][1], part[rt][nt][2], acc[rt][nt][2]);
-            acc[rt][nt][3] = fmaf(cur.sc[rt][1], part[rt][nt][3], acc[rt][nt][3]);
-          }
       }
     }
 

@@ -12,7 +12,7 @@ int go(const GemvParams &p, int sms, cudaStream_t st) {
   constexpr int UB = kUnitK / B;
   constexpr int PF = (R == 1) ? (UB < 8 ? UB : 8) : (UB < 4 ? UB : 4);
   auto kern = gemv_kernel<DA, NT, R, B, UB, PF>;
-  const int smem = 256 * 32 * 4 * (DA == Q4_BF16 ? 2 : 1);
+  const int smem = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
   static int occ = 0;
   if (occ == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
