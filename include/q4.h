@@ -154,6 +154,34 @@ Q4_API int q4_quantize(const void *W, int32_t w_dtype, int64_t rows, int64_t col
                 int32_t qtype, int32_t double_quant, q4_state *out, void *workspace,
                 size_t workspace_bytes, void *stream);
 
+/*
+ * q4_quantize_noalloc -- q4_quantize for callers that cannot allocate device
+ * memory when they quantize (a plugin whose host application owns every
+ * device allocation, a latency-critical path that must not pay for the
+ * device-wide synchronization of cudaMalloc/cudaFree, a runtime that reserves
+ * all memory at start-up).  It takes the same arguments as q4_quantize minus
+ * the workspace: the caller still passes W and the output state buffers.
+ * The pages have no counterpart to this call; it exists only for those
+ * callers.
+ *   Scratch: a fixed array of Q4_NOALLOC_SCRATCH_BYTES in the library's own
+ *   static device memory, held by every GPU that loads the library until the
+ *   process exits.  Its device address is looked up on the first call on
+ *   each device (with that device current); make that first call before any
+ *   stream capture.  Each call clears the part it uses with an asynchronous
+ *   memset on `stream`, and no call allocates or frees device memory.
+ *   All calls on a device share the array and it keeps the last call's
+ *   contents: calls that overlap on the GPU (different streams, or the same
+ *   call from several threads at once) race on it and must be serialized by
+ *   the caller.
+ *   Limit: returns Q4_ERR_WORKSPACE if the workspace q4_quantize would need
+ *   (q4_quantize_workspace_size) exceeds Q4_NOALLOC_SCRATCH_BYTES; every
+ *   other error is that of q4_quantize.
+ */
+#define Q4_NOALLOC_SCRATCH_BYTES 32768
+Q4_API int q4_quantize_noalloc(const void *W, int32_t w_dtype, int64_t rows, int64_t cols,
+                               int32_t blocksize, int32_t qtype, int32_t double_quant,
+                               q4_state *out, void *stream);
+
 /* ---- dequantize ------------------------------------------------------- */
 
 /*
