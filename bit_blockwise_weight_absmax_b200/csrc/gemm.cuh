@@ -96,8 +96,10 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 // Bounded wait: gives up after ~2 s, raises Q4_STATUS_TIMEOUT and sets *abort.
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *status, volatile int *abort) {
-  if (mbar_try(bar, parity)) return true;
+// The first probe is inlined; only a phase that is not yet complete pays the
+// call into the polling loop.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, int *status,
+                                                   volatile int *abort) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try(bar, parity)) return true;
@@ -108,6 +110,23 @@ static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *status, volatile int *abort) {
+  if (mbar_try(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, status, abort);
+}
+
+// Wait by a whole warp: only lane 0 polls the barrier (many polling lanes
+// would queue their try_waits ahead of the single-thread producers), then
+// the result is broadcast.  Must be called by all 32 lanes.
+// After lane 0 has seen the phase complete, each other lane queries it once
+// (returns at once) so that it acquires the data the phase published itself.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int *status, volatile int *abort) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok && (threadIdx.x & 31) != 0) (void)mbar_try(bar, parity);
+  return ok;
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y) {
@@ -320,7 +339,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const uint32_t use = it / kGemmStages;
         const float sc = sc_next;
         sc_next = scale_of(kb + 1);
-        if (!mbar_wait(full_bar(s), use & 1, p.status, abort)) {
+        if (!mbar_wait_warp(full_bar(s), use & 1, p.status, abort)) {
           ok = false;
           break;
         }
@@ -346,7 +365,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       }
       if (!ok) break;
       // ---- epilogue
-      if (!mbar_wait(accfull_bar, tcount & 1, p.status, abort)) break;
+      if (!mbar_wait_warp(accfull_bar, tcount & 1, p.status, abort)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {

@@ -1,52 +1,103 @@
-// k_gemv.cu -- launchers of the fused dequant-GEMV kernel.
+// k_gemv.cu -- launchers of the tcgen05 fused dequant-GEMV kernel.
 #include <algorithm>
 
 #include "q4_internal.h"
 
 namespace q4 {
 namespace {
-constexpr int kUnitK = 1024;  // k per work unit (must match the host plan)
 
-template <int DA, int NT, int R, int B>
-int go(const GemvParams &p, int sms, cudaStream_t st) {
-  constexpr int UB = kUnitK / B;
-  constexpr int PF = (R == 1) ? (UB < 8 ? UB : 8) : (UB < 4 ? UB : 4);
-  auto kern = gemv_kernel<DA, NT, R, B, UB, PF>;
-  const int smem = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
-  static int occ = 0;
-  if (occ == 0) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+template <int DA, int B, int MP>
+int go(const GvParams &p, int sms, cudaStream_t st) {
+  constexpr int NB = MP <= 16 ? 16 : 32;
+  constexpr int STAGE = NB * kGvStageK * 2 + kGvWTile;
+  constexpr int S = (DA == Q4_BF16) ? 4 : (NB == 16 ? 8 : 6);
+  constexpr int LUTB = (DA == Q4_BF16) ? 256 * 32 * 8 : 256 * 32 * 4;
+  constexpr int SCALES = 2 * kGvRows * (kGvUnitK / B + 1) * 4;
+  constexpr int SMEM = S * STAGE + LUTB + SCALES + 3 * S * 8 + 128 + 1024;
+  auto kern = gemv_tc_kernel<DA, B, MP, NB, S>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return Q4_ERR_CUDA;
-    int o = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kGemvWarps * 32, smem) != cudaSuccess || o < 1)
-      return Q4_ERR_CUDA;
-    occ = o;
+    attr = true;
   }
-  const int64_t want = (p.total_units + kGemvWarps - 1) / kGemvWarps;
-  const int grid = (int)std::min<int64_t>(want, (int64_t)sms * occ);
-  kern<<<grid, kGemvWarps * 32, smem, st>>>(p);
+  // CTAs per SM: two when their shared memory fits (228 KB per SM, 1 KB
+  // reserved per CTA) and the kernel was compiled for two (registers); their
+  // 2 x 256 tensor-memory columns always fit.
+  constexpr int OCC = (MP < 32 && 2 * (SMEM + 1024) <= 228 * 1024) ? 2 : 1;
+  const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * OCC);
+  kern<<<grid, kGvThreads, SMEM, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+template <int DA, int B>
+int by_mp(int mp, const GvParams &p, int sms, cudaStream_t st) {
+  switch (mp) {
+    case 1: return go<DA, B, 1>(p, sms, st);
+    case 2: return go<DA, B, 2>(p, sms, st);
+    case 4: return go<DA, B, 4>(p, sms, st);
+    case 8: return go<DA, B, 8>(p, sms, st);
+    case 16: return go<DA, B, 16>(p, sms, st);
+    case 32: return go<DA, B, 32>(p, sms, st);
+  }
+  return Q4_ERR_ARG;
+}
+
+template <int DA>
+int by_bs(int bs, int mp, const GvParams &p, int sms, cudaStream_t st) {
+  switch (bs) {
+    case 32: return by_mp<DA, 32>(mp, p, sms, st);
+    case 64: return by_mp<DA, 64>(mp, p, sms, st);
+    case 128: return by_mp<DA, 128>(mp, p, sms, st);
+    case 256: return by_mp<DA, 256>(mp, p, sms, st);
+  }
+  return Q4_ERR_ARG;
+}
+template <int DA, int NT, int R, int B>
+int go_small(const GsParams &p, int sms, cudaStream_t st) {
+  constexpr int UB = kGsUnitK / B;
+  // prefetch depth: about 40 bytes per lane and row in flight (R == 1), 32 (R == 2)
+  constexpr int PF0 = ((R == 1) ? 40 : 32) / (B / 8);
+  constexpr int PF = PF0 < 1 ? 1 : (UB < PF0 ? UB : PF0);
+  auto kern = gemv_small_kernel<DA, NT, R, B, PF>;
+  constexpr int SMEM = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return Q4_ERR_CUDA;
+    attr = true;
+  }
+  const int64_t want = (p.total_units + kGsWarps - 1) / kGsWarps;
+  const int grid = (int)std::min<int64_t>(want, (int64_t)sms * (R == 1 ? 3 : 2));
+  kern<<<grid, kGsWarps * 32, SMEM, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 template <int DA, int NT, int R>
-int by_bs(int bs, const GemvParams &p, int sms, cudaStream_t st) {
+int small_bs(int bs, const GsParams &p, int sms, cudaStream_t st) {
   switch (bs) {
-    case 32: return go<DA, NT, R, 32>(p, sms, st);
-    case 64: return go<DA, NT, R, 64>(p, sms, st);
-    case 128: return go<DA, NT, R, 128>(p, sms, st);
-    case 256: return go<DA, NT, R, 256>(p, sms, st);
+    case 32: return go_small<DA, NT, R, 32>(p, sms, st);
+    case 64: return go_small<DA, NT, R, 64>(p, sms, st);
+    case 128: return go_small<DA, NT, R, 128>(p, sms, st);
+    case 256: return go_small<DA, NT, R, 256>(p, sms, st);
   }
   return Q4_ERR_ARG;
 }
 template <int DA>
-int by_plan(int nt, int r, int bs, const GemvParams &p, int sms, cudaStream_t st) {
-  if (nt == 1 && r == 1) return by_bs<DA, 1, 1>(bs, p, sms, st);
-  if (nt == 2 && r == 2) return by_bs<DA, 2, 2>(bs, p, sms, st);
-  if (nt == 4 && r == 2) return by_bs<DA, 4, 2>(bs, p, sms, st);
-  return Q4_ERR_ARG;
+int small_m(int M, int bs, const GsParams &p, int sms, cudaStream_t st) {
+  if (M <= 8) return small_bs<DA, 1, 1>(bs, p, sms, st);
+  return small_bs<DA, 2, 2>(bs, p, sms, st);
 }
 }  // namespace
 
-int run_gemv(int da, int nt, int r, int bs, const GemvParams &p, int sms, cudaStream_t st) {
-  return da == Q4_F16 ? by_plan<Q4_F16>(nt, r, bs, p, sms, st) : by_plan<Q4_BF16>(nt, r, bs, p, sms, st);
+int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st) {
+  return da == Q4_F16 ? small_m<Q4_F16>(M, bs, p, sms, st) : small_m<Q4_BF16>(M, bs, p, sms, st);
+}
+
+int run_gemv(int da, int bs, int mp, const GvParams &p, int sms, cudaStream_t st) {
+  return da == Q4_F16 ? by_bs<Q4_F16>(bs, mp, p, sms, st) : by_bs<Q4_BF16>(bs, mp, p, sms, st);
 }
 }  // namespace q4

@@ -134,22 +134,23 @@ int check_state(const q4_state *s) {
   return Q4_OK;
 }
 
-// ---- GEMV planning: rows per unit (16 * r), n8 tiles, k per unit ---------------
-constexpr int kGemvUnitK = 1024;
-struct GemvPlan {
-  int nt, r;
-};
-GemvPlan gemv_plan(int64_t M) {
-  if (M <= 8) return {1, 1};
-  if (M <= 16) return {2, 2};
-  return {4, 2};
-}
+// ---- GEMV planning ----------------------------------------------------------
+// M <= 16: warp units of 16 R rows x 1024 k (mma.sync kernel); M > 16: CTA
+// units of 128 rows x 1024 k (tcgen05 kernel).  Workspace: two work counters,
+// then per split matrix fp32 [N][M] partial sums and per-tile counters.
+constexpr size_t kGemvWsHead = 256;
+int gemv_small_rows(int64_t M) { return M <= 8 ? 16 : 32; }
 size_t gemv_ws_for(const q4_state *s, int64_t M, int64_t *n_tiles, int64_t *n_splits) {
-  const GemvPlan pl = gemv_plan(M);
-  *n_tiles = ceil_div(s->rows, 16 * pl.r);
-  *n_splits = ceil_div(s->cols / s->blocksize, kGemvUnitK / s->blocksize);
+  const int64_t rows = M <= 16 ? gemv_small_rows(M) : kGvRows;
+  *n_tiles = ceil_div(s->rows, rows);
+  *n_splits = ceil_div(s->cols, M <= 16 ? kGsUnitK : kGvUnitK);
   if (*n_splits <= 1) return 0;
   return align256((size_t)s->rows * (size_t)M * 4) + align256((size_t)*n_tiles * 4);
+}
+int pow2_at_least(int64_t m) {
+  int p = 1;
+  while (p < m) p <<= 1;
+  return p;
 }
 
 // ---- TMA descriptors ----------------------------------------------------------------
@@ -182,6 +183,62 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The decode-batch path (M <= 16): the mma.sync kernel of gemv_small.cuh.
+int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *const *Wq, void *const *Y,
+                       int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  static thread_local GsParams p;
+  memset(&p, 0, sizeof(p));
+  p.count = count;
+  p.M = (int)M;
+  p.y_dtype = y_dtype;
+  const int bs = Wq[0]->blocksize;
+  const int dq = Wq[0]->double_quant;
+  const DeviceInfo di = device_info();
+  if (!workspace || workspace_bytes < kGemvWsHead) return Q4_ERR_WORKSPACE;
+  int64_t units = 0;
+  size_t ws_off = kGemvWsHead;
+  for (int i = 0; i < count; ++i) {
+    const q4_state *s = Wq[i];
+    int rc = check_state(s);
+    if (rc != Q4_OK) return rc;
+    if (s->qtype != Q4_NF4 || s->blocksize != bs || s->double_quant != dq) return Q4_ERR_ARG;
+    if (s->cols % bs || s->rows > INT32_MAX || s->cols > INT32_MAX) return Q4_ERR_SHAPE;
+    if (!A[i] || !Y[i]) return Q4_ERR_ARG;
+    if (!aligned16(A[i])) return Q4_ERR_ALIGN;
+    if (di.ok != Q4_OK) return di.ok;
+    int64_t n_tiles, n_splits;
+    const size_t need = gemv_ws_for(s, M, &n_tiles, &n_splits);
+    GsMat &m = p.mat[i];
+    m.packed = s->packed;
+    m.absmax = s->absmax;
+    m.absmax_q = s->absmax_q;
+    m.absmax_scale = s->absmax_scale;
+    m.absmax_mean = s->absmax_mean;
+    m.A = reinterpret_cast<const uint16_t *>(A[i]);
+    m.Y = Y[i];
+    m.N = (int32_t)s->rows;
+    m.K = (int32_t)s->cols;
+    m.n_tiles = (int32_t)n_tiles;
+    m.n_splits = (int32_t)n_splits;
+    m.unit_begin = units;
+    units += n_tiles * n_splits;
+    if (need) {
+      if (ws_off + need > workspace_bytes) return Q4_ERR_WORKSPACE;
+      m.acc = reinterpret_cast<float *>((char *)workspace + ws_off);
+      m.cnt = reinterpret_cast<unsigned *>((char *)workspace + ws_off +
+                                           align256((size_t)s->rows * (size_t)M * 4));
+      ws_off += need;
+    }
+  }
+  if (units > UINT32_MAX / 2) return Q4_ERR_SHAPE;
+  p.dq = dq;
+  p.total_units = units;
+  p.work = reinterpret_cast<unsigned *>(workspace);
+  memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+  return run_gemv_small(a_dtype, bs, (int)M, p, di.sms, (cudaStream_t)stream);
 }
 
 }  // namespace
@@ -333,9 +390,9 @@ int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream
 }
 
 int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {
-  if (!bytes || !Wq || count < 1 || count > kMaxGroup) return Q4_ERR_ARG;
+  if (!bytes || !Wq || count < 1 || count > kGvMaxGroup) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
-  size_t total = 0;
+  size_t total = kGemvWsHead;
   for (int i = 0; i < count; ++i) {
     if (!Wq[i]) return Q4_ERR_ARG;
     if (!valid_bs(Wq[i]->blocksize) || Wq[i]->cols % Wq[i]->blocksize) return Q4_ERR_SHAPE;
@@ -349,19 +406,23 @@ int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
 int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace,
                     size_t workspace_bytes, void *stream) {
-  if (count < 1 || count > kMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (count < 1 || count > kGvMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
-  GemvParams p;
+  if (!Wq[0]) return Q4_ERR_ARG;
+  if (M <= 16) return gemv_small_grouped(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
+  static thread_local GvParams p;  // host staging of the kernel parameters (~5 KB)
   memset(&p, 0, sizeof(p));
   p.count = count;
   p.M = (int)M;
   p.y_dtype = y_dtype;
-  if (!Wq[0]) return Q4_ERR_ARG;
   const int bs = Wq[0]->blocksize;
   const int dq = Wq[0]->double_quant;
+  const int mp = pow2_at_least(M);
+  const int nb = mp <= 16 ? 16 : 32;
+  const DeviceInfo di = device_info();
   int64_t units = 0;
-  size_t ws_off = 0;
+  size_t ws_off = kGemvWsHead;
   for (int i = 0; i < count; ++i) {
     const q4_state *s = Wq[i];
     int rc = check_state(s);
@@ -370,15 +431,20 @@ int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *
     if (s->cols % bs || s->rows > INT32_MAX || s->cols > INT32_MAX) return Q4_ERR_SHAPE;
     if (!A[i] || !Y[i]) return Q4_ERR_ARG;
     if (!aligned16(A[i])) return Q4_ERR_ALIGN;
+    if (di.ok != Q4_OK) return di.ok;
     int64_t n_tiles, n_splits;
     const size_t need = gemv_ws_for(s, M, &n_tiles, &n_splits);
-    GemvMat &m = p.mat[i];
-    m.packed = s->packed;
+    GvMat &m = p.mat[i];
+    const CUtensorMapDataType adt =
+        a_dtype == Q4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&m.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1,
+                  kGvStageK / 2, kGvRows, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !make_map(&m.tmA, adt, A[i], M, s->cols, 2, kGvStageK, nb, CU_TENSOR_MAP_SWIZZLE_128B))
+      return Q4_ERR_CUDA;
     m.absmax = s->absmax;
     m.absmax_q = s->absmax_q;
     m.absmax_scale = s->absmax_scale;
     m.absmax_mean = s->absmax_mean;
-    m.A = reinterpret_cast<const uint16_t *>(A[i]);
     m.Y = Y[i];
     m.N = (int32_t)s->rows;
     m.K = (int32_t)s->cols;
@@ -396,11 +462,9 @@ int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *
   }
   p.dq = dq;
   p.total_units = units;
+  p.status = di.status;
   memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
-  const DeviceInfo di = device_info();
-  if (di.ok != Q4_OK) return di.ok;
-  const GemvPlan pl = gemv_plan(M);
-  return run_gemv(a_dtype, pl.nt, pl.r, bs, p, di.sms, (cudaStream_t)stream);
+  return run_gemv(a_dtype, bs, mp, p, di.sms, (cudaStream_t)stream);
 }
 
 int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
@@ -413,7 +477,7 @@ int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void 
 
 int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream) {
-  if (count < 1 || count > kMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (count < 1 || count > kGvMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (y_dtype != Q4_F32 && y_dtype != a_dtype) return Q4_ERR_ARG;
   if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;
