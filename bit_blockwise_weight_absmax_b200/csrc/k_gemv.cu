@@ -55,14 +55,25 @@ int by_bs(int bs, int mp, const GvParams &p, int sms, cudaStream_t st) {
   }
   return Q4_ERR_ARG;
 }
-template <int DA, int NT, int R, int B>
+// Stages of the mma.sync kernel's ring: as many as fit two CTAs per SM
+// (228 KB per SM, 1 KB reserved per CTA), at most 12.
+template <int DA, int NT>
+constexpr int small_stages() {
+  constexpr int STAGE = kGsWTile + 8 * NT * 128;
+  constexpr int LUTB = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
+  constexpr int budget = (228 * 1024) / 2 - 1024 - LUTB - 1024 - 64;
+  constexpr int s = budget / (STAGE + 20);
+  return s < 12 ? s : 12;
+}
+template <int DA, int NT, int B>
 int go_small(const GsParams &p, int sms, cudaStream_t st) {
-  constexpr int UB = kGsUnitK / B;
-  // prefetch depth: about 40 bytes per lane and row in flight (R == 1), 32 (R == 2)
-  constexpr int PF0 = ((R == 1) ? 40 : 32) / (B / 8);
-  constexpr int PF = PF0 < 1 ? 1 : (UB < PF0 ? UB : PF0);
-  auto kern = gemv_small_kernel<DA, NT, R, B, PF>;
-  constexpr int SMEM = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
+  constexpr int S = small_stages<DA, NT>();
+  static_assert(S >= 4, "ring too small");
+  constexpr int STAGE = kGsWTile + 8 * NT * 128;
+  constexpr int LUTB = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
+  constexpr int SMEM = S * STAGE + LUTB + 2 * S * 8 + S * 4 + 1024;
+  static_assert(2 * (SMEM + 1024 + 64) <= 228 * 1024, "two CTAs per SM");
+  auto kern = gemv_small_kernel<DA, NT, B, S>;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess ||
@@ -71,25 +82,24 @@ int go_small(const GsParams &p, int sms, cudaStream_t st) {
       return Q4_ERR_CUDA;
     attr = true;
   }
-  const int64_t want = (p.total_units + kGsWarps - 1) / kGsWarps;
-  const int grid = (int)std::min<int64_t>(want, (int64_t)sms * (R == 1 ? 3 : 2));
-  kern<<<grid, kGsWarps * 32, SMEM, st>>>(p);
+  const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * 2);
+  kern<<<grid, kGsThreads, SMEM, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
-template <int DA, int NT, int R>
+template <int DA, int NT>
 int small_bs(int bs, const GsParams &p, int sms, cudaStream_t st) {
   switch (bs) {
-    case 32: return go_small<DA, NT, R, 32>(p, sms, st);
-    case 64: return go_small<DA, NT, R, 64>(p, sms, st);
-    case 128: return go_small<DA, NT, R, 128>(p, sms, st);
-    case 256: return go_small<DA, NT, R, 256>(p, sms, st);
+    case 32: return go_small<DA, NT, 32>(p, sms, st);
+    case 64: return go_small<DA, NT, 64>(p, sms, st);
+    case 128: return go_small<DA, NT, 128>(p, sms, st);
+    case 256: return go_small<DA, NT, 256>(p, sms, st);
   }
   return Q4_ERR_ARG;
 }
 template <int DA>
 int small_m(int M, int bs, const GsParams &p, int sms, cudaStream_t st) {
-  if (M <= 8) return small_bs<DA, 1, 1>(bs, p, sms, st);
-  return small_bs<DA, 2, 2>(bs, p, sms, st);
+  if (M <= 8) return small_bs<DA, 1>(bs, p, sms, st);
+  return small_bs<DA, 2>(bs, p, sms, st);
 }
 }  // namespace
 

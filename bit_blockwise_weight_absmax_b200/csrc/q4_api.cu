@@ -135,17 +135,18 @@ int check_state(const q4_state *s) {
 }
 
 // ---- GEMV planning ----------------------------------------------------------
-// M <= 16: warp units of 16 R rows x 1024 k (mma.sync kernel); M > 16: CTA
-// units of 128 rows x 1024 k (tcgen05 kernel).  Workspace: two work counters,
-// then per split matrix fp32 [N][M] partial sums and per-tile counters.
+// Units of 128 rows x 1024 k for both kernels (mma.sync for M <= 16, tcgen05
+// above).  Workspace: two work counters, then per split matrix fp32 [N][M]
+// partial sums and the arrival counters (one per 16 rows for the mma.sync
+// kernel, one per tile for the tcgen05 kernel).
 constexpr size_t kGemvWsHead = 256;
-int gemv_small_rows(int64_t M) { return M <= 8 ? 16 : 32; }
 size_t gemv_ws_for(const q4_state *s, int64_t M, int64_t *n_tiles, int64_t *n_splits) {
-  const int64_t rows = M <= 16 ? gemv_small_rows(M) : kGvRows;
-  *n_tiles = ceil_div(s->rows, rows);
-  *n_splits = ceil_div(s->cols, M <= 16 ? kGsUnitK : kGvUnitK);
+  const bool small = M <= 16;
+  *n_tiles = ceil_div(s->rows, small ? kGsRows : kGvRows);
+  *n_splits = ceil_div(s->cols, small ? kGsUnitK : kGvUnitK);
   if (*n_splits <= 1) return 0;
-  return align256((size_t)s->rows * (size_t)M * 4) + align256((size_t)*n_tiles * 4);
+  const int64_t counters = small ? ceil_div(s->rows, 16) : *n_tiles;
+  return align256((size_t)s->rows * (size_t)M * 4) + align256((size_t)counters * 4);
 }
 int pow2_at_least(int64_t m) {
   int p = 1;
@@ -212,6 +213,12 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
     int64_t n_tiles, n_splits;
     const size_t need = gemv_ws_for(s, M, &n_tiles, &n_splits);
     GsMat &m = p.mat[i];
+    const CUtensorMapDataType adt =
+        a_dtype == Q4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    if (!make_map(&m.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1, 32, kGsRows,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&m.tmA, adt, A[i], M, s->cols, 2, 64, M <= 8 ? 8 : 16, CU_TENSOR_MAP_SWIZZLE_128B))
+      return Q4_ERR_CUDA;
     m.packed = s->packed;
     m.absmax = s->absmax;
     m.absmax_q = s->absmax_q;
@@ -237,6 +244,7 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
   p.dq = dq;
   p.total_units = units;
   p.work = reinterpret_cast<unsigned *>(workspace);
+  p.status = di.status;
   memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
   return run_gemv_small(a_dtype, bs, (int)M, p, di.sms, (cudaStream_t)stream);
 }

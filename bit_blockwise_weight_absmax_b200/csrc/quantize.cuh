@@ -21,6 +21,8 @@
 // -> CTA run (streaming pairwise stack) -> the last CTA to finish combines the
 // per-CTA partial sums and writes the mean.
 #pragma once
+#include <type_traits>
+
 #include "q4_common.cuh"
 
 namespace q4 {
@@ -67,6 +69,18 @@ __device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
   return max(m & 0xFFFFu, m >> 16);
 }
 
+// NF4 code of x = RN(w / c) for |x| <= 1 (w finite): the bin is the low byte
+// of fmaf(x, 15, 1.5 * 2^23 + 15) (0..30), whose pattern is 0x4B4000jj, so
+// (pattern << 8) = 0x40000000 + 256 j and `tb` = table address of this lane
+// minus 0x40000000 gives the entry of bin j (32-bit shared addresses wrap).
+__device__ __forceinline__ uint32_t nf4_code_fast(float x, uint32_t tb) {
+  const uint32_t bits = __float_as_uint(__fmaf_rn(x, 15.0f, 12582927.0f));
+  float thr;
+  int base;
+  asm("ld.shared.v2.b32 {%0,%1}, [%2];" : "=f"(thr), "=r"(base) : "r"((bits << 8) + tb));
+  return (uint32_t)(base + (x >= thr ? 1 : 0));
+}
+
 template <int DT, int QT, int B, bool DQ>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
   constexpr int LPB = B / 8;                     // lanes per block
@@ -74,6 +88,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
   constexpr int IT_PER_CHUNK = kChunkBlocks * B / ELEMS_IT;  // = B / 8
   constexpr int BLK_IT = ELEMS_IT / B;           // blocks per CTA iteration
   constexpr int BATCH = IT_PER_CHUNK < 8 ? IT_PER_CHUNK : 8;
+  constexpr int64_t CHUNK_ELEMS = (int64_t)kChunkBlocks * B;
 
   __shared__ float2 s_tab[32 * 32];              // lane-private copies of the bin table
   __shared__ double s_blk[kChunkBlocks];         // block absmax of the current chunk
@@ -90,94 +105,61 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
     }
   }
   __syncthreads();
+  const uint32_t tlane = (uint32_t)__cvta_generic_to_shared(s_tab) + 8u * lane;  // bin 0, this lane
+  const uint32_t tb = tlane - 0x40000000u;
 
   int nonfinite = 0;
   int depth = 0;  // stack depth (thread 0)
   const int64_t c0 = (int64_t)blockIdx.x * p.run;
   const int64_t c1 = min(c0 + p.run, p.n_chunks);
 
-  for (int64_t chunk = c0; chunk < c1; ++chunk) {
-    const int64_t chunk_e0 = chunk * (int64_t)kChunkBlocks * B;
-    for (int it0 = 0; it0 < IT_PER_CHUNK; it0 += BATCH) {
-      uint4 v[BATCH];
+  // Codes of the thread's eight elements (element j in bits 4j..4j+3) and
+  // the block's scale; lanes of one block agree on `scale` and `z`.
+  auto quant8 = [&](const uint4 &v, float &scale, int &z) -> uint32_t {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
 #pragma unroll
-      for (int b = 0; b < BATCH; ++b) {
-        const int64_t e0 = chunk_e0 + (int64_t)(it0 + b) * ELEMS_IT + tid * 8;
-        if (e0 + 8 <= p.n) {
-          v[b] = ldg_stream_v4(p.W + e0);
+    for (int j = 0; j < 4; ++j) {
+      f[2 * j] = lo16<DT>(w[j]);
+      f[2 * j + 1] = hi16<DT>(w[j]);
+    }
+    uint32_t codes = 0;
+    if (QT == Q4_NF4 || QT == Q4_INT4_SYM) {
+      uint32_t m = absmax_bits8(v);
+#pragma unroll
+      for (int o = LPB / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      const float c = Dt<DT>::to_f((uint16_t)m);
+      if (!(c <= 3.4028235e38f)) nonfinite = 1;
+      if (QT == Q4_NF4) {
+        scale = c;
+        if (__all_sync(0xffffffffu, markstein_ok(c))) {
+          // every lane: finite weights with |w| <= c, so |x| <= 1
+          const float y = __frcp_rn(c);
+#pragma unroll
+          for (int j = 7; j >= 0; --j) codes = (codes << 4) + nf4_code_fast(div_markstein(f[j], c, y), tb);
         } else {
-          uint16_t t[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) t[j] = (e0 + j < p.n) ? p.W[e0 + j] : (uint16_t)0;
-          v[b] = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
-                            t[6] | (t[7] << 16));
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < BATCH; ++b) {
-        const int it = it0 + b;
-        const int64_t e0 = chunk_e0 + (int64_t)it * ELEMS_IT + tid * 8;
-        const int64_t blk = e0 / B;
-        const uint32_t w[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
-        float f[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          f[2 * j] = lo16<DT>(w[j]);
-          f[2 * j + 1] = hi16<DT>(w[j]);
-        }
-        uint32_t codes = 0;
-        float scale;
-        if (QT == Q4_NF4 || QT == Q4_INT4_SYM) {
-          uint32_t m = absmax_bits8(v[b]);
-#pragma unroll
-          for (int o = LPB / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-          const float c = Dt<DT>::to_f((uint16_t)m);
-          if (!(c <= 3.4028235e38f)) nonfinite = 1;
-          if (QT == Q4_NF4) {
-            scale = c;
-            const bool fast = markstein_ok(c);
-            const float y = fast ? __frcp_rn(c) : 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float x = fast ? div_markstein(f[j], c, y) : (c == 0.0f ? 0.0f : __fdiv_rn(f[j], c));
-              const float2 e = s_tab[nf4_bin(x) * 32 + lane];
-              const int code = __float_as_int(e.y) + (x >= e.x ? 1 : 0);
-              codes |= (uint32_t)code << (4 * j);
-            }
-          } else {
-            const float s = __fdiv_rn(c, 7.0f);
-            scale = s;
-            const bool fast = markstein_ok(s);
-            const float y = fast ? __frcp_rn(s) : 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              int q = 0;
-              if (s != 0.0f) {
-                float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
-                q = min(max(__float2int_rn(x), -8), 7);
-              }
-              codes |= (uint32_t)(q & 15) << (4 * j);
-            }
-          }
-        } else {  // Q4_INT4_ASYM
-          float mn = 0.0f, mx = 0.0f;
+          const bool fast = markstein_ok(c);
+          const float y = fast ? __frcp_rn(c) : 0.0f;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            mn = fminf(mn, f[j]);
-            mx = fmaxf(mx, f[j]);
+            float x = fast ? div_markstein(f[j], c, y) : (c == 0.0f ? 0.0f : __fdiv_rn(f[j], c));
+            const float2 e = s_tab[nf4_bin(x) * 32 + lane];
+            const int code = __float_as_int(e.y) + (x >= e.x ? 1 : 0);
+            codes |= (uint32_t)code << (4 * j);
           }
-          uint32_t m = absmax_bits8(v[b]);
+        }
+      } else {
+        const float s = __fdiv_rn(c, 7.0f);
+        scale = s;
+        if (__all_sync(0xffffffffu, markstein_ok(s))) {
+          // |w / s| <= 7 / (1 - 2^-24): rint never leaves [-7, 7], and adding
+          // 1.5 * 2^23 rounds to the nearest integer, ties to even, leaving
+          // its 4-bit two's complement in the low nibble
+          const float y = __frcp_rn(s);
 #pragma unroll
-          for (int o = LPB / 2; o >= 1; o >>= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-          }
-          if (!(Dt<DT>::to_f((uint16_t)m) <= 3.4028235e38f)) nonfinite = 1;
-          const float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-          scale = s;
-          int z = 0;
-          if (s != 0.0f) z = min(max(__float2int_rn(__fdiv_rn(-mn, s)), 0), 15);
+          for (int j = 7; j >= 0; --j)
+            codes = (codes << 4) | (__float_as_uint(__fadd_rn(div_markstein(f[j], s, y), 12582912.0f)) & 15u);
+        } else {
           const bool fast = markstein_ok(s);
           const float y = fast ? __frcp_rn(s) : 0.0f;
 #pragma unroll
@@ -185,39 +167,115 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
             int q = 0;
             if (s != 0.0f) {
               float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
-              q = min(max(__float2int_rn(x) + z, 0), 15);
+              q = min(max(__float2int_rn(x), -8), 7);
             }
-            codes |= (uint32_t)q << (4 * j);
+            codes |= (uint32_t)(q & 15) << (4 * j);
           }
-          if ((tid % LPB) == 0) s_zero[(tid * 8) / B] = (uint8_t)z;
-        }
-        // ---- stores
-        if (e0 + 8 <= p.n) {
-          *reinterpret_cast<uint32_t *>(p.packed + e0 / 2) = codes;
-        } else if (e0 < p.n) {
-          const int valid = (int)(p.n - e0);
-          for (int j = 0; j < 4; ++j) {
-            if (2 * j < valid) {
-              uint32_t byte = (codes >> (8 * j)) & 0xFFu;
-              if (2 * j + 1 >= valid) byte &= 0x0Fu;  // odd n: high nibble is padding
-              p.packed[e0 / 2 + j] = (uint8_t)byte;
-            }
-          }
-        }
-        if ((tid % LPB) == 0) {
-          if (blk < p.nb) p.absmax[blk] = scale;
-          if (DQ) s_blk[it * BLK_IT + (tid * 8) / B] = (blk < p.nb) ? (double)scale : 0.0;
-        }
-        if (QT == Q4_INT4_ASYM) {
-          __syncthreads();
-          if (tid < BLK_IT / 2) {
-            const int64_t b0 = (chunk_e0 + (int64_t)it * ELEMS_IT) / B + 2 * tid;
-            if (b0 < p.nb) p.zero[b0 / 2] = (uint8_t)(s_zero[2 * tid] | (s_zero[2 * tid + 1] << 4));
-          }
-          __syncthreads();
         }
       }
+    } else {  // Q4_INT4_ASYM
+      float mn = 0.0f, mx = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        mn = fminf(mn, f[j]);
+        mx = fmaxf(mx, f[j]);
+      }
+      uint32_t m = absmax_bits8(v);
+#pragma unroll
+      for (int o = LPB / 2; o >= 1; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      }
+      if (!(Dt<DT>::to_f((uint16_t)m) <= 3.4028235e38f)) nonfinite = 1;
+      const float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+      scale = s;
+      z = 0;
+      if (s != 0.0f) z = min(max(__float2int_rn(__fdiv_rn(-mn, s)), 0), 15);
+      const bool fast = markstein_ok(s);
+      const float y = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        int q = 0;
+        if (s != 0.0f) {
+          float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
+          q = min(max(__float2int_rn(x) + z, 0), 15);
+        }
+        codes |= (uint32_t)q << (4 * j);
+      }
     }
+    return codes;
+  };
+
+  for (int64_t chunk = c0; chunk < c1; ++chunk) {
+    const int64_t chunk_e0 = chunk * CHUNK_ELEMS;
+    const int64_t chunk_b0 = chunk * kChunkBlocks;
+    // FULL: the whole chunk lies inside the tensor (every chunk but the last)
+    auto run_chunk = [&](auto full_tag) {
+      constexpr bool FULL = decltype(full_tag)::value;
+      const uint16_t *wp = p.W + chunk_e0 + tid * 8;
+      uint8_t *pp = p.packed + chunk_e0 / 2 + tid * 4;
+      for (int it0 = 0; it0 < IT_PER_CHUNK; it0 += BATCH) {
+        uint4 v[BATCH];
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+          const int off = (it0 + b) * ELEMS_IT;
+          if (FULL) {
+            v[b] = ldg_stream_v4(wp + off);
+          } else {
+            const int64_t e0 = chunk_e0 + off + tid * 8;
+            if (e0 + 8 <= p.n) {
+              v[b] = ldg_stream_v4(wp + off);
+            } else {
+              uint16_t t[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) t[j] = (e0 + j < p.n) ? p.W[e0 + j] : (uint16_t)0;
+              v[b] = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
+                                t[6] | (t[7] << 16));
+            }
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+          const int it = it0 + b;
+          const int off = it * ELEMS_IT;
+          const int bl = it * BLK_IT + (tid * 8) / B;  // block within the chunk
+          float scale = 0.0f;
+          int z = 0;
+          const uint32_t codes = quant8(v[b], scale, z);
+          if (QT == Q4_INT4_ASYM && (tid % LPB) == 0) s_zero[(tid * 8) / B] = (uint8_t)z;
+          // ---- stores
+          const int64_t e0 = chunk_e0 + off + tid * 8;
+          if (FULL || e0 + 8 <= p.n) {
+            *reinterpret_cast<uint32_t *>(pp + off / 2) = codes;
+          } else if (e0 < p.n) {
+            const int valid = (int)(p.n - e0);
+            for (int j = 0; j < 4; ++j) {
+              if (2 * j < valid) {
+                uint32_t byte = (codes >> (8 * j)) & 0xFFu;
+                if (2 * j + 1 >= valid) byte &= 0x0Fu;  // odd n: high nibble is padding
+                pp[off / 2 + j] = (uint8_t)byte;
+              }
+            }
+          }
+          if ((tid % LPB) == 0) {
+            const bool in = FULL || chunk_b0 + bl < p.nb;
+            if (in) p.absmax[chunk_b0 + bl] = scale;
+            if (DQ) s_blk[bl] = in ? (double)scale : 0.0;
+          }
+          if (QT == Q4_INT4_ASYM) {
+            __syncthreads();
+            if (tid < BLK_IT / 2) {
+              const int64_t b0 = chunk_b0 + it * BLK_IT + 2 * tid;
+              if (b0 < p.nb) p.zero[b0 / 2] = (uint8_t)(s_zero[2 * tid] | (s_zero[2 * tid + 1] << 4));
+            }
+            __syncthreads();
+          }
+        }
+      }
+    };
+    if (chunk_e0 + CHUNK_ELEMS <= p.n) run_chunk(std::true_type{});
+    else run_chunk(std::false_type{});
     if (DQ) {
       // Pairwise fp64 sum of the chunk's 256 block values in tree order:
       // lane l reduces blocks 8l..8l+7 as ((0+1)+(2+3))+((4+5)+(6+7)), then
