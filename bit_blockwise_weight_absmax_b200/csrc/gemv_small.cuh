@@ -8,27 +8,39 @@
 // to the compute dtype, then a 16-bit matmul); the dequantization is fused
 // into the streaming of the packed weights.
 //
-// Design (B200, decode sizes): at M <= 16 the per-instruction cost of a
-// tcgen05 MMA (128 x 16 x 16 takes ~44 cycles) would cap the kernel at about
-// the HBM rate, while the warp-level mma.sync path (m16n8k16, ~0.44 per clock
-// per SM) has 2.5x headroom at M <= 8; what limits it is the load/store pipe
-// (each decoded byte is one shared-memory lookup) and the instructions spent
-// per weight.  So:
-//   * a CTA takes units of 128 weight rows x 1024 k from a work counter
-//     (balanced, self-resetting); its producer warp streams each 64-k stage
-//     of packed bytes ([128 x 32 B]) and activations ([8 NT x 64], 128-byte
-//     swizzle, rows >= M zero-filled) with TMA into a ring of stages;
-//   * each of 8 compute warps owns 16 rows (the MMA rows; swap-AB) and reads
-//     its bytes and the activations from shared memory without conflicts;
-//   * a byte maps to a pair of fp16 codebook values through a 256-entry table
-//     in shared memory (one copy per lane), the MMA runs on the unscaled
-//     values and each block's fp32 partial is scaled once by its c~; the k
-//     order inside a segment of min(B, 64) is permuted identically on both
-//     operands so that a lane reads consecutive bytes;
-//   * the unit's block scales come from a few vector loads of the int8
-//     double-quant codes;
-//   * split rows add fp32 partials into a workspace; the last warp of a
-//     16-row group writes Y and zeroes its rows again.
+// Design (B200, decode sizes).  At M <= 16 a tcgen05 MMA (128 x 16 x 16
+// takes ~44 cycles) would cap the kernel near the HBM rate, while the
+// warp-level mma.sync path (m16n8k16) has ample headroom; what limits a
+// decode GEMV on this part is the issue rate and the shared-memory pipe (one
+// table lookup per packed byte).  So the kernel spends as few instructions
+// per weight as it can:
+//   * one CTA per SM; a producer warp streams 128-k stages of packed bytes
+//     ([256 rows x 64 B], TMA) and of the M activation rows (two [M x 64]
+//     halves, 128-byte swizzle) into a ring in shared memory;
+//   * the work is the concatenation of every matrix's (256-row tile,
+//     128-k stage) pairs, cut into equal contiguous ranges, one per CTA: no tail,
+//     no work counter, and a CTA meets only a few tiles, so the split-K
+//     reduction runs a few times per CTA;
+//   * 16 compute warps own 16 rows each (the MMA rows; swap-AB) and read
+//     their bytes and the activation rows from the ring without conflicts;
+//     the two halves of a stage are independent chains (more work in flight
+//     per warp, half the barrier traffic of 64-k stages);
+//   * a byte maps to the pair of its two codebook values through a
+//     256-entry table in shared memory (one copy per lane) placed at a
+//     64 KB-aligned shared address, so a single PRMT forms the address
+//     (byte 1 = the packed byte, the other bytes = table base + lane);
+//   * the MMA runs on the unscaled fp16 levels and each block's fp32 partial
+//     is scaled once by its absmax c~; the k order inside a segment of
+//     min(B, 64) is permuted identically on both operands so that a lane
+//     reads consecutive bytes;
+//   * each warp computes the c~ of its rows for the next 16 blocks one unit
+//     ahead (loads issued a whole unit before they are needed) into a small
+//     buffer of its own;
+//   * only a CTA's first and last tiles can be partial: their fp32 partial
+//     rows go to two per-CTA slots with plain stores; after its last stage
+//     each warp counts its contributions per 16-row group, and the one that
+//     completes a group sums the slots of all contributors, in CTA order,
+//     into Y and zeroes them (deterministic; nothing waits mid-stream).
 // bf16 activations multiply the exact w^ = bf16(c~ * level) (the definition
 // dequantizes to the compute dtype first), with a binary32 pair table.
 #pragma once
@@ -39,29 +51,46 @@
 
 namespace q4 {
 
-constexpr int kGsWarps = 8;                 // compute warps (16 rows each)
-constexpr int kGsThreads = (kGsWarps + 1) * 32;  // + the TMA producer warp
-constexpr int kGsRows = 16 * kGsWarps;      // rows per unit (one CTA tile)
-constexpr int kGsUnitK = 1024;
+constexpr int kGsRows = 256;                      // rows per tile (16 per MMA row group)
+constexpr int kGsMaxCtas = 256;                   // grid bound (split-K slots are per CTA)
+constexpr int kGsStageK = 128;                    // k per stage (two 64-k halves)
+constexpr int kGsWTile = kGsRows * kGsStageK / 2; // packed bytes per stage
 constexpr int kGsMaxGroup = 16;
-constexpr int kGsWTile = kGsRows * 32;      // packed bytes per 64-k stage
+constexpr int kGsMaxStages = 16;
+constexpr int kGsWinBlocks = 16;                  // blocks per scale window
+constexpr int kGsScaleBuf = kGsWinBlocks * 16 * 4;        // c~ of one 16-row group's unit
+constexpr int kGsScaleBytes = (kGsRows / 16) * 2 * kGsScaleBuf;  // two per row group
+constexpr int kGsBarBytes = 2 * kGsMaxStages * 8 + 16;  // barriers + abort flag
+constexpr int kGsInfoBytes = 16 * 64;             // per-matrix fields, copied to shared memory
+constexpr int kGsSmemBytes = 227 * 1024;          // dynamic shared memory of a CTA
 
 struct alignas(64) GsMat {
-  CUtensorMap tmW;  // packed [N, K/2] bytes, box {32, 128}
-  CUtensorMap tmA;  // activations [M, K] 16-bit, box {64, 8 NT}, 128-byte swizzle
-  const uint8_t *packed;
+  CUtensorMap tmW;  // packed [N, K/2] bytes, box {32, 256}
+  CUtensorMap tmA;  // activations [M, K] 16-bit, box {64, M}, 128-byte swizzle
   const float *absmax;
   const int8_t *absmax_q;
   const float *absmax_scale;
   const float *absmax_mean;
-  const uint16_t *A;
   void *Y;
-  float *acc;      // split-K workspace [N][M] fp32 (n_splits > 1)
-  unsigned *cnt;   // per 16-row arrival counters
-  int64_t unit_begin;
+  unsigned *cnt;    // per 16-row group: stages counted so far (zero between calls)
+  uint32_t stage_begin;  // first global stage index of this matrix
   int32_t N, K;
-  int32_t n_tiles, n_splits;
+  int32_t n_tiles, n_stages;  // 256-row tiles; 128-k stages per tile
 };
+
+// The fields the kernel reads per unit, copied once into shared memory (a
+// dynamic index into the parameter block would miss the constant cache).
+struct alignas(16) GsInfo {
+  uint32_t stage_begin;
+  int32_t N, K, n_stages;
+  const float *absmax;
+  const int8_t *absmax_q;
+  const float *absmax_scale;
+  const float *absmax_mean;
+  void *Y;
+  unsigned *cnt;
+};
+static_assert(sizeof(GsInfo) == 64, "GsInfo layout");
 
 struct GsParams {
   GsMat mat[kGsMaxGroup];
@@ -69,28 +98,43 @@ struct GsParams {
   int32_t M;
   int32_t y_dtype;
   int32_t dq;
-  int64_t total_units;
-  unsigned *work;   // [2]: next unit, finished producers (both left at 0)
+  uint32_t total_stages;  // below 2^32 / kGsMaxCtas, so c * T fits 32 bits
+  float *slots;     // [grid][2][256 rows][8 NT] fp32 partial rows of each CTA's first / last tile
   int *status;
   float levels[16];
 };
+
+// CTA c covers global stages [c T / G, (c+1) T / G); the CTA holding stage x.
+__device__ __forceinline__ uint32_t gs_range_begin(uint32_t c, uint32_t T, uint32_t G) { return c * T / G; }
+__device__ __forceinline__ int gs_cta_of(uint32_t x, uint32_t T, uint32_t G) {
+  uint32_t c = x * G / T;
+  while (c + 1 < G && gs_range_begin(c + 1, T, G) <= x) ++c;
+  while (c > 0 && gs_range_begin(c, T, G) > x) --c;
+  return (int)c;
+}
 
 template <int DA> struct MmaS;
 template <> struct MmaS<Q4_F16> {
   static __device__ __forceinline__ void run(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+  // d = A . B (the accumulator starts at zero)
+  static __device__ __forceinline__ void run0(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
   }
 };
 template <> struct MmaS<Q4_BF16> {
   static __device__ __forceinline__ void run(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -103,350 +147,570 @@ __device__ __forceinline__ void gs_store(void *Y, int ydt, int64_t idx, float v)
   else reinterpret_cast<uint16_t *>(Y)[idx] = Dt<Q4_BF16>::from_f(v);
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+// Loads from the ring and the c~ buffer (ordered after the barrier waits:
+// volatile).
+__device__ __forceinline__ uint32_t lds32v(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+__device__ __forceinline__ uint2 lds64v(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+__device__ __forceinline__ uint4 lds128v(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ float2 lds64f(uint32_t addr) {
+__device__ __forceinline__ float2 lds64fv(uint32_t addr) {
   float2 v;
   asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
   return v;
 }
-// Table entry address for byte j of `word` (lane-private copies: entry e of
-// lane l at e * stride + esize * l; `lb` = table base + esize * l).
-template <int SHIFT>
+// Table lookups: the table is constant after the start-up barrier and the
+// address depends on ring data, so these need no ordering of their own.
+__device__ __forceinline__ uint32_t lut32(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float2 lut64f(uint32_t addr) {
+  float2 v;
+  asm("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Address of the table entry of byte j of `word`: byte 1 of the address is
+// the packed byte; bytes 0, 2, 3 come from `lb` (table base + lane offset,
+// whose byte 1 is zero because the table is 64 KB aligned).
 __device__ __forceinline__ uint32_t lut_addr(uint32_t word, int j, uint32_t lb) {
-  return (__byte_perm(word, 0u, 0x4440u | (uint32_t)j) << SHIFT) + lb;
+  return __byte_perm(word, lb, 0x7604u | ((uint32_t)j << 4));
 }
 
-// DA: activation dtype; NT: n8 tiles (M <= 8 NT); B: blocksize; S: stages.
-template <int DA, int NT, int B, int S>
-__global__ void __launch_bounds__(kGsThreads, 2) gemv_small_kernel(const __grid_constant__ GsParams p) {
+// One unit: the stages of one tile inside one window of 16 blocks, clipped
+// to the CTA's range.  A pure function of the global stage index, so the
+// producer and every compute warp walk the same sequence without talking.
+struct GsUnit {
+  int mi, tile, q0, q1;
+  bool first, last;  // first / last unit of this CTA on the tile
+};
+template <int B>
+__device__ __forceinline__ GsUnit gs_describe(const GsInfo *info, int count, int &mi, uint32_t g, uint32_t g0,
+                                             uint32_t g1) {
+  constexpr int W = kGsWinBlocks * B / kGsStageK;  // stages per window of 16 blocks
+#pragma unroll 1
+  while (mi + 1 < count && g >= info[mi + 1].stage_begin) ++mi;
+  const GsInfo &mt = info[mi];
+  const int local = (int)(g - mt.stage_begin);
+  GsUnit u;
+  u.mi = mi;
+  u.tile = local / mt.n_stages;
+  u.q0 = local - u.tile * mt.n_stages;
+  int q1 = min((u.q0 / W + 1) * W, mt.n_stages);
+  q1 = min(q1, u.q0 + (int)(g1 - g));
+  u.q1 = q1;
+  u.first = (u.q0 == 0) || (g == g0);
+  u.last = (q1 == mt.n_stages) || (g + (q1 - u.q0) == g1);
+  return u;
+}
+
+// Inputs of the c~ of 8 blocks of one row (lane: row r0 + (lane & 15),
+// blocks (lane >> 4) * 8 + j of the window), loaded one unit ahead.
+struct GsScaleIn {
+  uint32_t c0, c1;   // int8 codes (double quant)
+  float s2a, s2b, mu;
+  int bsplit, nvalid;
+  float f[8];        // fp32 absmax (no double quant)
+};
+
+template <int B>
+__device__ __forceinline__ void gs_scale_load(const GsInfo *info, bool dq, const GsUnit &u, int r0, int lane,
+                                              GsScaleIn &in) {
+  constexpr int W = kGsWinBlocks * B / kGsStageK;
+  const GsInfo &mt = info[u.mi];
+  const int row = u.tile * kGsRows + r0 + (lane & 15);
+  const int nbk = mt.K / B;
+  const int b0 = (u.q0 / W) * kGsWinBlocks + (lane >> 4) * 8;  // first block of the lane
+  in.nvalid = (row < mt.N) ? max(0, min(8, nbk - b0)) : 0;
+  in.c0 = in.c1 = 0;
+  in.s2a = in.s2b = in.mu = 0.0f;
+  in.bsplit = 8;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) in.f[j] = 0.0f;
+  if (in.nvalid == 0) return;
+  const int64_t bi0 = (int64_t)row * nbk + b0;
+  if (dq) {
+    in.mu = __ldg(mt.absmax_mean);
+    const int64_t g0 = bi0 >> 8;
+    in.s2a = __ldg(mt.absmax_scale + g0);
+    in.s2b = __ldg(mt.absmax_scale + ((bi0 + in.nvalid - 1) >> 8));
+    in.bsplit = (int)min((int64_t)8, ((g0 + 1) << 8) - bi0);
+    if (in.nvalid == 8 && (bi0 & 3) == 0) {
+      const unsigned *q = reinterpret_cast<const unsigned *>(mt.absmax_q + bi0);
+      in.c0 = __ldg(q);
+      in.c1 = __ldg(q + 1);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t b = (j < in.nvalid) ? (uint32_t)(uint8_t)__ldg(mt.absmax_q + bi0 + j) : 0u;
+        if (j < 4) in.c0 |= b << (8 * j);
+        else in.c1 |= b << (8 * (j - 4));
+      }
+    }
+  } else {
+    if (in.nvalid == 8 && (bi0 & 3) == 0) {
+      const float4 x = __ldg(reinterpret_cast<const float4 *>(mt.absmax + bi0));
+      const float4 y = __ldg(reinterpret_cast<const float4 *>(mt.absmax + bi0) + 1);
+      in.f[0] = x.x; in.f[1] = x.y; in.f[2] = x.z; in.f[3] = x.w;
+      in.f[4] = y.x; in.f[5] = y.y; in.f[6] = y.z; in.f[7] = y.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < in.nvalid) in.f[j] = __ldg(mt.absmax + bi0 + j);
+    }
+  }
+}
+
+// c~ = q2 * s2 + mu (two roundings, as dequantized), 0 for blocks past the
+// row end, for block blk0 + j (j = 0..7) of row r of the warp's 16.
+__device__ __forceinline__ float gs_scale_value(const GsScaleIn &in, bool dq, int j) {
+  if (!dq) return in.f[j];
+  const uint32_t w = j < 4 ? in.c0 : in.c1;
+  const int code = (int)(int8_t)((w >> (8 * (j & 3))) & 0xFFu);
+  const float v = __fadd_rn(__fmul_rn((float)code, j < in.bsplit ? in.s2a : in.s2b), in.mu);
+  return j < in.nvalid ? v : 0.0f;
+}
+
+// Compute warps and threads of the kernel for R row groups per warp.
+template <int R> struct GsShape {
+  static constexpr int kWarps = kGsRows / (16 * R);
+  static constexpr int kThreads = (kWarps + 1) * 32;  // + the TMA producer warp
+};
+
+// DA: activation dtype; NT: n8 tiles (M <= 8 NT); B: blocksize; R: 16-row
+// groups per compute warp.
+template <int DA, int NT, int B, int R>
+__global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(const __grid_constant__ GsParams p) {
+  constexpr int WARPS = GsShape<R>::kWarps;
+  constexpr int PRODUCER = WARPS;
   constexpr bool EXACT = (DA == Q4_BF16);
   constexpr int SEG = B < 64 ? B : 64;         // k per scale segment inside a stage
-  constexpr int SEGS = 64 / SEG;               // segments per stage
+  constexpr int SEGS = kGsStageK / SEG;        // segments per stage
+  constexpr int SPH = 64 / SEG;                // segments per 64-k half
   constexpr int STEPS = SEG / 16;              // MMA k-steps per segment
   constexpr int LB = SEG / 8;                  // packed bytes per lane per segment and row
-  constexpr int UB = kGsUnitK / B;             // blocks per unit
-  constexpr int QW = (UB + 3) / 4;             // words of int8 codes per row per unit
-  constexpr int ATILE = 8 * NT * 128;          // activation tile bytes per stage
-  constexpr int STAGE = kGsWTile + ATILE;
-  constexpr int LUTB = EXACT ? 256 * 32 * 8 : 256 * 32 * 4;
+  constexpr int WV = SEG == 64 ? 2 * SEGS : SEGS;  // packed words per lane and row per stage
+  constexpr int MW = 8 * NT;                   // columns of the MMA tile (M <= MW)
+  constexpr int ATILE = MW * 128;              // activation tile bytes per 64-k half
+  constexpr int STAGE = 2 * ATILE + kGsWTile;
+  constexpr uint32_t ES = EXACT ? 8u : 4u;     // table entry bytes per lane
+  // fp16 tables use 128 of every 256 bytes: the c~ buffers live in the gaps
+  constexpr int MISC = (EXACT ? kGsScaleBytes : 0) + kGsBarBytes + kGsInfoBytes;
   static_assert(STAGE % 1024 == 0, "stage alignment");
+  static_assert(EXACT || kGsScaleBytes == 256 * 128, "c~ buffers fill the table gaps");
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sStage = smem;                                  // [S][act tile | weight tile]
-  uint8_t *sLut = smem + S * STAGE;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sLut + LUTB);  // sfull[S], sempty[S]
-  unsigned *sUnit = reinterpret_cast<unsigned *>(bars + 2 * S);  // [S] unit ring
-  __shared__ int s_abort;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+
+  // ---- shared-memory layout (addresses in the shared window): the table at
+  // the first 64 KB boundary; barriers, the abort flag, the matrix fields
+  // (and the bf16 c~ buffers) in whichever free region holds them; the ring
+  // in up to two runs of stages.
+  const uint32_t base = smem_u32(smem_raw);
+  const uint32_t end = base + kGsSmemBytes;
+  const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;
+  uint32_t lo = base, hi = lut + 0x10000u;
+  uint32_t misc;
+  if (lut - lo >= (uint32_t)MISC) {
+    misc = lo;
+    lo += MISC;
+  } else {
+    misc = hi;
+    hi += MISC;
+  }
+  const uint32_t ra = (lo + 1023u) & ~1023u, rb = (hi + 1023u) & ~1023u;
+  int SA = ra < lut ? (int)((lut - ra) / STAGE) : 0;
+  const int SB = rb < end ? (int)((end - rb) / STAGE) : 0;
+  const int S = min(kGsMaxStages, SA + SB);
+  SA = min(SA, S);
+  const uint32_t rb_adj = rb - (uint32_t)SA * STAGE;  // stage s >= SA at rb_adj + s * STAGE
+  if (S < 4 || hi > end) {  // not reachable with this launch's shared-memory size; refuse loudly
+    if (threadIdx.x == 0) raise_status(p.status, Q4_STATUS_LAYOUT);
+    return;
+  }
+  auto stage_addr = [&](int s) { return (s < SA ? ra : rb_adj) + (uint32_t)s * STAGE; };
+  const uint32_t scales = misc;  // bf16 only
+  const uint32_t bar0 = misc + (EXACT ? kGsScaleBytes : 0);
+  auto sfull = [&](int s) { return bar0 + 8u * s; };
+  auto sempty = [&](int s) { return bar0 + 8u * (kGsMaxStages + s); };
+  volatile int *abort = reinterpret_cast<volatile int *>(smem_raw + (bar0 + 16u * kGsMaxStages - base));
+  GsInfo *info = reinterpret_cast<GsInfo *>(smem_raw + (bar0 + kGsBarBytes - base));
+  // c~ buffer of 16-row group grp (0..15), parity sb, byte offset o < 1024:
+  // contiguous (bf16) or in the 128-byte gaps of the table (fp16)
+  auto scale_addr = [&](int grp, uint32_t sb, uint32_t o) -> uint32_t {
+    if constexpr (EXACT) return scales + ((uint32_t)grp * 2u + sb) * (uint32_t)kGsScaleBuf + o;
+    else return lut + 128u + (((uint32_t)grp * 2u + sb) * 8u + (o >> 7)) * 256u + (o & 127u);
+  };
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
-  const uint32_t bar0 = smem_u32(bars);
-  auto sfull = [&](int s) { return bar0 + 8u * s; };
-  auto sempty = [&](int s) { return bar0 + 8u * (S + s); };
-
-  if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(sfull(s), 1);
-      mbar_init(sempty(s), kGsWarps);
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    s_abort = 0;
-  }
-  for (int i = tid; i < 256 * 32; i += kGsThreads) {
-    const int b = i >> 5;
-    if constexpr (EXACT) reinterpret_cast<float2 *>(sLut)[i] = make_float2(p.levels[b & 15], p.levels[b >> 4]);
-    else reinterpret_cast<uint32_t *>(sLut)[i] = Dt<DA>::pack2(p.levels[b & 15], p.levels[b >> 4]);
-  }
-  __syncthreads();
-  volatile int *abort = &s_abort;
   const int M = p.M;
+  const uint32_t T = p.total_stages, G = gridDim.x;
+  const uint32_t g0 = gs_range_begin(blockIdx.x, T, G);  // this CTA's stages [g0, g1)
+  const uint32_t g1 = gs_range_begin(blockIdx.x + 1, T, G);
+  const bool dq = p.dq != 0;
+  if (tid < p.count) {
+    const GsMat &m = p.mat[tid];
+    GsInfo &d = info[tid];
+    d.stage_begin = m.stage_begin;
+    d.N = m.N;
+    d.K = m.K;
+    d.n_stages = m.n_stages;
+    d.absmax = m.absmax;
+    d.absmax_q = m.absmax_q;
+    d.absmax_scale = m.absmax_scale;
+    d.absmax_mean = m.absmax_mean;
+    d.Y = m.Y;
+    d.cnt = m.cnt;
+  }
+  if (warp == PRODUCER && lane == 0) {
+    for (int b = 0; b < S; ++b) {
+      mbar_init(sfull(b), 1);
+      mbar_init(sempty(b), WARPS);  // one arrival per compute warp
+    }
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();  // barriers and matrix fields ready
 
-  if (warp == kGsWarps) {
+  if (warp == PRODUCER) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t gs = 0;
-      bool sent = false;
-      unsigned next = atomicAdd(p.work, 1u);
-      for (uint32_t gu = 0;; ++gu) {
-        const unsigned u = next;
-        const bool last = u >= p.total_units;
-        if (!last) next = atomicAdd(p.work, 1u);  // claimed now, used one unit later
-        const int s0 = gs % S;
-        if (!mbar_wait(sempty(s0), ((gs / S) & 1) ^ 1, p.status, abort)) break;
-        sUnit[gu % S] = u;
-        if (last) {
-          mbar_arrive(sfull(s0));  // completes the phase without data: the end marker
-          sent = true;
-          break;
+      const uint32_t tx = (uint32_t)kGsWTile + 2u * 128u * (uint32_t)M;
+      int s = 0, mi = 0, issued = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (uint32_t gi = g0; gi < g1 && ok;) {
+        const GsUnit u = gs_describe<B>(info, p.count, mi, gi, g0, g1);
+        const GsMat &mt = p.mat[u.mi];
+        for (int q = u.q0; q < u.q1; ++q) {
+          if (!mbar_wait(sempty(s), ph ^ 1u, p.status, abort)) { ok = false; break; }
+          // the compute warps' reads of this slot (generic proxy) come before
+          // the copy that overwrites it (async proxy)
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(sfull(s), tx);
+          const uint32_t st = stage_addr(s);
+          tma_load_2d(st, &mt.tmA, sfull(s), q * kGsStageK, 0);
+          tma_load_2d(st + ATILE, &mt.tmA, sfull(s), q * kGsStageK + 64, 0);
+          tma_load_2d(st + 2 * ATILE, &mt.tmW, sfull(s), q * (kGsStageK / 2), u.tile * kGsRows);
+          ++issued;
+          if (++s == S) { s = 0; ph ^= 1u; }
         }
-        int mi = 0;
-        while (mi + 1 < p.count && (int64_t)u >= p.mat[mi + 1].unit_begin) ++mi;
-        const GsMat &mt = p.mat[mi];
-        const int64_t local = (int64_t)u - mt.unit_begin;
-        const int tile = (int)(local % mt.n_tiles), split = (int)(local / mt.n_tiles);
-        const int k0 = split * kGsUnitK;
-        const int nst = (min(kGsUnitK, mt.K - k0) + 63) / 64;
-        bool ok = true;
-        for (int t = 0; t < nst; ++t, ++gs) {
-          const int s = gs % S;
-          if (t > 0 && !mbar_wait(sempty(s), ((gs / S) & 1) ^ 1, p.status, abort)) { ok = false; break; }
-          mbar_arrive_expect_tx(sfull(s), STAGE);
-          uint8_t *st = sStage + s * STAGE;
-          tma_load_2d(smem_u32(st), &mt.tmA, sfull(s), k0 + t * 64, 0);
-          tma_load_2d(smem_u32(st + ATILE), &mt.tmW, sfull(s), (k0 + t * 64) / 2, tile * kGsRows);
-        }
-        if (!ok) break;
+        gi += (uint32_t)(u.q1 - u.q0);
       }
       if (*abort) {
-        // The compute warps may have left: let the copies still in flight land
-        // before the CTA exits (stages before gs - S were released, so complete).
-        for (uint32_t j = (gs > (uint32_t)S ? gs - S : 0u); j < gs; ++j) {
-          if (sent && j % S == gs % S) continue;  // that slot's last phase was the end marker
+        // The compute warps may have left: let the copies still in flight
+        // land before the CTA exits (older stages were released, so complete).
+        int ss = s;
+        uint32_t pp = ph;
+        for (int j = 0; j < min(issued, S); ++j) {
+          if (--ss < 0) { ss = S - 1; pp ^= 1u; }
           int dummy = 0;
           volatile int no_abort = 0;
-          mbar_wait(sfull(j % S), (j / S) & 1, &dummy, &no_abort);
+          mbar_wait(sfull(ss), pp, &dummy, &no_abort);
         }
-      }
-      // The producer that finishes last leaves both counters at 0 for the next launch.
-      __threadfence();
-      if (atomicAdd(p.work + 1, 1u) == gridDim.x - 1) {
-        p.work[0] = 0u;
-        p.work[1] = 0u;
-        __threadfence();
       }
     }
     return;
   }
 
   // -------------------------------------------------------------- compute warps
-  const uint32_t lb = smem_u32(sLut) + (EXACT ? 8u : 4u) * lane;
-  uint32_t gs = 0;
-  for (uint32_t gu = 0;; ++gu) {
+  // the first unit's c~ inputs are loaded before the table is built
+  int mi = 0;
+  GsScaleIn sin[R];
+  GsUnit u;
+  if (g0 < g1) {
+    u = gs_describe<B>(info, p.count, mi, g0, g0, g1);
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, u, (warp * R + rt) * 16, lane, sin[rt]);
+  }
+  for (int i = tid; i < 256 * 32; i += WARPS * 32) {
+    const int b = i >> 5, l = i & 31;
+    const uint32_t a = lut + (uint32_t)b * 256u + (uint32_t)l * ES;
+    if constexpr (EXACT) sts64(a, __float_as_uint(p.levels[b & 15]), __float_as_uint(p.levels[b >> 4]));
+    else sts32(a, Dt<DA>::pack2(p.levels[b & 15], p.levels[b >> 4]));
+  }
+  // the table is complete for every compute warp (the producer does not wait)
+  asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32) : "memory");
+
+  const uint32_t lb = lut + ES * (uint32_t)lane;
+  uint32_t sb = 0;  // c~ buffer parity
+  // partial tiles of this CTA awaiting their count: [0] the one holding the
+  // CTA's first stage, [1] the one holding its last
+  int pend_mi0 = -1, pend_tile0 = 0, pend_len0 = 0;
+  int pend_mi1 = -1, pend_tile1 = 0, pend_len1 = 0;
+  float acc[R][NT][4];
+  int qstart = 0;
+  uint32_t av[NT][SEGS][SEG / 8];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int sg = 0; sg < SEGS; ++sg)
+#pragma unroll
+      for (int i = 0; i < SEG / 8; ++i) av[nt][sg][i] = 0u;
+  }
+  int s = 0;
+  uint32_t ph = 0;
+
+  bool ok = true;
+#pragma unroll 1
+  for (uint32_t gi = g0; gi < g1;) {
+    // c~ of this unit into the next buffers (rewritten a unit after their last read)
     {
-      const int s0 = gs % S;
-      if (!mbar_wait_warp(sfull(s0), (gs / S) & 1, p.status, abort)) break;
+      const int r = lane & 15, blk0 = (lane >> 4) * 8;
+#pragma unroll
+      for (int rt = 0; rt < R; ++rt)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t o = (uint32_t)(((blk0 + j) * 8 + (r & 7)) * 2 + (r >> 3)) * 4u;
+          sts32(scale_addr(warp * R + rt, sb, o), __float_as_uint(gs_scale_value(sin[rt], dq, j)));
+        }
     }
-    const unsigned u = sUnit[gu % S];
-    if (u >= p.total_units) break;
-    int mi = 0;
-#pragma unroll 1
-    while (mi + 1 < p.count && (int64_t)u >= p.mat[mi + 1].unit_begin) ++mi;
-    const GsMat &mt = p.mat[mi];
-    const int64_t local = (int64_t)u - mt.unit_begin;
-    const int tile = (int)(local % mt.n_tiles), split = (int)(local / mt.n_tiles);
+    __syncwarp();
+    uint32_t srd[R];  // this lane's (row g, row g+8) pair of block 0, per row group
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) srd[rt] = scale_addr(warp * R + rt, sb, (uint32_t)g * 8u);
+    sb ^= 1u;
+    const GsUnit cu = u;
+    const uint32_t gn = gi + (uint32_t)(cu.q1 - cu.q0);
+    if (gn < g1) {  // next unit: issue its c~ loads now, use them a unit later
+      u = gs_describe<B>(info, p.count, mi, gn, g0, g1);
+#pragma unroll
+      for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, u, (warp * R + rt) * 16, lane, sin[rt]);
+    }
+    const GsInfo &mt = info[cu.mi];
     const int K = mt.K, N = mt.N;
-    const int k0 = split * kGsUnitK;
-    const int klen = min(kGsUnitK, K - k0);
-    const int nst = (klen + 63) / 64;
-    const int nbk = K / B;
-    const int blk0 = k0 / B;
-    const int nblk = (klen + B - 1) / B;
-    const int r_base = tile * kGsRows + warp * 16;
-
-    // ---- block scales of this lane's rows g, g+8 for the unit
-    uint32_t q2w[2][QW];
-    float s2a[2], s2b[2], mu = 0.0f;
-    int bsplit[2];
-    const bool dq = p.dq != 0;
-    if (dq) mu = __ldg(mt.absmax_mean);
+    if (cu.first) {
+      qstart = cu.q0;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row = min(r_base + h * 8 + g, N - 1);
-      const int64_t bi0 = (int64_t)row * nbk + blk0;
-      if (dq) {
-        const int64_t g0 = bi0 >> 8;
-        s2a[h] = __ldg(mt.absmax_scale + g0);
-        s2b[h] = __ldg(mt.absmax_scale + ((bi0 + nblk - 1) >> 8));
-        bsplit[h] = (int)(((g0 + 1) << 8) - bi0);
-        if (((bi0 & 3) == 0) && nblk == UB) {
+      for (int rt = 0; rt < R; ++rt)
 #pragma unroll
-          for (int qw = 0; qw < QW; ++qw) q2w[h][qw] = __ldg(reinterpret_cast<const unsigned int *>(mt.absmax_q + bi0) + qw);
-        } else {
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int qw = 0; qw < QW; ++qw) {
-            uint32_t v = 0;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (4 * qw + e < nblk) v |= (uint32_t)(uint8_t)__ldg(mt.absmax_q + bi0 + 4 * qw + e) << (8 * e);
-            q2w[h][qw] = v;
-          }
-        }
-      }
+          for (int j = 0; j < 4; ++j) acc[rt][nt][j] = 0.0f;
     }
-    // Scales of the unit's blocks in order: the int8 codes are consumed from
-    // the front of q2w (register moves only, no dynamic register indexing).
-    int bi = 0;  // next block of the unit
-    float sc0 = 0.0f, sc1 = 0.0f;
-    auto next_scales = [&]() {
-      float v[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (dq) {
-          const int code = (int)(int8_t)(q2w[h][0] & 0xFFu);
-          const float s2 = (bi < bsplit[h]) ? s2a[h] : s2b[h];
-          v[h] = __fadd_rn(__fmul_rn((float)code, s2), mu);
-          q2w[h][0] >>= 8;
-          if ((bi & 3) == 3) {
-#pragma unroll
-            for (int qw = 0; qw + 1 < QW; ++qw) q2w[h][qw] = q2w[h][qw + 1];
-          }
-        } else {
-          const int row = min(r_base + h * 8 + g, N - 1);
-          v[h] = __ldg(mt.absmax + (int64_t)row * nbk + blk0 + bi);
-        }
-      }
-      sc0 = v[0];
-      sc1 = v[1];
-      ++bi;
-    };
+    const int w_base = cu.tile * kGsRows + warp * 16 * R;  // first row of this warp
 
-    float acc[NT][4], part[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[nt][j] = part[nt][j] = 0.0f;
-
-    bool ok = true;
 #pragma unroll 1
-    for (int t = 0; t < nst; ++t, ++gs) {
-      const int s = gs % S;
-      if (t > 0 && !mbar_wait_warp(sfull(s), (gs / S) & 1, p.status, abort)) { ok = false; break; }
-      const uint32_t st = smem_u32(sStage + s * STAGE);
-      // packed bytes of rows g and g+8 of this warp's tile (32 bytes per row)
-      uint32_t wv[2][2 * SEGS];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t ra = st + ATILE + (warp * 16 + h * 8 + g) * 32;
-        if constexpr (SEG == 64) {
-          const uint2 v = lds64(ra + tig * 8);
-          wv[h][0] = v.x;
-          wv[h][1] = v.y;
-        } else {
-#pragma unroll
-          for (int sg = 0; sg < SEGS; ++sg) wv[h][sg] = lds32(ra + sg * 16 + tig * 4);
-        }
+    for (int q = cu.q0; q < cu.q1; ++q) {
+      // lane 0 waits for the copy (acquire); the shuffle keeps the other
+      // lanes' reads of the stage after it
+      {
+        bool ready = true;
+        if (lane == 0) ready = mbar_wait(sfull(s), ph, p.status, abort);
+        if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) { ok = false; break; }
       }
-      // activation rows nt*8 + g: halves [seg*SEG + tig*SEG/4, + SEG/4), 128-byte swizzle
-      uint32_t av[NT][SEGS][SEG / 8];
+      const uint32_t st = stage_addr(s);
+      // packed bytes of rows g and g+8 of each row group (64 bytes per row);
+      // segment sg of a row is bytes [sg * SEG / 2, + SEG / 2), a lane's
+      // share of it the tig-th quarter
+      uint32_t wv[R][2][WV];
+#pragma unroll
+      for (int rt = 0; rt < R; ++rt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t ra_ = st + 2 * ATILE + (uint32_t)(warp * 16 * R + rt * 16 + h * 8 + g) * (kGsStageK / 2);
+#pragma unroll
+          for (int sg = 0; sg < SEGS; ++sg) {
+            if constexpr (SEG == 64) {
+              const uint2 v = lds64v(ra_ + sg * 32 + tig * 8);
+              wv[rt][h][2 * sg] = v.x;
+              wv[rt][h][2 * sg + 1] = v.y;
+            } else {
+              wv[rt][h][sg] = lds32v(ra_ + sg * 16 + tig * 4);
+            }
+          }
+        }
+      // activation rows nt*8 + g (< M only; the rest stay zero): 128-byte swizzle
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int ar = nt * 8 + g;
-        const uint32_t aa = st + ar * 128;
+        if (ar < M) {
 #pragma unroll
-        for (int sg = 0; sg < SEGS; ++sg) {
-          if constexpr (SEG == 64) {
-            const uint4 x0 = lds128(aa + (((2 * tig) ^ (ar & 7)) << 4));
-            const uint4 x1 = lds128(aa + (((2 * tig + 1) ^ (ar & 7)) << 4));
-            av[nt][sg][0] = x0.x; av[nt][sg][1] = x0.y; av[nt][sg][2] = x0.z; av[nt][sg][3] = x0.w;
-            av[nt][sg][4] = x1.x; av[nt][sg][5] = x1.y; av[nt][sg][6] = x1.z; av[nt][sg][7] = x1.w;
-          } else {
-            const uint4 x0 = lds128(aa + (((sg * 4 + tig) ^ (ar & 7)) << 4));
-            av[nt][sg][0] = x0.x; av[nt][sg][1] = x0.y; av[nt][sg][2] = x0.z; av[nt][sg][3] = x0.w;
+          for (int sg = 0; sg < SEGS; ++sg) {
+            const uint32_t aa = st + (uint32_t)(sg / SPH) * ATILE + (uint32_t)ar * 128u;  // the segment's half
+            const int sgh = sg % SPH;
+            if constexpr (SEG == 64) {
+              const uint4 x0 = lds128v(aa + (((2 * tig) ^ (ar & 7)) << 4));
+              const uint4 x1 = lds128v(aa + (((2 * tig + 1) ^ (ar & 7)) << 4));
+              av[nt][sg][0] = x0.x; av[nt][sg][1] = x0.y; av[nt][sg][2] = x0.z; av[nt][sg][3] = x0.w;
+              av[nt][sg][4] = x1.x; av[nt][sg][5] = x1.y; av[nt][sg][6] = x1.z; av[nt][sg][7] = x1.w;
+            } else {
+              const uint4 x0 = lds128v(aa + (((sgh * 4 + tig) ^ (ar & 7)) << 4));
+              av[nt][sg][0] = x0.x; av[nt][sg][1] = x0.y; av[nt][sg][2] = x0.z; av[nt][sg][3] = x0.w;
+            }
           }
         }
       }
+
 #pragma unroll
       for (int sg = 0; sg < SEGS; ++sg) {
-        const int kseg = t * 64 + sg * SEG;          // k offset of the segment in the unit
-        if (kseg >= klen) break;
-        if (kseg % B == 0) next_scales();
+        if (q * kGsStageK + sg * SEG >= K) break;
+        // block of this segment within the 16-block window
+        const int bw = ((q * kGsStageK + sg * SEG) / B) & (kGsWinBlocks - 1);
+        const uint32_t soff = EXACT ? (uint32_t)bw * 64u : (uint32_t)(bw >> 1) * 256u + (uint32_t)(bw & 1) * 64u;
 #pragma unroll
-        for (int q = 0; q < STEPS; ++q) {
-          // bytes 2q, 2q+1 of the lane's LB bytes of this segment
-          const int b0 = (sg * LB + 2 * q), b1 = b0 + 1;
-          const uint32_t w00 = wv[0][b0 >> 2], w10 = wv[1][b0 >> 2];
-          uint32_t a0, a1, a2, a3;
-          if constexpr (EXACT) {
-            const float2 e0 = lds64f(lut_addr<8>(w00, b0 & 3, lb));
-            const float2 e1 = lds64f(lut_addr<8>(w10, b0 & 3, lb));
-            const float2 e2 = lds64f(lut_addr<8>(w00, b1 & 3, lb));
-            const float2 e3 = lds64f(lut_addr<8>(w10, b1 & 3, lb));
-            a0 = Dt<DA>::pack2(__fmul_rn(sc0, e0.x), __fmul_rn(sc0, e0.y));
-            a1 = Dt<DA>::pack2(__fmul_rn(sc1, e1.x), __fmul_rn(sc1, e1.y));
-            a2 = Dt<DA>::pack2(__fmul_rn(sc0, e2.x), __fmul_rn(sc0, e2.y));
-            a3 = Dt<DA>::pack2(__fmul_rn(sc1, e3.x), __fmul_rn(sc1, e3.y));
-          } else {
-            a0 = lds32(lut_addr<7>(w00, b0 & 3, lb));
-            a1 = lds32(lut_addr<7>(w10, b0 & 3, lb));
-            a2 = lds32(lut_addr<7>(w00, b1 & 3, lb));
-            a3 = lds32(lut_addr<7>(w10, b1 & 3, lb));
+        for (int rt = 0; rt < R; ++rt) {
+          const float2 sc = lds64fv(srd[rt] + soff);
+          float part[NT][4];
+#pragma unroll
+          for (int qq = 0; qq < STEPS; ++qq) {
+            // bytes 2qq, 2qq+1 of the lane's LB bytes of this segment
+            const int b0 = sg * LB + 2 * qq, b1 = b0 + 1;
+            const uint32_t w0 = wv[rt][0][b0 >> 2], w1 = wv[rt][1][b0 >> 2];
+            uint32_t a0, a1, a2, a3;
+            if constexpr (EXACT) {
+              const float2 e0 = lut64f(lut_addr(w0, b0 & 3, lb));
+              const float2 e1 = lut64f(lut_addr(w1, b0 & 3, lb));
+              const float2 e2 = lut64f(lut_addr(w0, b1 & 3, lb));
+              const float2 e3 = lut64f(lut_addr(w1, b1 & 3, lb));
+              a0 = Dt<DA>::pack2(__fmul_rn(sc.x, e0.x), __fmul_rn(sc.x, e0.y));
+              a1 = Dt<DA>::pack2(__fmul_rn(sc.y, e1.x), __fmul_rn(sc.y, e1.y));
+              a2 = Dt<DA>::pack2(__fmul_rn(sc.x, e2.x), __fmul_rn(sc.x, e2.y));
+              a3 = Dt<DA>::pack2(__fmul_rn(sc.y, e3.x), __fmul_rn(sc.y, e3.y));
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt)
+                MmaS<DA>::run(acc[rt][nt], a0, a1, a2, a3, av[nt][sg][2 * qq], av[nt][sg][2 * qq + 1]);
+            } else {
+              a0 = lut32(lut_addr(w0, b0 & 3, lb));
+              a1 = lut32(lut_addr(w1, b0 & 3, lb));
+              a2 = lut32(lut_addr(w0, b1 & 3, lb));
+              a3 = lut32(lut_addr(w1, b1 & 3, lb));
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                if (qq == 0) MmaS<DA>::run0(part[nt], a0, a1, a2, a3, av[nt][sg][0], av[nt][sg][1]);
+                else MmaS<DA>::run(part[nt], a0, a1, a2, a3, av[nt][sg][2 * qq], av[nt][sg][2 * qq + 1]);
+              }
+            }
           }
+          if constexpr (!EXACT) {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            MmaS<DA>::run(EXACT ? acc[nt] : part[nt], a0, a1, a2, a3, av[nt][sg][2 * q], av[nt][sg][2 * q + 1]);
-        }
-        if (!EXACT && (((kseg + SEG) % B) == 0 || kseg + SEG >= klen)) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            acc[nt][0] = fmaf(sc0, part[nt][0], acc[nt][0]);
-            acc[nt][1] = fmaf(sc0, part[nt][1], acc[nt][1]);
-            acc[nt][2] = fmaf(sc1, part[nt][2], acc[nt][2]);
-            acc[nt][3] = fmaf(sc1, part[nt][3], acc[nt][3]);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) part[nt][j] = 0.0f;
+            for (int nt = 0; nt < NT; ++nt) {
+              acc[rt][nt][0] = fmaf(sc.x, part[nt][0], acc[rt][nt][0]);
+              acc[rt][nt][1] = fmaf(sc.x, part[nt][1], acc[rt][nt][1]);
+              acc[rt][nt][2] = fmaf(sc.y, part[nt][2], acc[rt][nt][2]);
+              acc[rt][nt][3] = fmaf(sc.y, part[nt][3], acc[rt][nt][3]);
+            }
           }
         }
       }
-      // Release the stage only now: the MMAs above have consumed every value
-      // loaded from it, so none of those shared-memory reads can still be in
-      // flight when the producer's next copy overwrites the slot (an arrive
-      // issued right after the loads may overtake them).
+      // Release the stage after the MMAs, which consumed every value read
+      // from it: no read of the slot can still be pending when the next copy
+      // overwrites it (an arrive issued right after the loads may overtake
+      // them).  __syncwarp orders all lanes' reads before lane 0's arrive.
       __syncwarp();
       if (lane == 0) mbar_arrive(sempty(s));
+      if (++s == S) { s = 0; ph ^= 1u; }
     }
     if (!ok) break;
 
-    // ---- D fragment: rows g / g+8, columns m = nt*8 + 2 tig + {0, 1}
-    if (mt.n_splits == 1) {
+    if (cu.last) {
+      const int Q = mt.n_stages;
+      if (qstart == 0 && cu.q1 == Q) {
+        // the whole k range of these rows went through this warp
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+        for (int rt = 0; rt < R; ++rt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = r_base + (j >> 1) * 8 + g;
-          const int m = nt * 8 + 2 * tig + (j & 1);
-          if (m < M && row < N) gs_store(mt.Y, p.y_dtype, (int64_t)m * N + row, acc[nt][j]);
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int row = w_base + rt * 16 + (j >> 1) * 8 + g;
+              const int m = nt * 8 + 2 * tig + (j & 1);
+              if (m < M && row < N) gs_store(mt.Y, p.y_dtype, (int64_t)m * N + row, acc[rt][nt][j]);
+            }
+      } else if (w_base < N) {
+        // a partial tile: its rows go to this CTA's slot for the role
+        const bool role0 = gi - (uint32_t)(cu.q0 - qstart) == g0;  // the segment holds the CTA's first stage
+        float *slot = p.slots + ((int64_t)(blockIdx.x * 2 + (role0 ? 0 : 1)) * kGsRows + warp * 16 * R + g) * MW + 2 * tig;
+#pragma unroll
+        for (int rt = 0; rt < R; ++rt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              __stcg(reinterpret_cast<float2 *>(slot + (rt * 16 + h * 8) * MW + nt * 8),
+                     make_float2(acc[rt][nt][2 * h], acc[rt][nt][2 * h + 1]));
+        if (role0) {
+          pend_mi0 = cu.mi; pend_tile0 = cu.tile; pend_len0 = cu.q1 - qstart;
+        } else {
+          pend_mi1 = cu.mi; pend_tile1 = cu.tile; pend_len1 = cu.q1 - qstart;
         }
-    } else if (r_base < N) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = r_base + (j >> 1) * 8 + g;
-          const int m = nt * 8 + 2 * tig + (j & 1);
-          if (m < M && row < N) atomicAdd(mt.acc + (int64_t)row * M + m, acc[nt][j]);
-        }
-      __threadfence();
-      const int sub = r_base / 16;  // 16-row counter index
-      unsigned ticket = 0;
-      if (lane == 0) ticket = atomicAdd(mt.cnt + sub, 1u);
-      ticket = __shfl_sync(0xffffffffu, ticket, 0);
-      if (ticket == (unsigned)(mt.n_splits - 1)) {
-        __threadfence();
-        const int rows = min(16, N - r_base);
-        for (int idx = lane; idx < rows * M; idx += 32) {
-          const int m = idx / rows, r = idx - m * rows;
-          float *ap = mt.acc + (int64_t)(r_base + r) * M + m;
-          const float v = __ldcg(ap);
-          __stcg(ap, 0.0f);
-          gs_store(mt.Y, p.y_dtype, (int64_t)m * N + r_base + r, v);
-        }
-        if (lane == 0) mt.cnt[sub] = 0u;
       }
+    }
+    gi = gn;
+  }
+  if (!ok || (pend_mi0 < 0 && pend_mi1 < 0)) return;
+
+  // ---- count this CTA's partial tiles; finish every 16-row group it completes
+  fence_acq_rel_gpu();  // this thread's slot stores are visible before its count
+  __syncwarp();
+#pragma unroll
+  for (int rl = 0; rl < 2; ++rl) {
+    const int pmi = rl ? pend_mi1 : pend_mi0;
+    if (pmi < 0) continue;
+    const GsInfo &mt = info[pmi];
+    const int N = mt.N, Q = mt.n_stages;
+    const int tile = rl ? pend_tile1 : pend_tile0;
+    const unsigned len = (unsigned)(rl ? pend_len1 : pend_len0);
+    const uint32_t x0 = mt.stage_begin + (uint32_t)(tile * Q);  // the tile's first stage
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) {
+      const int r_base = tile * kGsRows + warp * 16 * R + rt * 16;
+      if (r_base >= N) continue;
+      unsigned old = 0;
+      if (lane == 0) old = atomicAdd(mt.cnt + (r_base >> 4), len);
+      old = __shfl_sync(0xffffffffu, old, 0);
+      if (old + len != (unsigned)Q) continue;
+      // every contributor has counted: sum their slots in CTA order
+      __syncwarp();
+      fence_acq_rel_gpu();
+      const int c0 = gs_cta_of(x0, T, G), c1 = gs_cta_of(x0 + Q - 1, T, G);
+      float sum[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sum[nt][j] = 0.0f;
+      for (int c = c0; c <= c1; ++c) {
+        const int role = (gs_range_begin(c, T, G) >= x0) ? 0 : 1;  // c starts inside the tile
+        float *slot = p.slots + ((int64_t)(c * 2 + role) * kGsRows + warp * 16 * R + rt * 16 + g) * MW + 2 * tig;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float2 *sp = reinterpret_cast<float2 *>(slot + (h * 8) * MW + nt * 8);
+            const float2 v = __ldcg(sp);
+            __stcg(sp, make_float2(0.0f, 0.0f));  // the workspace is left zeroed
+            sum[nt][2 * h] += v.x;
+            sum[nt][2 * h + 1] += v.y;
+          }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = r_base + (j >> 1) * 8 + g;
+          const int m = nt * 8 + 2 * tig + (j & 1);
+          if (m < M && row < N) gs_store(mt.Y, p.y_dtype, (int64_t)m * N + row, sum[nt][j]);
+        }
+      if (lane == 0) mt.cnt[r_base >> 4] = 0u;
     }
   }
 }

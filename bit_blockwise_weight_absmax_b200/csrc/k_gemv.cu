@@ -55,35 +55,24 @@ int by_bs(int bs, int mp, const GvParams &p, int sms, cudaStream_t st) {
   }
   return Q4_ERR_ARG;
 }
-// Stages of the mma.sync kernel's ring: as many as fit two CTAs per SM
-// (228 KB per SM, 1 KB reserved per CTA), at most 12.
-template <int DA, int NT>
-constexpr int small_stages() {
-  constexpr int STAGE = kGsWTile + 8 * NT * 128;
-  constexpr int LUTB = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
-  constexpr int budget = (228 * 1024) / 2 - 1024 - LUTB - 1024 - 64;
-  constexpr int s = budget / (STAGE + 20);
-  return s < 12 ? s : 12;
-}
+// The mma.sync kernel: one CTA per SM with all of its shared memory (the
+// kernel lays out its table, buffers and ring itself).
 template <int DA, int NT, int B>
 int go_small(const GsParams &p, int sms, cudaStream_t st) {
-  constexpr int S = small_stages<DA, NT>();
-  static_assert(S >= 4, "ring too small");
-  constexpr int STAGE = kGsWTile + 8 * NT * 128;
-  constexpr int LUTB = 256 * 32 * (DA == Q4_BF16 ? 8 : 4);
-  constexpr int SMEM = S * STAGE + LUTB + 2 * S * 8 + S * 4 + 1024;
-  static_assert(2 * (SMEM + 1024 + 64) <= 228 * 1024, "two CTAs per SM");
-  auto kern = gemv_small_kernel<DA, NT, B, S>;
+  // 16-row groups per compute warp: M <= 8 fits 16 compute warps (+ the
+  // producer) in the registers; M <= 16 uses 8 warps of 32 rows
+  constexpr int R = NT == 1 ? 1 : 2;
+  auto kern = gemv_small_kernel<DA, NT, B, R>;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess ||
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGsSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return Q4_ERR_CUDA;
     attr = true;
   }
-  const int grid = (int)std::min<int64_t>(p.total_units, (int64_t)sms * 2);
-  kern<<<grid, kGsThreads, SMEM, st>>>(p);
+  const int grid = (int)std::min<int64_t>(p.total_stages, (int64_t)std::min(sms, kGsMaxCtas));
+  kern<<<grid, GsShape<R>::kThreads, kGsSmemBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 template <int DA, int NT>

@@ -135,18 +135,25 @@ int check_state(const q4_state *s) {
 }
 
 // ---- GEMV planning ----------------------------------------------------------
-// Units of 128 rows x 1024 k for both kernels (mma.sync for M <= 16, tcgen05
-// above).  Workspace: two work counters, then per split matrix fp32 [N][M]
-// partial sums and the arrival counters (one per 16 rows for the mma.sync
-// kernel, one per tile for the tcgen05 kernel).
+// M <= 16 (mma.sync kernel): 256-row tiles cut into 128-k stages, the stages
+// of all matrices split evenly over at most kGsMaxCtas CTAs; workspace: a
+// 256-byte head, the per-CTA partial-row slots, then per matrix one counter
+// per 16 rows.  M > 16 (tcgen05 kernel): units of 128 rows x 1024 k;
+// workspace: the head (work counters), then per split matrix fp32 [N][M]
+// partial sums and one counter per 128-row tile.
 constexpr size_t kGemvWsHead = 256;
 size_t gemv_ws_for(const q4_state *s, int64_t M, int64_t *n_tiles, int64_t *n_splits) {
   const bool small = M <= 16;
   *n_tiles = ceil_div(s->rows, small ? kGsRows : kGvRows);
-  *n_splits = ceil_div(s->cols, small ? kGsUnitK : kGvUnitK);
+  *n_splits = ceil_div(s->cols, small ? kGsStageK : kGvUnitK);  // small: stages per tile
+  if (small) return align256((size_t)ceil_div(s->rows, 16) * 4);
   if (*n_splits <= 1) return 0;
-  const int64_t counters = small ? ceil_div(s->rows, 16) : *n_tiles;
-  return align256((size_t)s->rows * (size_t)M * 4) + align256((size_t)counters * 4);
+  return align256((size_t)s->rows * (size_t)M * 4) + align256((size_t)*n_tiles * 4);
+}
+// Slots of the mma.sync kernel: [grid][2][256 rows][8 or 16] fp32.
+size_t gemv_small_slots(int64_t total_stages, int64_t M) {
+  const int64_t grid = std::min<int64_t>(total_stages, kGsMaxCtas);
+  return align256((size_t)grid * 2 * kGsRows * (M <= 8 ? 8 : 16) * 4);
 }
 int pow2_at_least(int64_t m) {
   int p = 1;
@@ -190,7 +197,7 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
 int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *const *Wq, void *const *Y,
                        int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace, size_t workspace_bytes,
                        void *stream) {
-  static thread_local GsParams p;
+  static thread_local GsParams p;  // host staging of the kernel parameters (~6 KB)
   memset(&p, 0, sizeof(p));
   p.count = count;
   p.M = (int)M;
@@ -199,8 +206,17 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
   const int dq = Wq[0]->double_quant;
   const DeviceInfo di = device_info();
   if (!workspace || workspace_bytes < kGemvWsHead) return Q4_ERR_WORKSPACE;
-  int64_t units = 0;
-  size_t ws_off = kGemvWsHead;
+  int64_t total = 0;
+  for (int i = 0; i < count; ++i) {
+    int64_t t, q;
+    gemv_ws_for(Wq[i], M, &t, &q);
+    total += t * q;
+  }
+  const size_t slot_bytes = gemv_small_slots(total, M);
+  int64_t stages = 0;
+  size_t ws_off = kGemvWsHead + slot_bytes;
+  if (ws_off > workspace_bytes) return Q4_ERR_WORKSPACE;
+  p.slots = reinterpret_cast<float *>((char *)workspace + kGemvWsHead);
   for (int i = 0; i < count; ++i) {
     const q4_state *s = Wq[i];
     int rc = check_state(s);
@@ -210,40 +226,34 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
     if (!A[i] || !Y[i]) return Q4_ERR_ARG;
     if (!aligned16(A[i])) return Q4_ERR_ALIGN;
     if (di.ok != Q4_OK) return di.ok;
-    int64_t n_tiles, n_splits;
-    const size_t need = gemv_ws_for(s, M, &n_tiles, &n_splits);
+    int64_t n_tiles, n_stages;
+    const size_t need = gemv_ws_for(s, M, &n_tiles, &n_stages);
+    if (n_tiles * n_stages > INT32_MAX) return Q4_ERR_SHAPE;
     GsMat &m = p.mat[i];
     const CUtensorMapDataType adt =
         a_dtype == Q4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (!make_map(&m.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1, 32, kGsRows,
+    if (!make_map(&m.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1, kGsStageK / 2, kGsRows,
                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&m.tmA, adt, A[i], M, s->cols, 2, 64, M <= 8 ? 8 : 16, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map(&m.tmA, adt, A[i], M, s->cols, 2, 64, (int)M, CU_TENSOR_MAP_SWIZZLE_128B))
       return Q4_ERR_CUDA;
-    m.packed = s->packed;
     m.absmax = s->absmax;
     m.absmax_q = s->absmax_q;
     m.absmax_scale = s->absmax_scale;
     m.absmax_mean = s->absmax_mean;
-    m.A = reinterpret_cast<const uint16_t *>(A[i]);
     m.Y = Y[i];
     m.N = (int32_t)s->rows;
     m.K = (int32_t)s->cols;
     m.n_tiles = (int32_t)n_tiles;
-    m.n_splits = (int32_t)n_splits;
-    m.unit_begin = units;
-    units += n_tiles * n_splits;
-    if (need) {
-      if (ws_off + need > workspace_bytes) return Q4_ERR_WORKSPACE;
-      m.acc = reinterpret_cast<float *>((char *)workspace + ws_off);
-      m.cnt = reinterpret_cast<unsigned *>((char *)workspace + ws_off +
-                                           align256((size_t)s->rows * (size_t)M * 4));
-      ws_off += need;
-    }
+    m.n_stages = (int32_t)n_stages;
+    m.stage_begin = (uint32_t)stages;
+    stages += n_tiles * n_stages;
+    if (stages * kGsMaxCtas >= ((int64_t)1 << 32)) return Q4_ERR_SHAPE;  // 32-bit stage indices
+    if (ws_off + need > workspace_bytes) return Q4_ERR_WORKSPACE;
+    m.cnt = reinterpret_cast<unsigned *>((char *)workspace + ws_off);
+    ws_off += need;
   }
-  if (units > UINT32_MAX / 2) return Q4_ERR_SHAPE;
   p.dq = dq;
-  p.total_units = units;
-  p.work = reinterpret_cast<unsigned *>(workspace);
+  p.total_stages = (uint32_t)stages;
   p.status = di.status;
   memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
   return run_gemv_small(a_dtype, bs, (int)M, p, di.sms, (cudaStream_t)stream);
@@ -401,12 +411,15 @@ int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
   if (!bytes || !Wq || count < 1 || count > kGvMaxGroup) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
   size_t total = kGemvWsHead;
+  int64_t stages = 0;
   for (int i = 0; i < count; ++i) {
     if (!Wq[i]) return Q4_ERR_ARG;
     if (!valid_bs(Wq[i]->blocksize) || Wq[i]->cols % Wq[i]->blocksize) return Q4_ERR_SHAPE;
     int64_t t, s;
     total += gemv_ws_for(Wq[i], M, &t, &s);
+    stages += t * s;
   }
+  if (M <= 16) total += gemv_small_slots(stages, M);
   *bytes = total;
   return Q4_OK;
 }

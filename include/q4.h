@@ -69,6 +69,7 @@ extern "C" {
 /* Sticky device status bits (q4_device_status). */
 #define Q4_STATUS_NONFINITE 1  /* quantize met a block with a non-finite absmax */
 #define Q4_STATUS_TIMEOUT 2    /* a bounded device-side wait gave up */
+#define Q4_STATUS_LAYOUT 4     /* a kernel found too little shared memory and computed nothing */
 
 /* ---- enums ------------------------------------------------------------- */
 typedef enum {

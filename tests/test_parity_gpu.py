@@ -223,3 +223,21 @@ def test_gemv_repeat_calls_agree(q4, oracle):
     torch.cuda.synchronize()
     d = (y1.float() - y2.float()).abs().max().item()
     assert d <= 1e-3 * y1.float().abs().max().item()
+
+
+def test_gemv_workspace_reuse_across_batch_sizes(q4, oracle):
+    """One cached workspace serves every batch size in turn: each call leaves
+    it zeroed, so a later call of another M (a different layout of partial
+    sums and counters) still gets the right answer."""
+    g = torch.Generator().manual_seed(8)
+    N, K = 1024, 11008
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    st = q4.quantize(dev(W), 64, "nf4", True)
+    ost = oracle_state(oracle, W, 64, 0, True)
+    rows = np.arange(0, N, 7)
+    w16 = oracle.dequantize(ost, False).reshape(N, K)[rows]
+    for M in (16, 1, 32, 8, 17, 4, 16, 1):
+        A = torch.randn(M, K, generator=g).half()
+        y = q4.gemv(dev(A), st)
+        ref = oracle.matmul(bits(A), False, w16, False, M, len(rows), K)
+        assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
