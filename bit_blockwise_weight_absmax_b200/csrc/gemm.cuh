@@ -10,17 +10,21 @@
 // into shared memory and consumed there by the tensor cores, so the 16-bit
 // weight matrix never exists in HBM.
 //
-// Design (one CTA per SM, persistent over output tiles of 256 x 256):
+// Design (one CTA per SM, persistent over output tiles of 256 x 128, m-tiles
+// fastest so that neighbouring CTAs share a weight tile in L2):
 //   warp 0      TMA producer: the A tile [256 x 64] (128B-swizzled, K-major)
-//               and the raw packed tile [256 rows x 32 bytes] per k-block.
+//               and the raw packed tile [128 rows x 32 bytes] per k-block,
+//               into a ring of 4 stages.
 //   warp 1      TMEM allocator and MMA issuer: per k-block 2 x 4
-//               tcgen05.mma kind::f16 (M=128, N=256, K=16) into two fp32
-//               accumulators (512 TMEM columns), committed to the stage's
-//               "empty" barrier.
-//   warps 4..11 dequant: thread d expands weight row d of the tile (64 codes)
-//               with its block scale into bf16/fp16 and writes it in the
-//               128B-swizzled K-major layout the UMMA descriptor reads; then
-//               the epilogue: tcgen05.ld of the accumulators, convert, store.
+//               tcgen05.mma kind::f16 (M=128, N=128, K=16) into two fp32
+//               accumulators of 128 columns; the two accumulator sets of a
+//               tile alternate between tiles (512 TMEM columns), so the
+//               epilogue of one tile overlaps the MMAs of the next.
+//   warps 2..17 dequant: four threads per weight row, 16 codes each, scaled
+//               by the row's block scale into bf16/fp16 and written in the
+//               128B-swizzled K-major layout the UMMA descriptor reads; the
+//               block scales come 16 blocks per load.  Then the epilogue:
+//               tcgen05.ld of the accumulators, convert, store.
 // Every mbarrier wait is bounded in time; a timeout sets Q4_STATUS_TIMEOUT,
 // stops the pipeline, waits for issued copies and frees TMEM.
 #pragma once
@@ -31,15 +35,17 @@
 namespace q4 {
 
 constexpr int kGemmBM = 256;
-constexpr int kGemmBN = 256;
+constexpr int kGemmBN = 128;
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 3;
-constexpr int kGemmThreads = 384;
+constexpr int kGemmStages = 4;
+constexpr int kGemmDqWarps = 16;                          // dequant + epilogue warps (2..17)
+constexpr int kGemmThreads = (2 + kGemmDqWarps) * 32;
 constexpr int kGemmATile = kGemmBM * kGemmBK * 2;   // 32 KB
-constexpr int kGemmBTile = kGemmBN * kGemmBK * 2;   // 32 KB
-constexpr int kGemmRawTile = kGemmBN * kGemmBK / 2; // 8 KB
+constexpr int kGemmBTile = kGemmBN * kGemmBK * 2;   // 16 KB
+constexpr int kGemmRawTile = kGemmBN * kGemmBK / 2; // 4 KB
 constexpr int kGemmStageBytes = kGemmATile + kGemmBTile + kGemmRawTile;
-constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kGemmScBytes = kGemmBN * 16 * 4;     // c~ of 16 blocks per weight row
+constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmScBytes + 1024 /*align*/ + 256 /*barriers*/;
 
 struct alignas(64) GemmMat {
   CUtensorMap tmA;  // A [M, K] 16-bit, box {64, 256}, 128B swizzle
@@ -136,6 +142,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -206,15 +217,17 @@ __device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t t) {
   return TileCoord{mi, (int)(local % tm_count), (int)(local / tm_count)};
 }
 
-template <int DA>
+// DA: activation dtype; DQ: double-quantized block scales.
+template <int DA, bool DQ>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sA = smem;                                        // [stages][32 KB]
-  uint8_t *sB = smem + kGemmStages * kGemmATile;             // [stages][32 KB]
-  uint8_t *sR = sB + kGemmStages * kGemmBTile;               // [stages][8 KB]
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sR + kGemmStages * kGemmRawTile);
-  // bars: full[S], bfull[S], empty[S], accfull, accempty
+  uint8_t *sB = smem + kGemmStages * kGemmATile;             // [stages][16 KB]
+  uint8_t *sR = sB + kGemmStages * kGemmBTile;               // [stages][4 KB]
+  float *sSc = reinterpret_cast<float *>(sR + kGemmStages * kGemmRawTile);  // [128 rows][16]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sSc) + kGemmScBytes);
+  // bars: full[S], bfull[S], empty[S], accfull[2], accempty[2]
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ float s_lv[16 * 32];
@@ -224,17 +237,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto bfull_bar = [&](int s) { return bar0 + 8u * (kGemmStages + s); };
   auto empty_bar = [&](int s) { return bar0 + 8u * (2 * kGemmStages + s); };
-  const uint32_t accfull_bar = bar0 + 8u * (3 * kGemmStages);
-  const uint32_t accempty_bar = bar0 + 8u * (3 * kGemmStages + 1);
+  auto accfull_bar = [&](int b) { return bar0 + 8u * (3 * kGemmStages + b); };
+  auto accempty_bar = [&](int b) { return bar0 + 8u * (3 * kGemmStages + 2 + b); };
 
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(bfull_bar(s), 8);
+      mbar_init(bfull_bar(s), kGemmDqWarps);
       mbar_init(empty_bar(s), 1);
     }
-    mbar_init(accfull_bar, 1);
-    mbar_init(accempty_bar, 8);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull_bar(b), 1);
+      mbar_init(accempty_bar(b), kGemmDqWarps);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     s_abort = 0;
   }
@@ -282,7 +297,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++tcount) {
         const TileCoord tc = gemm_tile(p, t);
         const int nk = p.mat[tc.mi].K / kGemmBK;
-        if (!mbar_wait(accempty_bar, (tcount & 1) ^ 1, p.status, abort)) break;
+        const int ab = tcount & 1;  // accumulator set of this tile
+        if (!mbar_wait(accempty_bar(ab), ((tcount >> 1) & 1) ^ 1, p.status, abort)) break;
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -302,79 +318,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint64_t da = umma_desc_sw128(a0 + h * (kGemmATile / 2) + 32 * k16);
-              umma_f16(tmem + h * kGemmBN, da, db, idesc, (kb | k16) != 0);
+              umma_f16(tmem + (uint32_t)(ab * 2 * kGemmBN + h * kGemmBN), da, db, idesc, (kb | k16) != 0);
             }
           }
           umma_commit(empty_bar(s));
         }
         if (!ok) break;
-        umma_commit(accfull_bar);
+        umma_commit(accfull_bar(ab));
+      }
+      // the last commits land before the CTA may exit
+      if (tcount > 0 && !*abort) {
+        int dummy = 0;
+        volatile int no_abort = 0;
+        const uint32_t last = tcount - 1;
+        mbar_wait(accfull_bar(last & 1), (last >> 1) & 1, &dummy, &no_abort);
       }
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ dequant + epilogue
-    const int d = tid - 128;  // weight row within the tile, 0..255
-    const int q = warp & 3;   // TMEM lane quadrant of this warp
-    const int ch = (warp - 4) >> 2;  // column half handled in the epilogue
-    const bool dq = p.dq != 0;
-    uint32_t it = 0, tcount = 0;
-    for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++tcount) {
-      const TileCoord tc = gemm_tile(p, t);
+    const int dt = tid - 64;        // 0..511
+    const int d = dt >> 2;          // weight row within the tile, 0..127
+    const int qk = dt & 3;          // k quarter of the 64-k block: codes 16 qk .. 16 qk + 15
+    const int q = warp & 3;         // TMEM lane quadrant of this warp
+    const int cc = (warp - 2) >> 2; // 32-column chunk handled in the epilogue
+    const uint32_t lvb = smem_u32(s_lv) + 4u * lane;
+    // epilogue of a finished tile: its accumulator set -> Y
+    // (the MMAs of the next tile go to the other accumulator set meanwhile)
+    auto epilogue = [&](const TileCoord &tc, uint32_t tcount) -> bool {
       const GemmMat &m = p.mat[tc.mi];
-      const int nk = m.K / kGemmBK;
-      const int row = tc.tn * kGemmBN + d;
-      const bool row_ok = row < m.N;
-      const float mu = (dq && row_ok) ? __ldg(m.absmax_mean) : 0.0f;
-      const int64_t bi0 = (int64_t)row * nk;
-      auto scale_of = [&](int kb) -> float {
-        if (!row_ok || kb >= nk) return 0.0f;
-        const int64_t bi = bi0 + kb;
-        if (dq) return __fadd_rn(__fmul_rn((float)__ldg(m.absmax_q + bi), __ldg(m.absmax_scale + (bi >> 8))), mu);
-        return __ldg(m.absmax + bi);
-      };
-      float sc_next = scale_of(0);
-      bool ok = true;
-      for (int kb = 0; kb < nk; ++kb, ++it) {
-        const int s = it % kGemmStages;
-        const uint32_t use = it / kGemmStages;
-        const float sc = sc_next;
-        sc_next = scale_of(kb + 1);
-        if (!mbar_wait_warp(full_bar(s), use & 1, p.status, abort)) {
-          ok = false;
-          break;
-        }
-        const uint4 *raw = reinterpret_cast<const uint4 *>(sR + s * kGemmRawTile + d * 32);
-        const uint4 r0 = raw[0], r1 = raw[1];
-        const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-        uint8_t *brow = sB + s * kGemmBTile + (d >> 3) * 1024 + (d & 7) * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = k 8c..8c+7 = packed word c
-          const uint32_t w = words[c];
-          uint32_t o[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float l0 = s_lv[((w >> (8 * j)) & 15) * 32 + lane];
-            const float l1 = s_lv[((w >> (8 * j + 4)) & 15) * 32 + lane];
-            o[j] = Dt<DA>::pack2(__fmul_rn(sc, l0), __fmul_rn(sc, l1));
-          }
-          *reinterpret_cast<uint4 *>(brow + ((c ^ (d & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bfull_bar(s));
-      }
-      if (!ok) break;
-      // ---- epilogue
-      if (!mbar_wait_warp(accfull_bar, tcount & 1, p.status, abort)) break;
-      tc_fence_after();
+        const int ab = tcount & 1;
+        if (!mbar_wait_warp(accfull_bar(ab), (tcount >> 1) & 1, p.status, abort)) return false;
+        tc_fence_after();
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int mrow = tc.tm * kGemmBM + h * 128 + q * 32 + lane;
-#pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-          const int col0 = ch * 128 + j * 32;
+        for (int h = 0; h < 2; ++h) {
+          const int mrow = tc.tm * kGemmBM + h * 128 + q * 32 + lane;
+          const int col0 = cc * 32;
           uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * kGemmBN + col0), r);
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * 2 * kGemmBN + h * kGemmBN + col0), r);
           const int n0 = tc.tn * kGemmBN + col0;
           if (mrow < m.M && n0 < m.N) {
             if (p.y_dtype == Q4_F32) {
@@ -400,11 +380,143 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(accempty_bar(ab));
+      return true;
+    };
+    bool have_prev = false;
+    TileCoord prev_tc{0, 0, 0};
+    uint32_t prev_count = 0;
+    uint32_t it = 0, tcount = 0;
+    for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++tcount) {
+      const TileCoord tc = gemm_tile(p, t);
+      const GemmMat &m = p.mat[tc.mi];
+      const int nk = m.K / kGemmBK;
+      const int row = tc.tn * kGemmBN + d;
+      const bool row_ok = row < m.N;
+      const float mu = (DQ && row_ok) ? __ldg(m.absmax_mean) : 0.0f;
+      const int64_t bi0 = (int64_t)min(row, m.N - 1) * nk;
+      // block scales: the c~ of 16 blocks of the row at a time, computed by
+      // the row's four threads (four blocks each) from inputs requested 16
+      // blocks ahead, kept in shared memory for the row
+      struct In4 {
+        uint32_t cw;     // int8 codes of four blocks (double quant)
+        float s2a, s2b;  // second-level scales of their (at most two) 256-groups
+        int bsplit;
+        float f[4];      // fp32 absmax (no double quant)
+      };
+      auto load4 = [&](int kb0, In4 &o) {  // blocks kb0 + 4 qk .. + 3
+        const int b0 = kb0 + 4 * qk;
+        const int nv = max(0, min(4, nk - b0));
+        const int64_t bi = bi0 + b0;
+        if (nv == 0) {
+          o.cw = 0;
+          o.s2a = o.s2b = 0.0f;
+          o.bsplit = 4;
+          o.f[0] = o.f[1] = o.f[2] = o.f[3] = 0.0f;
+          return;
+        }
+        if constexpr (DQ) {
+          o.s2a = __ldg(m.absmax_scale + (bi >> 8));
+          o.s2b = __ldg(m.absmax_scale + ((bi + nv - 1) >> 8));
+          o.bsplit = (int)min((int64_t)4, (((bi >> 8) + 1) << 8) - bi);
+          if (nv == 4 && (bi & 3) == 0) {
+            o.cw = __ldg(reinterpret_cast<const unsigned *>(m.absmax_q + bi));
+          } else {
+            uint32_t w = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (e < nv) w |= (uint32_t)(uint8_t)__ldg(m.absmax_q + bi + e) << (8 * e);
+            o.cw = w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o.f[e] = e < nv ? __ldg(m.absmax + bi + e) : 0.0f;
+        }
+      };
+      float *scrow = sSc + d * 16;
+      auto store4 = [&](const In4 &o) {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (DQ) {
+            const int code = (int)(int8_t)((o.cw >> (8 * e)) & 0xFFu);
+            v[e] = __fadd_rn(__fmul_rn((float)code, e < o.bsplit ? o.s2a : o.s2b), mu);
+          } else {
+            v[e] = o.f[e];
+          }
+          if (!row_ok) v[e] = 0.0f;
+        }
+        *reinterpret_cast<float4 *>(scrow + 4 * qk) = make_float4(v[0], v[1], v[2], v[3]);
+      };
+      In4 nin;
+      {
+        In4 cin;
+        load4(0, cin);
+        if (nk > 16) load4(16, nin);
+        __syncwarp();  // the row's previous c~ have been read
+        store4(cin);
+        __syncwarp();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(accempty_bar);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % kGemmStages;
+        const uint32_t use = it / kGemmStages;
+        if ((kb & 15) == 0 && kb > 0) {
+          __syncwarp();  // the row's c~ of the previous 16 blocks have been read
+          store4(nin);
+          __syncwarp();
+          if (kb + 16 < nk) load4(kb + 16, nin);
+        }
+        const float sc = scrow[kb & 15];
+        // lane 0 waits for the copy (acquire); the shuffle keeps the other
+        // lanes' reads of the stage after it
+        {
+          bool ready = true;
+          if (lane == 0) ready = mbar_wait(full_bar(s), use & 1, p.status, abort);
+          if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) {
+            ok = false;
+            break;
+          }
+        }
+        // 8 packed bytes = codes 16 qk .. 16 qk + 15 of row d
+        const uint2 raw = *reinterpret_cast<const uint2 *>(sR + s * kGemmRawTile + d * 32 + qk * 8);
+        uint8_t *brow = sB + s * kGemmBTile + (d >> 3) * 1024 + (d & 7) * 128;
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {  // 16-byte chunk 2 qk + c2 = k 8 (2 qk + c2) .. + 7
+          const uint32_t w = c2 ? raw.y : raw.x;
+          const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;  // codes 2j, 2j+1
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // level table: entry e of this lane at lvb + e * 128
+            const float l0 = lds_f32((__byte_perm(lo, 0u, 0x4440u | j) << 7) + lvb);
+            const float l1 = lds_f32((__byte_perm(hi, 0u, 0x4440u | j) << 7) + lvb);
+            o[j] = Dt<DA>::pack2(__fmul_rn(sc, l0), __fmul_rn(sc, l1));
+          }
+          const int c = 2 * qk + c2;
+          *reinterpret_cast<uint4 *>(brow + ((c ^ (d & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bfull_bar(s));
+        // the previous tile's epilogue once this tile's first stages are
+        // queued: its stores overlap the MMAs of those stages
+        if (have_prev && kb == min(kGemmStages, nk) - 1) {
+          if (!epilogue(prev_tc, prev_count)) {
+            ok = false;
+            break;
+          }
+          have_prev = false;
+        }
+      }
+      if (!ok) break;
+      have_prev = true;
+      prev_tc = tc;
+      prev_count = tcount;
     }
+    if (have_prev && !*abort) epilogue(prev_tc, prev_count);
   }
 
   tc_fence_before();

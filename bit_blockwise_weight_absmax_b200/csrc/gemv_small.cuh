@@ -688,19 +688,34 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int j = 0; j < 4; ++j) sum[nt][j] = 0.0f;
-      for (int c = c0; c <= c1; ++c) {
-        const int role = (gs_range_begin(c, T, G) >= x0) ? 0 : 1;  // c starts inside the tile
-        float *slot = p.slots + ((int64_t)(c * 2 + role) * kGsRows + warp * 16 * R + rt * 16 + g) * MW + 2 * tig;
+      for (int cb = c0; cb <= c1; cb += 4) {
+        // up to four contributors' rows in flight at once, added in CTA order
+        float2 v[4][NT][2];
+        float *slot[4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int k = 0; k < 4; ++k) {
+          const int c = min(cb + k, c1);
+          const int role = (gs_range_begin(c, T, G) >= x0) ? 0 : 1;  // c starts inside the tile
+          slot[k] = p.slots + ((int64_t)(c * 2 + role) * kGsRows + warp * 16 * R + rt * 16 + g) * MW + 2 * tig;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            float2 *sp = reinterpret_cast<float2 *>(slot + (h * 8) * MW + nt * 8);
-            const float2 v = __ldcg(sp);
-            __stcg(sp, make_float2(0.0f, 0.0f));  // the workspace is left zeroed
-            sum[nt][2 * h] += v.x;
-            sum[nt][2 * h + 1] += v.y;
-          }
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              v[k][nt][h] = __ldcg(reinterpret_cast<const float2 *>(slot[k] + (h * 8) * MW + nt * 8));
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (cb + k > c1) break;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // the workspace is left zeroed
+              __stcg(reinterpret_cast<float2 *>(slot[k] + (h * 8) * MW + nt * 8), make_float2(0.0f, 0.0f));
+              sum[nt][2 * h] += v[k][nt][h].x;
+              sum[nt][2 * h + 1] += v[k][nt][h].y;
+            }
+        }
       }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)

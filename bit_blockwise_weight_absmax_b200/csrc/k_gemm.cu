@@ -5,22 +5,26 @@
 
 namespace q4 {
 namespace {
-template <int DA>
+template <int DA, bool DQ>
 int go(const GemmParams &p, int sms, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(gemm_kernel<DA>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
+    if (cudaFuncSetAttribute(gemm_kernel<DA, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
         cudaSuccess)
       return Q4_ERR_CUDA;
     attr = true;
   }
   const int grid = (int)std::min<int64_t>(p.total_tiles, (int64_t)sms);
-  gemm_kernel<DA><<<grid, kGemmThreads, kGemmSmem, st>>>(p);
+  gemm_kernel<DA, DQ><<<grid, kGemmThreads, kGemmSmem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+template <int DA>
+int by_dq(const GemmParams &p, int sms, cudaStream_t st) {
+  return p.dq ? go<DA, true>(p, sms, st) : go<DA, false>(p, sms, st);
 }
 }  // namespace
 
 int run_gemm(int da, const GemmParams &p, int sms, cudaStream_t st) {
-  return da == Q4_F16 ? go<Q4_F16>(p, sms, st) : go<Q4_BF16>(p, sms, st);
+  return da == Q4_F16 ? by_dq<Q4_F16>(p, sms, st) : by_dq<Q4_BF16>(p, sms, st);
 }
 }  // namespace q4
