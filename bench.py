@@ -40,6 +40,27 @@ PREFILL_M = 512
 N_COPIES = 4
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture of the kernel on one layer of this workload, keyed by the
+# SHA-256 of the kernel source it was taken on: a changed source reports null.
+# Outputs still dirty in L2 when the kernel ends are not counted as writes.
+NCU_TRAFFIC = {
+    "gemm": ("bit_blockwise_weight_absmax_b200/csrc/gemm.cuh",
+             "3c9e1c4a4ba87d63886d89ff07fdc24835c8cc5de88d312b0a592409a68e7373", 166_386_176),
+    "gemv": ("bit_blockwise_weight_absmax_b200/csrc/gemv_small.cuh",
+             "bcae850413da9eae58c41c43eac60c129af67aed0a6fd1f820223f44f6b854ed", 114_144_768),
+}
+
+
+def _ncu_traffic(kernel):
+    import hashlib
+    if kernel not in NCU_TRAFFIC:
+        return None
+    path, digest, nbytes = NCU_TRAFFIC[kernel]
+    with open(os.path.join(ROOT, path), "rb") as f:
+        return nbytes if hashlib.sha256(f.read()).hexdigest() == digest else None
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -117,12 +138,16 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- CPU oracle ---
-def oracle_sample(rows_per_matrix=16, seed=0):
-    """Time the oracle on a bounded sample of the same workload: NF4 + DQ
-    quantize of one 4096x4096 bf16 matrix, and the GEMV reference (dequantize
-    + binary64 matmul) of the first `rows_per_matrix` rows of every matrix of
-    the layer at M = 1, 4, 16.  Returns (TB/s of GEMV algorithmic bytes,
-    quantize GB/s, threads, description, seconds)."""
+def oracle_sample(rows_per_matrix=16, quantize_layer=True, seed=0):
+    """Time the oracle on a bounded sample of the same workload and scale it
+    to one whole layer.  Quantize: NF4 + DQ of the full layer (all seven
+    matrices) when `quantize_layer`, else of the 4096x4096 q matrix.  GEMV:
+    the reference (dequantize + binary64 matmul) of the first
+    `rows_per_matrix` output rows of every matrix at M = 1, 4, 16; each
+    matrix's time is scaled by N / rows to the full matrix, and the value is
+    the layer's algorithmic GEMV bytes over the scaled time, summed over M
+    like the GPU arm.  Returns (TB/s, quantize GB/s, threads, description,
+    seconds spent, scaled ms of the whole layer's GEMVs at the three M)."""
     import numpy as np
     import torch
 
@@ -130,46 +155,53 @@ def oracle_sample(rows_per_matrix=16, seed=0):
     from bit_blockwise_weight_absmax_b200 import workloads as wl
     threads = oracle.set_threads(os.cpu_count() or 1)
     t0 = time.perf_counter()
-    W = wl.gaussian((4096, 4096), 0.02, torch.bfloat16, seed)
-    wb = W.view(torch.int16).numpy().view(np.uint16).reshape(-1)
-    tq = time.perf_counter()
-    oracle.quantize(wb, True, 64, oracle.QT_NF4, True)
-    tq = time.perf_counter() - tq
-    q_gbs = wb.size * 2 / tq / 1e9
-    sub_bytes = 0
-    tg = 0.0
+    q_bytes, tq = 0, 0.0
+    for i, (_, N, K) in enumerate(wl.LAYER_7B if quantize_layer else wl.LAYER_7B[:1]):
+        W = wl.gaussian((N, K), 0.02, torch.bfloat16, seed + 100 + i)
+        wb = W.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+        del W
+        t = time.perf_counter()
+        oracle.quantize(wb, True, 64, oracle.QT_NF4, True)
+        tq += time.perf_counter() - t
+        q_bytes += wb.size * 2
+    q_gbs = q_bytes / tq / 1e9
+    t_full = {M: 0.0 for M in DECODE_M}
     for i, (_, N, K) in enumerate(wl.LAYER_7B):
-        Wr = wl.gaussian((rows_per_matrix, K), 0.02, torch.bfloat16, seed + 1 + i)
+        r = min(rows_per_matrix, N)
+        Wr = wl.gaussian((r, K), 0.02, torch.bfloat16, seed + 1 + i)
         st = oracle.quantize(Wr.view(torch.int16).numpy().view(np.uint16).reshape(-1), True, 64,
                              oracle.QT_NF4, True)
         for M in DECODE_M:
             A = wl.activation(M, K, torch.float16, seed + 50 + i)
             ab = A.view(torch.int16).numpy().view(np.uint16).reshape(-1)
             t = time.perf_counter()
-            oracle.gemv_reference(ab, False, st, rows_per_matrix, K)
-            tg += time.perf_counter() - t
-            sub_bytes += layer_state_bytes([("s", rows_per_matrix, K)]) + 2 * M * K + 2 * M * rows_per_matrix
-    desc = (f"oracle on host cores: NF4+DQ quantize of one 4096x4096 bf16 matrix, and the GEMV "
-            f"reference (dequantize + fp64 matmul) of the first {rows_per_matrix} rows of each "
-            f"of the 7 layer matrices at M=1,4,16; bytes scaled per row")
-    return sub_bytes / tg / 1e12, q_gbs, threads, desc, time.perf_counter() - t0
+            oracle.gemv_reference(ab, False, st, r, K)
+            t_full[M] += (time.perf_counter() - t) * N / r
+    tb = sum(gemv_bytes(wl.LAYER_7B, M) for M in DECODE_M) / sum(t_full.values()) / 1e12
+    desc = (f"oracle on {threads} host threads: NF4+DQ quantize of "
+            f"{'the whole 7B layer (7 matrices, 202M bf16 weights)' if quantize_layer else 'the 4096x4096 q matrix'}"
+            f"; GEMV reference (dequantize + fp64 matmul) of the first {rows_per_matrix} output rows "
+            f"of each of the 7 layer matrices at M=1,4,16, each matrix's time scaled by N/rows "
+            f"to the whole layer")
+    return tb, q_gbs, threads, desc, time.perf_counter() - t0, sum(t_full.values()) * 1e3
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
     steps, warm = args.steps, args.warmup
-    vals, qs = [], []
+    vals, qs, ms = [], [], []
     for i in range(warm + steps):
-        tb, qg, thr, desc, secs = oracle_sample(rows_per_matrix=8, seed=i)
+        tb, qg, thr, desc, secs, est_ms = oracle_sample(rows_per_matrix=256, quantize_layer=False, seed=i)
         if i >= warm:
             vals.append(tb)
             qs.append(qg)
+            ms.append(est_ms)
     v = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
-            "steps": steps, "warmup": warm, "ms_per_step": None, "higher_is_better": True,
+            "steps": steps, "warmup": warm, "ms_per_step": statistics.mean(ms), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "decode_M": list(DECODE_M), "sample": "8 rows per matrix"},
+            "config": {"workload": WORKLOAD, "decode_M": list(DECODE_M), "sample": "256 rows per matrix, scaled to the layer"},
             "quantize_gbs": statistics.mean(qs),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -328,7 +360,8 @@ def run_gpu(args, rank, world, local_rank):
     dom["kernel"] = dominant
     dom["launch_us"] = (gemv_ms if dominant == "gemv" else ph_ms[dominant]) * 1e3 / (
         args.steps * (L * len(DECODE_M) if dominant == "gemv" else launches[dominant]))
-    dom["traffic"] = None
+    dom["traffic"] = _ncu_traffic(dominant)
+    dom["traffic_unit"] = "bytes per launch (ncu, one layer)"
     dom["peak_source"] = f"{peaks['source']} ({'bf16_tflops_sustained' if dom['bound'] == 'tensor' else 'hbm_gbs'})"
 
     # ---- end to end through the public API: pinned host activations in,
@@ -371,7 +404,7 @@ def run_gpu(args, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
-        tb, qg, thr, desc, secs = oracle_sample(rows_per_matrix=16)
+        tb, qg, thr, desc, secs, _ = oracle_sample(rows_per_matrix=args.cpu_rows)
         cpu = {"value": tb, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc,
                "quantize_gbs": qg, "seconds": round(secs, 1)}
 
@@ -409,6 +442,8 @@ def main():
     ap.add_argument("--impl", default="q4", choices=["q4", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=2048,
+                    help="output rows per matrix in the timed oracle sample (cpu_baseline)")
     ap.add_argument("--profile", default=None,
                     help="run one phase eagerly (quantize, gemv_m1, gemv_m4, gemv_m16, dequantize, "
                          "gemm) --steps+1 times for a profiler capture; prints no metric")
