@@ -1,11 +1,13 @@
 // k_dequantize.cu -- launchers of the dequantize kernel.
+#include <algorithm>
+
 #include "q4_internal.h"
 
 namespace q4 {
 namespace {
 template <int QT, int DO, int B, bool DQ>
 void go(const DequantParams &p, int grid, cudaStream_t st) {
-  dequantize_kernel<QT, DO, B, DQ><<<grid, 256, 0, st>>>(p);
+  dequantize_kernel<QT, DO, B, DQ><<<grid, kDqThreads, 0, st>>>(p);
 }
 template <int QT, int DO, bool DQ>
 int by_bs(int bs, const DequantParams &p, int grid, cudaStream_t st) {
@@ -23,8 +25,12 @@ int by_do(int dout, int bs, const DequantParams &p, int grid, cudaStream_t st) {
 }
 }  // namespace
 
-int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int grid,
+int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int sms,
                    cudaStream_t st) {
+  // one warp per span, 8 resident blocks of 8 warps per SM at most
+  const int64_t spans = (p.n + kDqSpan - 1) / kDqSpan;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((spans + kDqThreads / 32 - 1) / (kDqThreads / 32),
+                                                                 (int64_t)sms * 8));
   int rc;
   if (qt == Q4_NF4) rc = dq ? by_do<Q4_NF4, true>(dout, bs, p, grid, st) : by_do<Q4_NF4, false>(dout, bs, p, grid, st);
   else if (qt == Q4_INT4_SYM) rc = by_do<Q4_INT4_SYM, false>(dout, bs, p, grid, st);

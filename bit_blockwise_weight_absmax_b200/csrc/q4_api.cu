@@ -401,9 +401,7 @@ int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream
   p.n = Wq->n;
   p.out = out;
   memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
-  const int64_t groups = ceil_div(Wq->n, 16);
-  const int grid = (int)std::min<int64_t>(ceil_div(groups, 256), (int64_t)di.sms * 8);
-  return run_dequantize(Wq->qtype, out_dtype, Wq->blocksize, Wq->double_quant != 0, p, grid,
+  return run_dequantize(Wq->qtype, out_dtype, Wq->blocksize, Wq->double_quant != 0, p, di.sms,
                         (cudaStream_t)stream);
 }
 

@@ -15,7 +15,7 @@ namespace q4 {
 int run_quantize(int dt, int qt, int bs, bool dq, const QuantParams &p, int grid, cudaStream_t st);
 int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t *absmax_q,
                      float *absmax_scale, cudaStream_t st);
-int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int grid,
+int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int sms,
                    cudaStream_t st);
 int run_gemv(int da, int bs, int mp, const GvParams &p, int sms, cudaStream_t st);
 int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st);
