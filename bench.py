@@ -46,7 +46,7 @@ N_COPIES = 4
 # Outputs still dirty in L2 when the kernel ends are not counted as writes.
 NCU_TRAFFIC = {
     "gemm": ("bit_blockwise_weight_absmax_b200/csrc/gemm.cuh",
-             "3c9e1c4a4ba87d63886d89ff07fdc24835c8cc5de88d312b0a592409a68e7373", 166_386_176),
+             "337fd611724776050739860fe577d68ae6e5124bb3f982c7fada606f081f7263", 166_386_176),
     "gemv": ("bit_blockwise_weight_absmax_b200/csrc/gemv_small.cuh",
              "bcae850413da9eae58c41c43eac60c129af67aed0a6fd1f820223f44f6b854ed", 114_144_768),
 }
@@ -85,6 +85,24 @@ def layer_state_bytes(shapes, blocksize=64):
 
 def gemv_bytes(shapes, M):
     return layer_state_bytes(shapes) + sum(2 * M * K + 2 * M * N for _, N, K in shapes)
+
+
+# ------------------------------------------------------------- replicas --
+def max_over_ranks(values, world, device=None):
+    """Element-wise max over all ranks of per-rank device times (ms): the
+    slowest replica sets the whole job's time.  Identity at world size 1."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank, world, max_ms):
+    """Units per second of the whole job: every rank's units over the
+    slowest rank's time (weak scaling: each replica does the same work)."""
+    return world * units_per_rank / (max_ms / 1e3)
 
 
 # ------------------------------------------------------------------ clocks --
@@ -329,14 +347,11 @@ def run_gpu(args, rank, world, local_rank):
     gemm_flops = 2 * PREFILL_M * n_params * L * args.steps
 
     # max over ranks of the device times; value = all ranks' bytes / that time
-    import torch as _t
-    vec = _t.tensor([total_ms, gemv_ms] + [ph_ms[p] for p in phases], dtype=_t.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vec, op=dist.ReduceOp.MAX)
-    total_ms, gemv_ms = vec[0].item(), vec[1].item()
-    ph_ms = {p: vec[2 + i].item() for i, p in enumerate(phases)}
+    vec = max_over_ranks([total_ms, gemv_ms] + [ph_ms[p] for p in phases], world, dev)
+    total_ms, gemv_ms = vec[0], vec[1]
+    ph_ms = {p: vec[2 + i] for i, p in enumerate(phases)}
 
-    value = world * sum(gemv_B.values()) / (gemv_ms / 1e3) / 1e12
+    value = whole_job_rate(sum(gemv_B.values()), world, gemv_ms) / 1e12
     per_m = {f"M={M}": {"tb_s": gemv_B[M] / (ph_ms[f"gemv_m{M}"] / 1e3) / 1e12,
                         "us_per_layer": ph_ms[f"gemv_m{M}"] * 1e3 / (L * args.steps),
                         "bytes_per_layer": gemv_bytes(shapes, M)} for M in DECODE_M}
@@ -392,12 +407,8 @@ def run_gpu(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        v = _t.tensor([e2e_ms], dtype=_t.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(v, op=dist.ReduceOp.MAX)
-        e2e_ms = v.item()
-        e2e = {"value": world * sum(gemv_B.values()) / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+        e2e = {"value": whole_job_rate(sum(gemv_B.values()), world, e2e_ms) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "what": "q4.gemv_grouped at M=1,4,16 over the resident layer copies, activations "
                        "copied from pinned host memory and outputs read back every call"}

@@ -49,7 +49,7 @@ constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmScBytes + 1024 /*
 
 struct alignas(64) GemmMat {
   CUtensorMap tmA;  // A [M, K] 16-bit, box {64, 256}, 128B swizzle
-  CUtensorMap tmW;  // packed [N, K/2] bytes, box {32, 256}
+  CUtensorMap tmW;  // packed [N, K/2] bytes, box {32, 128}
   const int8_t *absmax_q;
   const float *absmax_scale;
   const float *absmax_mean;

@@ -1,4 +1,4 @@
-// gemv_tc.cuh -- fused NF4 dequant-GEMV for decode on tcgen05 (sm_100a):
+// gemv.cuh -- fused NF4 dequant-GEMV for decode on tcgen05 (sm_100a):
 // Y[M,N] = A[M,K] . W^[N,K]^T, 1 <= M <= 32.
 //
 // What it computes: n4n.ai, "What is 4-bit quantization and why does it

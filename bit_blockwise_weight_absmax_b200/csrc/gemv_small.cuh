@@ -223,6 +223,35 @@ __device__ __forceinline__ GsUnit gs_describe(const GsInfo *info, int count, int
   return u;
 }
 
+// The unit after `c`, which ended at global stage g: the same tile's next
+// window, else the next tile of the matrix, else the next matrix (the same
+// sequence gs_describe gives, without its division).
+template <int B>
+__device__ __forceinline__ GsUnit gs_next(const GsInfo *info, int count, const GsUnit &c, uint32_t g, uint32_t g0,
+                                         uint32_t g1) {
+  constexpr int W = kGsWinBlocks * B / kGsStageK;
+  GsUnit u;
+  u.mi = c.mi;
+  u.tile = c.tile;
+  u.q0 = c.q1;
+  if (c.q1 == info[c.mi].n_stages) {
+    u.q0 = 0;
+    u.tile = c.tile + 1;
+#pragma unroll 1
+    while (u.mi + 1 < count && g >= info[u.mi + 1].stage_begin) {
+      ++u.mi;
+      u.tile = 0;
+    }
+  }
+  const int ns = info[u.mi].n_stages;
+  int q1 = min((u.q0 / W + 1) * W, ns);
+  q1 = min(q1, u.q0 + (int)(g1 - g));
+  u.q1 = q1;
+  u.first = (u.q0 == 0) || (g == g0);
+  u.last = (q1 == ns) || (g + (q1 - u.q0) == g1);
+  return u;
+}
+
 // Inputs of the c~ of 8 blocks of one row (lane: row r0 + (lane & 15),
 // blocks (lane >> 4) * 8 + j of the window), loaded one unit ahead.
 struct GsScaleIn {
@@ -398,8 +427,10 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
       int s = 0, mi = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
+      GsUnit u;
+      if (g0 < g1) u = gs_describe<B>(info, p.count, mi, g0, g0, g1);
       for (uint32_t gi = g0; gi < g1 && ok;) {
-        const GsUnit u = gs_describe<B>(info, p.count, mi, gi, g0, g1);
+        if (gi != g0) u = gs_next<B>(info, p.count, u, gi, g0, g1);
         const GsMat &mt = p.mat[u.mi];
         for (int q = u.q0; q < u.q1; ++q) {
           if (!mbar_wait(sempty(s), ph ^ 1u, p.status, abort)) { ok = false; break; }
@@ -470,29 +501,55 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   int s = 0;
   uint32_t ph = 0;
 
+  // c~ buffer addresses at parity 0 (parity 1 at + kSbStride): where this
+  // lane writes block (lane >> 4) * 8 of its row lane & 15 (block j further at
+  // + joff(j)), and where it reads the (row g, row g + 8) pair of block 0
+  constexpr uint32_t kSbStride = EXACT ? (uint32_t)kGsScaleBuf : 8u * 256u;
+  auto joff = [](int j) -> uint32_t {
+    return EXACT ? (uint32_t)j * 64u : (uint32_t)(j >> 1) * 256u + (uint32_t)(j & 1) * 64u;
+  };
+  uint32_t cst[R], srd0[R];
+#pragma unroll
+  for (int rt = 0; rt < R; ++rt) {
+    const int r = lane & 15, blk0 = (lane >> 4) * 8;
+    cst[rt] = scale_addr(warp * R + rt, 0u, (uint32_t)((blk0 * 8 + (r & 7)) * 2 + (r >> 3)) * 4u);
+    srd0[rt] = scale_addr(warp * R + rt, 0u, (uint32_t)g * 8u);
+  }
+
   bool ok = true;
 #pragma unroll 1
   for (uint32_t gi = g0; gi < g1;) {
     // c~ of this unit into the next buffers (rewritten a unit after their last read)
     {
-      const int r = lane & 15, blk0 = (lane >> 4) * 8;
+      bool plain = dq;  // full windows inside one 256-group: no selects
 #pragma unroll
-      for (int rt = 0; rt < R; ++rt)
+      for (int rt = 0; rt < R; ++rt) plain = plain && sin[rt].nvalid == 8 && sin[rt].bsplit == 8;
+      if (__all_sync(0xffffffffu, plain)) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t o = (uint32_t)(((blk0 + j) * 8 + (r & 7)) * 2 + (r >> 3)) * 4u;
-          sts32(scale_addr(warp * R + rt, sb, o), __float_as_uint(gs_scale_value(sin[rt], dq, j)));
-        }
+        for (int rt = 0; rt < R; ++rt)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t w = j < 4 ? sin[rt].c0 : sin[rt].c1;
+            const float code = (float)(int)(int8_t)(uint8_t)(w >> (8 * (j & 3)));
+            sts32(cst[rt] + sb * kSbStride + joff(j), __float_as_uint(__fadd_rn(__fmul_rn(code, sin[rt].s2a), sin[rt].mu)));
+          }
+      } else {
+#pragma unroll
+        for (int rt = 0; rt < R; ++rt)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            sts32(cst[rt] + sb * kSbStride + joff(j), __float_as_uint(gs_scale_value(sin[rt], dq, j)));
+      }
     }
     __syncwarp();
     uint32_t srd[R];  // this lane's (row g, row g+8) pair of block 0, per row group
 #pragma unroll
-    for (int rt = 0; rt < R; ++rt) srd[rt] = scale_addr(warp * R + rt, sb, (uint32_t)g * 8u);
+    for (int rt = 0; rt < R; ++rt) srd[rt] = srd0[rt] + sb * kSbStride;
     sb ^= 1u;
     const GsUnit cu = u;
     const uint32_t gn = gi + (uint32_t)(cu.q1 - cu.q0);
     if (gn < g1) {  // next unit: issue its c~ loads now, use them a unit later
-      u = gs_describe<B>(info, p.count, mi, gn, g0, g1);
+      u = gs_next<B>(info, p.count, cu, gn, g0, g1);
 #pragma unroll
       for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, u, (warp * R + rt) * 16, lane, sin[rt]);
     }

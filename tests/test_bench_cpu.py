@@ -1,0 +1,63 @@
+"""The replica path of bench.py on CPU: world size 2 over gloo.
+
+The hot path does not shard (one GPU holds a whole 70B stack), so with
+--gpus N every rank runs an independent replica and the only cross-rank
+step is the max of the device times.  These tests run that step, and the
+reference arm's rank gating, as two gloo processes on 127.0.0.1."""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        # rank r took (r + 1) ms for phase 0 and (10 - r) ms for phase 1
+        mx = bench.max_over_ranks([rank + 1.0, 10.0 - rank], world)
+        rate = bench.whole_job_rate(1e9, world, mx[0])
+        # the reference arm: rank 0 alone works; the others return at once
+        class A:
+            steps, warmup = 0, 0
+        skipped = bench.run_reference(A, rank, world) is None if rank else True
+        q.put((rank, mx, rate, skipped))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replicas_max_over_ranks_gloo_world2():
+    ctx = mp.get_context("spawn")
+    q = ctx.SimpleQueue()
+    port = _free_port()
+    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    for p in ps:
+        p.join(120)
+        assert p.exitcode == 0
+    got = sorted(q.get() for _ in range(2))
+    for rank, mx, rate, skipped in got:
+        assert mx == [2.0, 10.0]                 # the slowest rank per phase
+        assert rate == pytest.approx(2 * 1e9 / 2e-3)  # both ranks' units over the max time
+        assert skipped
+
+
+def test_single_rank_is_identity():
+    import bench
+    assert bench.max_over_ranks([3.5, 4.0], 1) == [3.5, 4.0]
+    assert bench.whole_job_rate(5e8, 1, 2.0) == pytest.approx(2.5e11)
