@@ -48,7 +48,7 @@ NCU_TRAFFIC = {
     "gemm": ("bit_blockwise_weight_absmax_b200/csrc/gemm.cuh",
              "337fd611724776050739860fe577d68ae6e5124bb3f982c7fada606f081f7263", 166_386_176),
     "gemv": ("bit_blockwise_weight_absmax_b200/csrc/gemv_small.cuh",
-             "bcae850413da9eae58c41c43eac60c129af67aed0a6fd1f820223f44f6b854ed", 114_144_768),
+             "6395969006e7298a1ade6edb5c3659c5c1f2fbc5bd9e4d9177b1a4600250879b", 117_004_032),
 }
 
 
@@ -196,11 +196,14 @@ def oracle_sample(rows_per_matrix=16, quantize_layer=True, seed=0):
             oracle.gemv_reference(ab, False, st, r, K)
             t_full[M] += (time.perf_counter() - t) * N / r
     tb = sum(gemv_bytes(wl.LAYER_7B, M) for M in DECODE_M) / sum(t_full.values()) / 1e12
+    whole = all(rows_per_matrix >= N for _, N, K in wl.LAYER_7B)
+    gemv_part = ("GEMV reference (dequantize + fp64 matmul) of the whole layer at M=1,4,16" if whole else
+                 f"GEMV reference (dequantize + fp64 matmul) of the first {rows_per_matrix} output rows "
+                 f"of each of the 7 layer matrices at M=1,4,16, each matrix's time scaled by N/rows "
+                 f"to the whole layer")
     desc = (f"oracle on {threads} host threads: NF4+DQ quantize of "
             f"{'the whole 7B layer (7 matrices, 202M bf16 weights)' if quantize_layer else 'the 4096x4096 q matrix'}"
-            f"; GEMV reference (dequantize + fp64 matmul) of the first {rows_per_matrix} output rows "
-            f"of each of the 7 layer matrices at M=1,4,16, each matrix's time scaled by N/rows "
-            f"to the whole layer")
+            f"; {gemv_part}")
     return tb, q_gbs, threads, desc, time.perf_counter() - t0, sum(t_full.values()) * 1e3
 
 
@@ -453,8 +456,9 @@ def main():
     ap.add_argument("--impl", default="q4", choices=["q4", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=2048,
-                    help="output rows per matrix in the timed oracle sample (cpu_baseline)")
+    ap.add_argument("--cpu-rows", type=int, default=11008,
+                    help="output rows per matrix in the timed oracle sample (cpu_baseline); "
+                         "the default covers every row of the layer")
     ap.add_argument("--profile", default=None,
                     help="run one phase eagerly (quantize, gemv_m1, gemv_m4, gemv_m16, dequantize, "
                          "gemm) --steps+1 times for a profiler capture; prints no metric")

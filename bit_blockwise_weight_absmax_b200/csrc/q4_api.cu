@@ -135,30 +135,23 @@ int check_state(const q4_state *s) {
 }
 
 // ---- GEMV planning ----------------------------------------------------------
-// M <= 16 (mma.sync kernel): 256-row tiles cut into 128-k stages, the stages
-// of all matrices split evenly over at most kGsMaxCtas CTAs; workspace: a
-// 256-byte head, the per-CTA partial-row slots, then per matrix one counter
-// per 16 rows.  M > 16 (tcgen05 kernel): units of 128 rows x 1024 k;
-// workspace: the head (work counters), then per split matrix fp32 [N][M]
-// partial sums and one counter per 128-row tile.
+// The decode kernel takes M <= 16 rows of activations; 16 < M <= 32 runs it
+// twice (rows 0..15, then the rest), reading the weights twice.  Tiles of
+// 256 rows cut into 128-k stages, the stages of all matrices split evenly
+// over at most kGsMaxCtas CTAs.  Workspace: a 256-byte head, the per-CTA
+// partial-row slots, then per matrix one counter per 16 rows; both passes
+// reuse it (each leaves it zeroed).
 constexpr size_t kGemvWsHead = 256;
-size_t gemv_ws_for(const q4_state *s, int64_t M, int64_t *n_tiles, int64_t *n_splits) {
-  const bool small = M <= 16;
-  *n_tiles = ceil_div(s->rows, small ? kGsRows : kGvRows);
-  *n_splits = ceil_div(s->cols, small ? kGsStageK : kGvUnitK);  // small: stages per tile
-  if (small) return align256((size_t)ceil_div(s->rows, 16) * 4);
-  if (*n_splits <= 1) return 0;
-  return align256((size_t)s->rows * (size_t)M * 4) + align256((size_t)*n_tiles * 4);
+constexpr int kGemvPassRows = 16;
+size_t gemv_ws_for(const q4_state *s, int64_t *n_tiles, int64_t *n_stages) {
+  *n_tiles = ceil_div(s->rows, kGsRows);
+  *n_stages = ceil_div(s->cols, kGsStageK);  // stages per tile
+  return align256((size_t)ceil_div(s->rows, 16) * 4);
 }
-// Slots of the mma.sync kernel: [grid][2][256 rows][8 or 16] fp32.
+// Slots of the decode kernel: [grid][2][256 rows][8 or 16] fp32.
 size_t gemv_small_slots(int64_t total_stages, int64_t M) {
   const int64_t grid = std::min<int64_t>(total_stages, kGsMaxCtas);
   return align256((size_t)grid * 2 * kGsRows * (M <= 8 ? 8 : 16) * 4);
-}
-int pow2_at_least(int64_t m) {
-  int p = 1;
-  while (p < m) p <<= 1;
-  return p;
 }
 
 // ---- TMA descriptors ----------------------------------------------------------------
@@ -209,7 +202,7 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
   int64_t total = 0;
   for (int i = 0; i < count; ++i) {
     int64_t t, q;
-    gemv_ws_for(Wq[i], M, &t, &q);
+    gemv_ws_for(Wq[i], &t, &q);
     total += t * q;
   }
   const size_t slot_bytes = gemv_small_slots(total, M);
@@ -227,7 +220,7 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
     if (!aligned16(A[i])) return Q4_ERR_ALIGN;
     if (di.ok != Q4_OK) return di.ok;
     int64_t n_tiles, n_stages;
-    const size_t need = gemv_ws_for(s, M, &n_tiles, &n_stages);
+    const size_t need = gemv_ws_for(s, &n_tiles, &n_stages);
     if (n_tiles * n_stages > INT32_MAX) return Q4_ERR_SHAPE;
     GsMat &m = p.mat[i];
     const CUtensorMapDataType adt =
@@ -406,7 +399,7 @@ int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream
 }
 
 int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {
-  if (!bytes || !Wq || count < 1 || count > kGvMaxGroup) return Q4_ERR_ARG;
+  if (!bytes || !Wq || count < 1 || count > kGsMaxGroup) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
   size_t total = kGemvWsHead;
   int64_t stages = 0;
@@ -414,10 +407,10 @@ int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
     if (!Wq[i]) return Q4_ERR_ARG;
     if (!valid_bs(Wq[i]->blocksize) || Wq[i]->cols % Wq[i]->blocksize) return Q4_ERR_SHAPE;
     int64_t t, s;
-    total += gemv_ws_for(Wq[i], M, &t, &s);
+    total += gemv_ws_for(Wq[i], &t, &s);
     stages += t * s;
   }
-  if (M <= 16) total += gemv_small_slots(stages, M);
+  total += gemv_small_slots(stages, std::min<int64_t>(M, kGemvPassRows));
   *bytes = total;
   return Q4_OK;
 }
@@ -425,65 +418,25 @@ int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
 int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace,
                     size_t workspace_bytes, void *stream) {
-  if (count < 1 || count > kGvMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (count < 1 || count > kGsMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
   if (!Wq[0]) return Q4_ERR_ARG;
-  if (M <= 16) return gemv_small_grouped(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
-  static thread_local GvParams p;  // host staging of the kernel parameters (~5 KB)
-  memset(&p, 0, sizeof(p));
-  p.count = count;
-  p.M = (int)M;
-  p.y_dtype = y_dtype;
-  const int bs = Wq[0]->blocksize;
-  const int dq = Wq[0]->double_quant;
-  const int mp = pow2_at_least(M);
-  const int nb = mp <= 16 ? 16 : 32;
-  const DeviceInfo di = device_info();
-  int64_t units = 0;
-  size_t ws_off = kGemvWsHead;
+  if (M <= kGemvPassRows)
+    return gemv_small_grouped(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
+  // two passes of the decode kernel: activation rows 0..15, then 16..M-1
+  int rc = gemv_small_grouped(count, A, Wq, Y, kGemvPassRows, a_dtype, y_dtype, workspace, workspace_bytes,
+                              stream);
+  if (rc != Q4_OK) return rc;
+  const void *A2[kGsMaxGroup];
+  void *Y2[kGsMaxGroup];
+  const size_t ysize = y_dtype == Q4_F32 ? 4 : 2;
   for (int i = 0; i < count; ++i) {
-    const q4_state *s = Wq[i];
-    int rc = check_state(s);
-    if (rc != Q4_OK) return rc;
-    if (s->qtype != Q4_NF4 || s->blocksize != bs || s->double_quant != dq) return Q4_ERR_ARG;
-    if (s->cols % bs || s->rows > INT32_MAX || s->cols > INT32_MAX) return Q4_ERR_SHAPE;
-    if (!A[i] || !Y[i]) return Q4_ERR_ARG;
-    if (!aligned16(A[i])) return Q4_ERR_ALIGN;
-    if (di.ok != Q4_OK) return di.ok;
-    int64_t n_tiles, n_splits;
-    const size_t need = gemv_ws_for(s, M, &n_tiles, &n_splits);
-    GvMat &m = p.mat[i];
-    const CUtensorMapDataType adt =
-        a_dtype == Q4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (!make_map(&m.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1,
-                  kGvStageK / 2, kGvRows, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !make_map(&m.tmA, adt, A[i], M, s->cols, 2, kGvStageK, nb, CU_TENSOR_MAP_SWIZZLE_128B))
-      return Q4_ERR_CUDA;
-    m.absmax = s->absmax;
-    m.absmax_q = s->absmax_q;
-    m.absmax_scale = s->absmax_scale;
-    m.absmax_mean = s->absmax_mean;
-    m.Y = Y[i];
-    m.N = (int32_t)s->rows;
-    m.K = (int32_t)s->cols;
-    m.n_tiles = (int32_t)n_tiles;
-    m.n_splits = (int32_t)n_splits;
-    m.unit_begin = units;
-    units += n_tiles * n_splits;
-    if (need) {
-      if (!workspace || ws_off + need > workspace_bytes) return Q4_ERR_WORKSPACE;
-      m.acc = reinterpret_cast<float *>((char *)workspace + ws_off);
-      m.cnt = reinterpret_cast<unsigned *>((char *)workspace + ws_off +
-                                           align256((size_t)s->rows * (size_t)M * 4));
-      ws_off += need;
-    }
+    A2[i] = static_cast<const char *>(A[i]) + (size_t)kGemvPassRows * (size_t)Wq[i]->cols * 2;
+    Y2[i] = static_cast<char *>(Y[i]) + (size_t)kGemvPassRows * (size_t)Wq[i]->rows * ysize;
   }
-  p.dq = dq;
-  p.total_units = units;
-  p.status = di.status;
-  memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
-  return run_gemv(a_dtype, bs, mp, p, di.sms, (cudaStream_t)stream);
+  return gemv_small_grouped(count, A2, Wq, Y2, M - kGemvPassRows, a_dtype, y_dtype, workspace, workspace_bytes,
+                            stream);
 }
 
 int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
@@ -496,7 +449,7 @@ int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void 
 
 int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream) {
-  if (count < 1 || count > kGvMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (count < 1 || count > kGsMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (y_dtype != Q4_F32 && y_dtype != a_dtype) return Q4_ERR_ARG;
   if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;

@@ -7,7 +7,6 @@
 #include "q4_common.cuh"
 #include "quantize.cuh"
 #include "dequantize.cuh"
-#include "gemv.cuh"
 #include "gemv_small.cuh"
 #include "gemm.cuh"
 
@@ -17,7 +16,6 @@ int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t 
                      float *absmax_scale, cudaStream_t st);
 int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int sms,
                    cudaStream_t st);
-int run_gemv(int da, int bs, int mp, const GvParams &p, int sms, cudaStream_t st);
 int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st);
 int run_gemm(int da, const GemmParams &p, int sms, cudaStream_t st);
 }  // namespace q4

@@ -206,7 +206,9 @@ Q4_API int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int6
  * q4_gemv -- Y[M, N] = A[M, K] . W^[N, K]^T for 1 <= M <= 32 ([NF4] "Why it
  * matters": memory-bound decode at small batch; [BWQ]/[BNB] dequantize to
  * the compute dtype then matmul), with the dequantization fused into the
- * streaming of the packed weights and fp32 accumulation.
+ * streaming of the packed weights and fp32 accumulation.  The kernel takes
+ * 16 activation rows at a time: 16 < M <= 32 runs it twice (rows 0..15, then
+ * the rest), so the weights stream twice.
  *   A      device, a_dtype (Q4_F16 / Q4_BF16), [M, K] row-major, 16-byte
  *          aligned, K = Wq->cols.
  *   Wq     NF4 state, K % blocksize == 0, blocksize in {32, 64, 128, 256}.
@@ -218,8 +220,8 @@ Q4_API int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int6
 Q4_API int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
             int32_t y_dtype, void *workspace, size_t workspace_bytes, void *stream);
 
-/* q4_gemv over `count` (1..16) independent matrices in ONE launch (e.g. the
- * seven projections of a decoder layer).  A[i], Wq[i], Y[i] are host arrays
+/* q4_gemv over `count` (1..16) independent matrices in ONE launch per 16
+ * activation rows (e.g. the seven projections of a decoder layer).  A[i], Wq[i], Y[i] are host arrays
  * of device pointers / host structs; M, dtypes and the rules of q4_gemv
  * apply to every entry. */
 Q4_API int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
