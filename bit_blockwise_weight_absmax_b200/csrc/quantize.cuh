@@ -81,17 +81,22 @@ __device__ __forceinline__ uint32_t nf4_code_fast(float x, uint32_t tb) {
   return (uint32_t)(base + (x >= thr ? 1 : 0));
 }
 
+// Four resident CTAs of 256 threads per SM (at most 64 registers): more
+// warps to hide the division and table latencies, with four 16-byte loads
+// in flight per thread.
 template <int DT, int QT, int B, bool DQ>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
+__global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
   constexpr int LPB = B / 8;                     // lanes per block
   constexpr int ELEMS_IT = kQThreads * 8;        // elements per CTA iteration
   constexpr int IT_PER_CHUNK = kChunkBlocks * B / ELEMS_IT;  // = B / 8
   constexpr int BLK_IT = ELEMS_IT / B;           // blocks per CTA iteration
-  constexpr int BATCH = IT_PER_CHUNK < 8 ? IT_PER_CHUNK : 8;
+  constexpr int BATCH = IT_PER_CHUNK < 4 ? IT_PER_CHUNK : 4;  // loads in flight per thread
   constexpr int64_t CHUNK_ELEMS = (int64_t)kChunkBlocks * B;
 
   __shared__ float2 s_tab[32 * 32];              // lane-private copies of the bin table
-  __shared__ double s_blk[kChunkBlocks];         // block absmax of the current chunk
+  // per chunk parity: the sums of each warp's blocks of each iteration
+  // (aligned subtrees of the chunk's pairwise tree), iteration-major
+  __shared__ double s_part[2][IT_PER_CHUNK * 8];
   __shared__ uint8_t s_zero[BLK_IT];             // INT4_ASYM zero-points of one iteration
   __shared__ double s_stack[24];                 // streaming pairwise stack (thread 0)
   __shared__ int s_last;
@@ -110,6 +115,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
 
   int nonfinite = 0;
   int depth = 0;  // stack depth (thread 0)
+  int cpar = 0;   // parity of s_part for the current chunk
   const int64_t c0 = (int64_t)blockIdx.x * p.run;
   const int64_t c1 = min(c0 + p.run, p.n_chunks);
 
@@ -258,10 +264,15 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
               }
             }
           }
-          if ((tid % LPB) == 0) {
-            const bool in = FULL || chunk_b0 + bl < p.nb;
-            if (in) p.absmax[chunk_b0 + bl] = scale;
-            if (DQ) s_blk[bl] = in ? (double)scale : 0.0;
+          const bool in = FULL || chunk_b0 + bl < p.nb;
+          if ((tid % LPB) == 0 && in) p.absmax[chunk_b0 + bl] = scale;
+          if (DQ) {
+            // the warp's 32 / LPB blocks: xor shuffles at distance LPB, 2 LPB,
+            // ... pair adjacent blocks, then adjacent pairs (tree order)
+            double v = in ? (double)scale : 0.0;
+#pragma unroll
+            for (int o = LPB; o < 32; o <<= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) s_part[cpar][it * 8 + (tid >> 5)] = v;
           }
           if (QT == Q4_INT4_ASYM) {
             __syncthreads();
@@ -277,13 +288,20 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
     if (chunk_e0 + CHUNK_ELEMS <= p.n) run_chunk(std::true_type{});
     else run_chunk(std::false_type{});
     if (DQ) {
-      // Pairwise fp64 sum of the chunk's 256 block values in tree order:
-      // lane l reduces blocks 8l..8l+7 as ((0+1)+(2+3))+((4+5)+(6+7)), then
-      // xor shuffles at distance 1, 2, 4, 8, 16 pair adjacent subtrees.
+      // Pairwise fp64 sum of the chunk's 256 block values in tree order,
+      // from the B warp partials (aligned subtrees of 256 / B blocks): lane l
+      // combines partials PL l .. PL l + PL - 1 pairwise, then xor shuffles at
+      // distance 1, 2, 4, 8, 16 pair adjacent subtrees.  One barrier: the
+      // next chunk writes the other parity.
       __syncthreads();
       if (tid < 32) {
-        const double *q = s_blk + 8 * tid;
-        double s = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
+        constexpr int PL = B / 32;  // partials per lane
+        const double *q = s_part[cpar] + PL * tid;
+        double s;
+        if constexpr (PL == 1) s = q[0];
+        else if constexpr (PL == 2) s = q[0] + q[1];
+        else if constexpr (PL == 4) s = (q[0] + q[1]) + (q[2] + q[3]);
+        else s = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) s = s + __shfl_xor_sync(0xffffffffu, s, o);
         if (tid == 0) {
@@ -296,7 +314,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(QuantParams p) {
           }
         }
       }
-      __syncthreads();
+      cpar ^= 1;
     }
   }
 
