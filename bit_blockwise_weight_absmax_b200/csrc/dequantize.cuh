@@ -115,6 +115,7 @@ __device__ __forceinline__ void dq_span(const DequantParams &p, int64_t base, in
 
 template <int QT, int DOUT, int B, bool DQ>
 __global__ void __launch_bounds__(kDqThreads, QT == Q4_INT4_ASYM ? 6 : 8) dequantize_kernel(const __grid_constant__ DequantParams p) {
+  pdl_launch_then_wait();
   static_assert(B % 8 == 0, "a chunk never straddles two blocks");
   __shared__ float s_lv[16 * 32];  // [level][lane]
   const int lane = threadIdx.x & 31;

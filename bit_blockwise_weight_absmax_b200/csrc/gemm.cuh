@@ -220,6 +220,7 @@ __device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t t) {
 // DA: activation dtype; DQ: double-quantized block scales.
 template <int DA, bool DQ>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  pdl_launch_then_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sA = smem;                                        // [stages][32 KB]

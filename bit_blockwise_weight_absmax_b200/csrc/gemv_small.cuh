@@ -329,6 +329,7 @@ template <int R> struct GsShape {
 // groups per compute warp.
 template <int DA, int NT, int B, int R>
 __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(const __grid_constant__ GsParams p) {
+  pdl_launch_then_wait();
   constexpr int WARPS = GsShape<R>::kWarps;
   constexpr int PRODUCER = WARPS;
   constexpr bool EXACT = (DA == Q4_BF16);

@@ -7,7 +7,7 @@ namespace q4 {
 namespace {
 template <int QT, int DO, int B, bool DQ>
 void go(const DequantParams &p, int grid, cudaStream_t st) {
-  dequantize_kernel<QT, DO, B, DQ><<<grid, kDqThreads, 0, st>>>(p);
+  launch_pdl(dequantize_kernel<QT, DO, B, DQ>, dim3(grid), dim3(kDqThreads), 0, st, p);
 }
 template <int QT, int DO, bool DQ>
 int by_bs(int bs, const DequantParams &p, int grid, cudaStream_t st) {

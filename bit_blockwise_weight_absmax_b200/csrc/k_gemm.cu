@@ -15,7 +15,7 @@ int go(const GemmParams &p, int sms, cudaStream_t st) {
     attr = true;
   }
   const int grid = (int)std::min<int64_t>(p.total_tiles, (int64_t)sms);
-  gemm_kernel<DA, DQ><<<grid, kGemmThreads, kGemmSmem, st>>>(p);
+  launch_pdl(gemm_kernel<DA, DQ>, dim3(grid), dim3(kGemmThreads), kGemmSmem, st, p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 template <int DA>

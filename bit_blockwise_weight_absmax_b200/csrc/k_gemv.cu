@@ -23,7 +23,7 @@ int go_small(const GsParams &p, int sms, cudaStream_t st) {
     attr = true;
   }
   const int grid = (int)std::min<int64_t>(p.total_stages, (int64_t)std::min(sms, kGsMaxCtas));
-  kern<<<grid, GsShape<R>::kThreads, kGsSmemBytes, st>>>(p);
+  launch_pdl(kern, dim3(grid), dim3(GsShape<R>::kThreads), kGsSmemBytes, st, p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 template <int DA, int NT>

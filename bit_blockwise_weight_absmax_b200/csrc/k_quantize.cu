@@ -5,7 +5,7 @@ namespace q4 {
 namespace {
 template <int DT, int QT, int B, bool DQ>
 void go(const QuantParams &p, int grid, cudaStream_t st) {
-  quantize_kernel<DT, QT, B, DQ><<<grid, kQThreads, 0, st>>>(p);
+  launch_pdl(quantize_kernel<DT, QT, B, DQ>, dim3(grid), dim3(kQThreads), 0, st, p);
 }
 template <int DT, int QT, bool DQ>
 int by_bs(int bs, const QuantParams &p, int grid, cudaStream_t st) {
@@ -35,7 +35,8 @@ int run_quantize(int dt, int qt, int bs, bool dq, const QuantParams &p, int grid
 int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t *absmax_q,
                      float *absmax_scale, cudaStream_t st) {
   const int64_t ng = (nb + Q4_DQ_GROUP - 1) / Q4_DQ_GROUP;
-  double_quant_kernel<<<(unsigned)((ng + 7) / 8), 256, 0, st>>>(absmax, nb, mean, absmax_q, absmax_scale);
+  launch_pdl(double_quant_kernel, dim3((unsigned)((ng + 7) / 8)), dim3(256), 0, st, absmax, nb, mean, absmax_q,
+             absmax_scale);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 }  // namespace q4

@@ -11,6 +11,16 @@
 namespace q4 {
 
 // Sticky status word (Q4_STATUS_* bits): kernels receive its device address.
+// Programmatic dependent launch: every kernel of this library is launched
+// with programmatic stream serialization, so it may become resident while
+// the previous kernel of the stream drains.  It first lets the next kernel
+// start launching, then waits until the previous one has completed and its
+// memory operations are visible, before touching global memory.
+__device__ __forceinline__ void pdl_launch_then_wait() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void raise_status(int *status, int bit) {
   if (status) atomicOr(status, bit);
 }

@@ -86,6 +86,7 @@ __device__ __forceinline__ uint32_t nf4_code_fast(float x, uint32_t tb) {
 // in flight per thread.
 template <int DT, int QT, int B, bool DQ>
 __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
+  pdl_launch_then_wait();
   constexpr int LPB = B / 8;                     // lanes per block
   constexpr int ELEMS_IT = kQThreads * 8;        // elements per CTA iteration
   constexpr int IT_PER_CHUNK = kChunkBlocks * B / ELEMS_IT;  // = B / 8
@@ -373,6 +374,7 @@ static __global__ void __launch_bounds__(256) double_quant_kernel(const float *_
                                                            const float *__restrict__ mean,
                                                            int8_t *__restrict__ absmax_q,
                                                            float *__restrict__ absmax_scale) {
+  pdl_launch_then_wait();
   const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int64_t ng = (nb + Q4_DQ_GROUP - 1) / Q4_DQ_GROUP;
