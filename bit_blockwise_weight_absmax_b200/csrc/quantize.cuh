@@ -87,17 +87,19 @@ __device__ __forceinline__ uint32_t nf4_code_fast(float x, uint32_t tb) {
 template <int DT, int QT, int B, bool DQ>
 __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
   pdl_launch_then_wait();
-  constexpr int LPB = B / 8;                     // lanes per block
-  constexpr int ELEMS_IT = kQThreads * 8;        // elements per CTA iteration
-  constexpr int IT_PER_CHUNK = kChunkBlocks * B / ELEMS_IT;  // = B / 8
+  constexpr int E = 16;                          // consecutive elements per thread (one block)
+  constexpr int V = E / 8;                       // 16-byte words per thread
+  constexpr int LPB = B / E;                     // lanes per block
+  constexpr int ELEMS_IT = kQThreads * E;        // elements per CTA iteration
+  constexpr int IT_PER_CHUNK = kChunkBlocks * B / ELEMS_IT;  // = B / 16
   constexpr int BLK_IT = ELEMS_IT / B;           // blocks per CTA iteration
-  constexpr int BATCH = IT_PER_CHUNK < 4 ? IT_PER_CHUNK : 4;  // loads in flight per thread
+  constexpr int BATCH = IT_PER_CHUNK < 2 ? IT_PER_CHUNK : 2;  // iterations of loads in flight
+  static_assert(B % E == 0, "a thread's elements lie in one block");
+  static_assert(V == 2, "the packed codes of a thread are one 8-byte store");
   constexpr int64_t CHUNK_ELEMS = (int64_t)kChunkBlocks * B;
 
   __shared__ float2 s_tab[32 * 32];              // lane-private copies of the bin table
-  // per chunk parity: the sums of each warp's blocks of each iteration
-  // (aligned subtrees of the chunk's pairwise tree), iteration-major
-  __shared__ double s_part[2][IT_PER_CHUNK * 8];
+  __shared__ double s_blk[2][kChunkBlocks];      // block absmax of a chunk, by chunk parity
   __shared__ uint8_t s_zero[BLK_IT];             // INT4_ASYM zero-points of one iteration
   __shared__ double s_stack[24];                 // streaming pairwise stack (thread 0)
   __shared__ int s_last;
@@ -116,23 +118,29 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
 
   int nonfinite = 0;
   int depth = 0;  // stack depth (thread 0)
-  int cpar = 0;   // parity of s_part for the current chunk
+  int cpar = 0;   // parity of s_blk for the current chunk
   const int64_t c0 = (int64_t)blockIdx.x * p.run;
   const int64_t c1 = min(c0 + p.run, p.n_chunks);
 
-  // Codes of the thread's eight elements (element j in bits 4j..4j+3) and
-  // the block's scale; lanes of one block agree on `scale` and `z`.
-  auto quant8 = [&](const uint4 &v, float &scale, int &z) -> uint32_t {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float f[8];
+  // Codes of the thread's E elements (element 8k + j in bits 4j..4j+3 of
+  // codes[k]) and the block's scale; lanes of one block agree on `scale`
+  // and `z`.
+  auto quantE = [&](const uint4 (&v)[V], float &scale, int &z, uint32_t (&codes)[V]) {
+    float f[E];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      f[2 * j] = lo16<DT>(w[j]);
-      f[2 * j + 1] = hi16<DT>(w[j]);
+    for (int k = 0; k < V; ++k) {
+      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f[8 * k + 2 * j] = lo16<DT>(w[j]);
+        f[8 * k + 2 * j + 1] = hi16<DT>(w[j]);
+      }
+      codes[k] = 0;
     }
-    uint32_t codes = 0;
     if (QT == Q4_NF4 || QT == Q4_INT4_SYM) {
-      uint32_t m = absmax_bits8(v);
+      uint32_t m = absmax_bits8(v[0]);
+#pragma unroll
+      for (int k = 1; k < V; ++k) m = max(m, absmax_bits8(v[k]));
 #pragma unroll
       for (int o = LPB / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
       const float c = Dt<DT>::to_f((uint16_t)m);
@@ -143,16 +151,19 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
           // every lane: finite weights with |w| <= c, so |x| <= 1
           const float y = __frcp_rn(c);
 #pragma unroll
-          for (int j = 7; j >= 0; --j) codes = (codes << 4) + nf4_code_fast(div_markstein(f[j], c, y), tb);
+          for (int k = 0; k < V; ++k)
+#pragma unroll
+            for (int j = 7; j >= 0; --j)
+              codes[k] = (codes[k] << 4) + nf4_code_fast(div_markstein(f[8 * k + j], c, y), tb);
         } else {
           const bool fast = markstein_ok(c);
           const float y = fast ? __frcp_rn(c) : 0.0f;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < E; ++j) {
             float x = fast ? div_markstein(f[j], c, y) : (c == 0.0f ? 0.0f : __fdiv_rn(f[j], c));
             const float2 e = s_tab[nf4_bin(x) * 32 + lane];
             const int code = __float_as_int(e.y) + (x >= e.x ? 1 : 0);
-            codes |= (uint32_t)code << (4 * j);
+            codes[j >> 3] |= (uint32_t)code << (4 * (j & 7));
           }
         }
       } else {
@@ -164,30 +175,35 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
           // its 4-bit two's complement in the low nibble
           const float y = __frcp_rn(s);
 #pragma unroll
-          for (int j = 7; j >= 0; --j)
-            codes = (codes << 4) | (__float_as_uint(__fadd_rn(div_markstein(f[j], s, y), 12582912.0f)) & 15u);
+          for (int k = 0; k < V; ++k)
+#pragma unroll
+            for (int j = 7; j >= 0; --j)
+              codes[k] = (codes[k] << 4) |
+                         (__float_as_uint(__fadd_rn(div_markstein(f[8 * k + j], s, y), 12582912.0f)) & 15u);
         } else {
           const bool fast = markstein_ok(s);
           const float y = fast ? __frcp_rn(s) : 0.0f;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < E; ++j) {
             int q = 0;
             if (s != 0.0f) {
               float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
               q = min(max(__float2int_rn(x), -8), 7);
             }
-            codes |= (uint32_t)(q & 15) << (4 * j);
+            codes[j >> 3] |= (uint32_t)(q & 15) << (4 * (j & 7));
           }
         }
       }
     } else {  // Q4_INT4_ASYM
       float mn = 0.0f, mx = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < E; ++j) {
         mn = fminf(mn, f[j]);
         mx = fmaxf(mx, f[j]);
       }
-      uint32_t m = absmax_bits8(v);
+      uint32_t m = absmax_bits8(v[0]);
+#pragma unroll
+      for (int k = 1; k < V; ++k) m = max(m, absmax_bits8(v[k]));
 #pragma unroll
       for (int o = LPB / 2; o >= 1; o >>= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -202,16 +218,15 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
       const bool fast = markstein_ok(s);
       const float y = fast ? __frcp_rn(s) : 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < E; ++j) {
         int q = 0;
         if (s != 0.0f) {
           float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
           q = min(max(__float2int_rn(x) + z, 0), 15);
         }
-        codes |= (uint32_t)q << (4 * j);
+        codes[j >> 3] |= (uint32_t)q << (4 * (j & 7));
       }
     }
-    return codes;
   };
 
   for (int64_t chunk = c0; chunk < c1; ++chunk) {
@@ -220,25 +235,28 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
     // FULL: the whole chunk lies inside the tensor (every chunk but the last)
     auto run_chunk = [&](auto full_tag) {
       constexpr bool FULL = decltype(full_tag)::value;
-      const uint16_t *wp = p.W + chunk_e0 + tid * 8;
-      uint8_t *pp = p.packed + chunk_e0 / 2 + tid * 4;
+      const uint16_t *wp = p.W + chunk_e0 + tid * E;
+      uint8_t *pp = p.packed + chunk_e0 / 2 + tid * (E / 2);
       for (int it0 = 0; it0 < IT_PER_CHUNK; it0 += BATCH) {
-        uint4 v[BATCH];
+        uint4 v[BATCH][V];
 #pragma unroll
         for (int b = 0; b < BATCH; ++b) {
           const int off = (it0 + b) * ELEMS_IT;
-          if (FULL) {
-            v[b] = ldg_stream_v4(wp + off);
-          } else {
-            const int64_t e0 = chunk_e0 + off + tid * 8;
-            if (e0 + 8 <= p.n) {
-              v[b] = ldg_stream_v4(wp + off);
-            } else {
-              uint16_t t[8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) t[j] = (e0 + j < p.n) ? p.W[e0 + j] : (uint16_t)0;
-              v[b] = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
-                                t[6] | (t[7] << 16));
+          for (int k = 0; k < V; ++k) {
+            if (FULL) {
+              v[b][k] = ldg_stream_v4(wp + off + 8 * k);
+            } else {
+              const int64_t e0 = chunk_e0 + off + tid * E + 8 * k;
+              if (e0 + 8 <= p.n) {
+                v[b][k] = ldg_stream_v4(wp + off + 8 * k);
+              } else {
+                uint16_t t[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) t[j] = (e0 + j < p.n) ? p.W[e0 + j] : (uint16_t)0;
+                v[b][k] = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
+                                     t[6] | (t[7] << 16));
+              }
             }
           }
         }
@@ -246,34 +264,31 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
         for (int b = 0; b < BATCH; ++b) {
           const int it = it0 + b;
           const int off = it * ELEMS_IT;
-          const int bl = it * BLK_IT + (tid * 8) / B;  // block within the chunk
+          const int bl = it * BLK_IT + (tid * E) / B;  // block within the chunk
           float scale = 0.0f;
           int z = 0;
-          const uint32_t codes = quant8(v[b], scale, z);
-          if (QT == Q4_INT4_ASYM && (tid % LPB) == 0) s_zero[(tid * 8) / B] = (uint8_t)z;
+          uint32_t codes[V];
+          quantE(v[b], scale, z, codes);
+          if (QT == Q4_INT4_ASYM && (tid % LPB) == 0) s_zero[(tid * E) / B] = (uint8_t)z;
           // ---- stores
-          const int64_t e0 = chunk_e0 + off + tid * 8;
-          if (FULL || e0 + 8 <= p.n) {
-            *reinterpret_cast<uint32_t *>(pp + off / 2) = codes;
+          const int64_t e0 = chunk_e0 + off + tid * E;
+          if (FULL || e0 + E <= p.n) {
+            *reinterpret_cast<uint2 *>(pp + off / 2) = make_uint2(codes[0], codes[1]);
           } else if (e0 < p.n) {
             const int valid = (int)(p.n - e0);
-            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+            for (int j = 0; j < E / 2; ++j) {
               if (2 * j < valid) {
-                uint32_t byte = (codes >> (8 * j)) & 0xFFu;
+                uint32_t byte = (codes[j >> 2] >> (8 * (j & 3))) & 0xFFu;
                 if (2 * j + 1 >= valid) byte &= 0x0Fu;  // odd n: high nibble is padding
                 pp[off / 2 + j] = (uint8_t)byte;
               }
             }
           }
-          const bool in = FULL || chunk_b0 + bl < p.nb;
-          if ((tid % LPB) == 0 && in) p.absmax[chunk_b0 + bl] = scale;
-          if (DQ) {
-            // the warp's 32 / LPB blocks: xor shuffles at distance LPB, 2 LPB,
-            // ... pair adjacent blocks, then adjacent pairs (tree order)
-            double v = in ? (double)scale : 0.0;
-#pragma unroll
-            for (int o = LPB; o < 32; o <<= 1) v = v + __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) s_part[cpar][it * 8 + (tid >> 5)] = v;
+          if ((tid % LPB) == 0) {
+            const bool in = FULL || chunk_b0 + bl < p.nb;
+            if (in) p.absmax[chunk_b0 + bl] = scale;
+            if (DQ) s_blk[cpar][bl] = in ? (double)scale : 0.0;
           }
           if (QT == Q4_INT4_ASYM) {
             __syncthreads();
@@ -289,20 +304,14 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
     if (chunk_e0 + CHUNK_ELEMS <= p.n) run_chunk(std::true_type{});
     else run_chunk(std::false_type{});
     if (DQ) {
-      // Pairwise fp64 sum of the chunk's 256 block values in tree order,
-      // from the B warp partials (aligned subtrees of 256 / B blocks): lane l
-      // combines partials PL l .. PL l + PL - 1 pairwise, then xor shuffles at
-      // distance 1, 2, 4, 8, 16 pair adjacent subtrees.  One barrier: the
-      // next chunk writes the other parity.
+      // Pairwise fp64 sum of the chunk's 256 block values in tree order:
+      // lane l reduces blocks 8l..8l+7 as ((0+1)+(2+3))+((4+5)+(6+7)), then
+      // xor shuffles at distance 1, 2, 4, 8, 16 pair adjacent subtrees.  One
+      // barrier: the next chunk writes the other parity.
       __syncthreads();
       if (tid < 32) {
-        constexpr int PL = B / 32;  // partials per lane
-        const double *q = s_part[cpar] + PL * tid;
-        double s;
-        if constexpr (PL == 1) s = q[0];
-        else if constexpr (PL == 2) s = q[0] + q[1];
-        else if constexpr (PL == 4) s = (q[0] + q[1]) + (q[2] + q[3]);
-        else s = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
+        const double *q = s_blk[cpar] + 8 * tid;
+        double s = ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) s = s + __shfl_xor_sync(0xffffffffu, s, o);
         if (tid == 0) {

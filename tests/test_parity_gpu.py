@@ -161,6 +161,27 @@ def test_gemv_blocksizes_dtypes(q4, oracle, bs, a_dtype):
         assert_matmul_close(y, ref)
 
 
+@pytest.mark.parametrize("M", [20, 32])
+@pytest.mark.parametrize("a_dtype,out_dtype", [(torch.bfloat16, None), (torch.float16, torch.float32),
+                                               (torch.bfloat16, torch.float32)])
+def test_gemv_two_pass_grouped_dtypes(q4, oracle, M, a_dtype, out_dtype):
+    """16 < M <= 32 runs the decode kernel twice (activation rows 0..15, then
+    the rest): a grouped call over two matrices of different shapes, with
+    16-bit and fp32 outputs, so the second pass's A and Y row offsets are
+    exercised for every element size."""
+    g = torch.Generator().manual_seed(M)
+    shapes = [(384, 1024), (272, 3072)]
+    Ws = [torch.randn(N, K, generator=g).mul(0.02).bfloat16() for N, K in shapes]
+    As = [torch.randn(M, K, generator=g).to(a_dtype) for N, K in shapes]
+    sts = [q4.quantize(dev(W), 64, "nf4", True) for W in Ws]
+    ys = q4.gemv_grouped([dev(A) for A in As], sts, out_dtype)
+    for (N, K), W, A, y in zip(shapes, Ws, As, ys):
+        assert y.shape == (M, N) and y.dtype == (out_dtype or a_dtype)
+        ost = oracle_state(oracle, W, 64, 0, True)
+        ref = oracle.gemv_reference(bits(A), a_dtype == torch.bfloat16, ost, N, K)
+        assert_matmul_close(y, ref)
+
+
 def test_gemv_fp32_output_tight(q4, oracle):
     """fp32 output against the unrounded reference: the fused path's own error
     (fp16 codebook values, fp32 accumulation) stays far below the tolerance."""
