@@ -416,6 +416,65 @@ def run_gpu(args, rank, world, local_rank):
                "what": "q4.gemv_grouped at M=1,4,16 over the resident layer copies, activations "
                        "copied from pinned host memory and outputs read back every call"}
 
+    # ---- the pages' own method, timed beside the fused path on the same
+    # resident states: dequantize every weight to a 16-bit buffer, then a
+    # library (cuBLAS) matmul.  Same algorithmic bytes / flops as the fused
+    # phases, so the ratio is the fusion's gain.
+    unfused = None
+    if not args.no_unfused:
+        w16 = {dt: [torch.empty(N, K, dtype=dt, device=dev) for _, N, K in shapes]
+               for dt in (torch.float16, torch.bfloat16)}
+
+        def un_gemv(M):
+            for l in range(L):
+                for st, w, a, y in zip(states[l], w16[torch.float16], A_dec[M], y_dec[M][l]):
+                    q4.dequantize(st, torch.float16, out=w)
+                    torch.matmul(a, w.t(), out=y)
+
+        def un_gemm():
+            for l in range(L):
+                for st, w, a, y in zip(states[l], w16[torch.bfloat16], A_pre, y_pre):
+                    q4.dequantize(st, torch.bfloat16, out=w)
+                    torch.matmul(a, w.t(), out=y)
+
+        ufns = {f"gemv_m{M}": (lambda M=M: un_gemv(M)) for M in DECODE_M}
+        ufns["gemm"] = un_gemm
+        for f in ufns.values():
+            f()
+        torch.cuda.synchronize()
+        ugraphs = {}
+        for name, f in ufns.items():
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                f()
+            ugraphs[name] = g
+        for g in ugraphs.values():
+            g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ums = {}
+        for name, g in ugraphs.items():
+            e0, e1 = ev(), ev()
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ums[name] = e0.elapsed_time(e1)
+        uv = max_over_ranks([ums[n] for n in ufns], world, dev)
+        ums = dict(zip(ufns, uv))
+        ugemv_ms = sum(ums[f"gemv_m{M}"] for M in DECODE_M)
+        unfused = {
+            "what": "q4.dequantize of every weight to a 16-bit buffer, then torch.matmul (cuBLAS), "
+                    "per matrix; same workload, bytes and flops as the fused phases",
+            "gemv_tb_s": whole_job_rate(sum(gemv_B.values()), world, ugemv_ms) / 1e12,
+            "gemv_us_per_layer": {f"M={M}": ums[f"gemv_m{M}"] * 1e3 / (L * args.steps) for M in DECODE_M},
+            "gemm_tflops": whole_job_rate(gemm_flops, world, ums["gemm"]) / 1e12,
+            "fused_speedup": {"gemv": ugemv_ms / gemv_ms, "gemm": ums["gemm"] / ph_ms["gemm"]},
+        }
+        del w16, ugraphs
+
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         tb, qg, thr, desc, secs, _ = oracle_sample(rows_per_matrix=args.cpu_rows)
@@ -442,6 +501,7 @@ def run_gpu(args, rank, world, local_rank):
             "launches_per_step": launches,
             "clocks": clk,
             "e2e": e2e,
+            "unfused_baseline": unfused,
             "cpu_baseline": cpu,
             "peaks": peaks,
         }
@@ -455,6 +515,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="q4", choices=["q4", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-unfused", action="store_true",
+                    help="skip timing the unfused dequantize-then-cuBLAS baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=11008,
                     help="output rows per matrix in the timed oracle sample (cpu_baseline); "

@@ -12,10 +12,10 @@
 // by HBM.  A warp owns spans of 256 * kDqChunks elements; within a span, lane
 // l expands the 8-element chunks l, l + 32, ... so that every 16-byte store
 // instruction of the warp covers 512 contiguous bytes, and every 4-byte load
-// of packed codes covers 128 contiguous bytes.  All loads of a span (codes and
-// block scales) are issued before the first multiply, to keep enough bytes in
-// flight per SM.  The 16 levels sit in shared memory, one copy per lane, so a
-// warp's 32 lookups hit 32 distinct banks.
+// of packed codes covers 128 contiguous bytes.  The raw inputs of a warp's
+// next span (codes, scale codes, group scales) are loaded while the current
+// one is expanded, so two spans' loads overlap.  The 16 levels sit in shared
+// memory, one copy per lane, so a warp's 32 lookups hit 32 distinct banks.
 #pragma once
 #include "q4_common.cuh"
 
@@ -46,46 +46,59 @@ __device__ __forceinline__ float dq_lds(uint32_t addr) {
 // One span of kDqSpan elements starting at `base` (chunks past the end of
 // the tensor are skipped).  lb: this lane's level table base (entry e of the
 // lane at lb + 128 e).
-template <int QT, int DOUT, int B, bool DQ>
-__device__ __forceinline__ void dq_span(const DequantParams &p, int64_t base, int lane, uint32_t lb, float mu,
-                                        uint16_t *out) {
+// The raw inputs of one span: loaded a span ahead, used a span later.
+struct DqRaw {
+  uint32_t pk[kDqChunks];  // 8 codes per chunk
+  int q[kDqChunks];        // int8 scale code (double quant) / zero-point byte (INT4 asym)
+  float s[kDqChunks];      // second-level scale (double quant) or the block scale
+};
+
+template <int QT, int B, bool DQ>
+__device__ __forceinline__ void dq_load(const DequantParams &p, int64_t base, int lane, DqRaw &r) {
   const int64_t n = p.n;
   const uint8_t *pk_base = p.packed + base / 2 + lane * 4;  // chunk u at + 128 u
   const int64_t b_base = base / B;
-  uint32_t pk[kDqChunks];
-  float sc[kDqChunks];
-  int z[kDqChunks];
 #pragma unroll
   for (int u = 0; u < kDqChunks; ++u) {
     const uint32_t off = (uint32_t)(u * 256 + lane * 8);  // element offset inside the span
-    pk[u] = 0u;
-    sc[u] = 0.0f;
-    z[u] = 0;
+    r.pk[u] = 0u;
+    r.q[u] = 0;
+    r.s[u] = 0.0f;
     if (base + off >= n) continue;
     if (base + off + 8 <= n) {
-      pk[u] = ldg_stream_u32(pk_base + u * 128);
+      r.pk[u] = ldg_stream_u32(pk_base + u * 128);
     } else {
 #pragma unroll
       for (int j = 0; j < 4; ++j)
-        if (base + off + 2 * j < n) pk[u] |= (uint32_t)pk_base[u * 128 + j] << (8 * j);
+        if (base + off + 2 * j < n) r.pk[u] |= (uint32_t)pk_base[u * 128 + j] << (8 * j);
     }
     const int64_t b = b_base + (int64_t)(off / B);
-    if (DQ) sc[u] = __fadd_rn(__fmul_rn((float)__ldg(p.absmax_q + b), __ldg(p.absmax_scale + b / Q4_DQ_GROUP)), mu);
-    else sc[u] = __ldg(p.absmax + b);
-    if (QT == Q4_INT4_ASYM) z[u] = (__ldg(p.zero + (b >> 1)) >> ((b & 1) * 4)) & 15;
+    if (DQ) {
+      r.q[u] = __ldg(p.absmax_q + b);
+      r.s[u] = __ldg(p.absmax_scale + b / Q4_DQ_GROUP);
+    } else {
+      r.s[u] = __ldg(p.absmax + b);
+      if (QT == Q4_INT4_ASYM) r.q[u] = __ldg(p.zero + (b >> 1)) >> ((b & 1) * 4);
+    }
   }
+}
+
+template <int QT, int DOUT, int B, bool DQ>
+__device__ __forceinline__ void dq_emit(const DequantParams &p, int64_t base, int lane, uint32_t lb, float mu,
+                                        uint16_t *out, const DqRaw &r) {
+  const int64_t n = p.n;
 #pragma unroll
   for (int u = 0; u < kDqChunks; ++u) {
     const uint32_t off = (uint32_t)(u * 256 + lane * 8);
     if (base + off >= n) break;  // chunks past the end are all later in the span
-    const uint32_t w = pk[u];
+    const float sc = DQ ? __fadd_rn(__fmul_rn((float)r.q[u], r.s[u]), mu) : r.s[u];
+    const int z = QT == Q4_INT4_ASYM ? (r.q[u] & 15) : 0;
+    const uint32_t w = r.pk[u];
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float l0, l1;
       if (QT == Q4_NF4) {
-        // code 2j at bits 8j..8j+3 and code 2j+1 at bits 8j+4..8j+7, moved
-        // to bits 7..10 (the entry stride of 128 bytes)
         const uint32_t a0 = (j == 0 ? (w << 7) : (w >> (8 * j - 7))) & 0x780u;
         const uint32_t a1 = (j == 0 ? (w << 3) : (w >> (8 * j - 3))) & 0x780u;
         l0 = dq_lds(lb + a0);
@@ -96,11 +109,11 @@ __device__ __forceinline__ void dq_span(const DequantParams &p, int64_t base, in
           l0 = (float)((c0 ^ 8) - 8);
           l1 = (float)((c1 ^ 8) - 8);
         } else {
-          l0 = (float)(c0 - z[u]);
-          l1 = (float)(c1 - z[u]);
+          l0 = (float)(c0 - z);
+          l1 = (float)(c1 - z);
         }
       }
-      o[j] = Dt<DOUT>::pack2(__fmul_rn(sc[u], l0), __fmul_rn(sc[u], l1));
+      o[j] = Dt<DOUT>::pack2(__fmul_rn(sc, l0), __fmul_rn(sc, l1));
     }
     const int64_t e = base + off;
     if (e + 8 <= n) {
@@ -113,8 +126,11 @@ __device__ __forceinline__ void dq_span(const DequantParams &p, int64_t base, in
   }
 }
 
+// Resident CTAs per SM: the registers of two spans' raw inputs.
+template <int QT> constexpr int dq_ctas_per_sm() { return QT == Q4_INT4_ASYM ? 4 : 5; }
+
 template <int QT, int DOUT, int B, bool DQ>
-__global__ void __launch_bounds__(kDqThreads, QT == Q4_INT4_ASYM ? 6 : 8) dequantize_kernel(const __grid_constant__ DequantParams p) {
+__global__ void __launch_bounds__(kDqThreads, dq_ctas_per_sm<QT>()) dequantize_kernel(const __grid_constant__ DequantParams p) {
   pdl_launch_then_wait();
   static_assert(B % 8 == 0, "a chunk never straddles two blocks");
   __shared__ float s_lv[16 * 32];  // [level][lane]
@@ -126,12 +142,19 @@ __global__ void __launch_bounds__(kDqThreads, QT == Q4_INT4_ASYM ? 6 : 8) dequan
   const uint32_t lb = (uint32_t)__cvta_generic_to_shared(s_lv) + 4u * (uint32_t)lane;
   const float mu = DQ ? __ldg(p.absmax_mean) : 0.0f;
   uint16_t *out = reinterpret_cast<uint16_t *>(p.out);
-  const int64_t n = p.n;
-  const int64_t nspan = (n + kDqSpan - 1) / kDqSpan;
+  const int64_t nspan = (p.n + kDqSpan - 1) / kDqSpan;
   const int wpb = blockDim.x >> 5;
-  for (int64_t sp = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5); sp < nspan; sp += (int64_t)gridDim.x * wpb) {
-    const int64_t base = sp * kDqSpan;
-    dq_span<QT, DOUT, B, DQ>(p, base, lane, lb, mu, out);
+  const int64_t stride = (int64_t)gridDim.x * wpb;
+  int64_t sp = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5);
+  if (sp >= nspan) return;
+  DqRaw cur;
+  dq_load<QT, B, DQ>(p, sp * kDqSpan, lane, cur);
+  for (; sp < nspan; sp += stride) {
+    // the next span's loads are in flight while this one is expanded
+    DqRaw nxt;
+    if (sp + stride < nspan) dq_load<QT, B, DQ>(p, (sp + stride) * kDqSpan, lane, nxt);
+    dq_emit<QT, DOUT, B, DQ>(p, sp * kDqSpan, lane, lb, mu, out, cur);
+    cur = nxt;
   }
 }
 

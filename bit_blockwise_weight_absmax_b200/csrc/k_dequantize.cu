@@ -27,10 +27,11 @@ int by_do(int dout, int bs, const DequantParams &p, int grid, cudaStream_t st) {
 
 int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int sms,
                    cudaStream_t st) {
-  // one warp per span, 8 resident blocks of 8 warps per SM at most
+  // one warp per span at a time, as many CTAs as are resident at once
   const int64_t spans = (p.n + kDqSpan - 1) / kDqSpan;
+  const int occ = qt == Q4_INT4_ASYM ? dq_ctas_per_sm<Q4_INT4_ASYM>() : dq_ctas_per_sm<Q4_NF4>();
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((spans + kDqThreads / 32 - 1) / (kDqThreads / 32),
-                                                                 (int64_t)sms * 8));
+                                                                 (int64_t)sms * occ));
   int rc;
   if (qt == Q4_NF4) rc = dq ? by_do<Q4_NF4, true>(dout, bs, p, grid, st) : by_do<Q4_NF4, false>(dout, bs, p, grid, st);
   else if (qt == Q4_INT4_SYM) rc = by_do<Q4_INT4_SYM, false>(dout, bs, p, grid, st);

@@ -197,6 +197,7 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
   p.y_dtype = y_dtype;
   const int bs = Wq[0]->blocksize;
   const int dq = Wq[0]->double_quant;
+  const int qt = Wq[0]->qtype;
   const DeviceInfo di = device_info();
   if (!workspace || workspace_bytes < kGemvWsHead) return Q4_ERR_WORKSPACE;
   int64_t total = 0;
@@ -214,7 +215,11 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
     const q4_state *s = Wq[i];
     int rc = check_state(s);
     if (rc != Q4_OK) return rc;
-    if (s->qtype != Q4_NF4 || s->blocksize != bs || s->double_quant != dq) return Q4_ERR_ARG;
+    // NF4, or INT4 symmetric (its codebook: the integers -8..7); one
+    // format per grouped call
+    if ((s->qtype != Q4_NF4 && s->qtype != Q4_INT4_SYM) || s->qtype != qt || s->blocksize != bs ||
+        s->double_quant != dq)
+      return Q4_ERR_ARG;
     if (s->cols % bs || s->rows > INT32_MAX || s->cols > INT32_MAX) return Q4_ERR_SHAPE;
     if (!A[i] || !Y[i]) return Q4_ERR_ARG;
     if (!aligned16(A[i])) return Q4_ERR_ALIGN;
@@ -248,7 +253,12 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
   p.dq = dq;
   p.total_stages = (uint32_t)stages;
   p.status = di.status;
-  memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+  if (qt == Q4_NF4) {
+    memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+  } else {
+    // INT4 symmetric: code j is the two's-complement nibble of q, w^ = q * s
+    for (int j = 0; j < 16; ++j) p.levels[j] = (float)((j ^ 8) - 8);
+  }
   return run_gemv_small(a_dtype, bs, (int)M, p, di.sms, (cudaStream_t)stream);
 }
 

@@ -211,7 +211,10 @@ Q4_API int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int6
  * the rest), so the weights stream twice.
  *   A      device, a_dtype (Q4_F16 / Q4_BF16), [M, K] row-major, 16-byte
  *          aligned, K = Wq->cols.
- *   Wq     NF4 state, K % blocksize == 0, blocksize in {32, 64, 128, 256}.
+ *   Wq     NF4 state (with or without double quantization) or INT4 symmetric
+ *          state (the codebook is then the integers -8..7 and the group scale
+ *          takes the place of c~), K % blocksize == 0, blocksize in
+ *          {32, 64, 128, 256}.  INT4 asymmetric states return Q4_ERR_ARG.
  *   Y      device, y_dtype (Q4_F16 / Q4_BF16 / Q4_F32), [M, N] row-major.
  *   workspace  device, q4_gemv_workspace_size() bytes, zero-filled.
  * Result: within relative Frobenius error 1e-3 of the binary64 product of A

@@ -1,0 +1,45 @@
+"""Host logic of the Linear4bit module: which layers replace_linear swaps,
+argument checks, and that a forward pass without a GPU fails loudly (there
+is no CPU path)."""
+import pytest
+import torch
+
+from bit_blockwise_weight_absmax_b200 import linear4bit, q4
+
+
+class _Toy(torch.nn.Module):
+    def __init__(self):
+        super().__init__()
+        self.embed = torch.nn.Embedding(10, 64)
+        self.layers = torch.nn.ModuleList([torch.nn.ModuleDict({
+            "q_proj": torch.nn.Linear(64, 64),
+            "mlp": torch.nn.Sequential(torch.nn.Linear(64, 128), torch.nn.GELU(), torch.nn.Linear(128, 64)),
+        }) for _ in range(2)])
+        self.norm = torch.nn.LayerNorm(64)
+        self.lm_head = torch.nn.Linear(64, 10)
+
+
+def test_linears_to_replace_keeps_head_embeddings_norms():
+    names = linear4bit.linears_to_replace(_Toy())
+    assert names == ["layers.0.q_proj", "layers.0.mlp.0", "layers.0.mlp.2",
+                     "layers.1.q_proj", "layers.1.mlp.0", "layers.1.mlp.2"]
+    assert "lm_head" in linear4bit.linears_to_replace(_Toy(), skip=())
+
+
+def _dummy_state():
+    z = torch.zeros(16, dtype=torch.uint8)
+    return q4.Q4State(q4.NF4, torch.float16, 4, 8, 64, False, z, torch.zeros(1))
+
+
+def test_rejects_fp32_compute_dtype():
+    with pytest.raises(q4.Q4Error):
+        linear4bit.Linear4bit(_dummy_state(), compute_dtype=torch.float32)
+
+
+def test_forward_without_gpu_fails_loudly():
+    m = linear4bit.Linear4bit(_dummy_state())
+    assert m.in_features == 8 and m.out_features == 4
+    with pytest.raises(q4.Q4Error):
+        m(torch.zeros(2, 8))
+    with pytest.raises(q4.Q4Error):
+        m(torch.zeros(2, 7))  # wrong width is caught before any kernel call

@@ -182,6 +182,32 @@ def test_gemv_two_pass_grouped_dtypes(q4, oracle, M, a_dtype, out_dtype):
         assert_matmul_close(y, ref)
 
 
+@pytest.mark.parametrize("M", [1, 16, 24])
+@pytest.mark.parametrize("a_dtype", [torch.float16, torch.bfloat16])
+def test_gemv_int4_sym(q4, oracle, a_dtype, M):
+    """INT4 symmetric, group 128 (the scheme-coverage format): the decode
+    kernel with the integer codebook -8..7 and the group scale in place of
+    c~, against the oracle's dequantize + binary64 matmul."""
+    g = torch.Generator().manual_seed(128 + M)
+    N, K = 400, 4096 + 128
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).to(a_dtype)
+    st = q4.quantize(dev(W), 128, "int4_sym", False)
+    ost = oracle_state(oracle, W, 128, 1, False)
+    assert_state_equal(st, ost)
+    y = q4.gemv(dev(A), st)
+    ref = oracle.gemv_reference(bits(A), a_dtype == torch.bfloat16, ost, N, K)
+    assert_matmul_close(y, ref)
+
+
+def test_gemv_rejects_int4_asym(q4):
+    """The asymmetric format's per-group zero-point has no place in the
+    decode kernel's codebook: the call fails instead of computing garbage."""
+    st = q4.quantize(dev(torch.randn(64, 128).half()), 128, "int4_asym", False)
+    with pytest.raises(q4.Q4Error):
+        q4.gemv(dev(torch.randn(1, 128).half()), st)
+
+
 def test_gemv_fp32_output_tight(q4, oracle):
     """fp32 output against the unrounded reference: the fused path's own error
     (fp16 codebook values, fp32 accumulation) stays far below the tolerance."""
