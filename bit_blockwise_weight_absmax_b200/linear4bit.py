@@ -55,17 +55,20 @@ class Linear4bit(torch.nn.Module):
         lead = x.shape[:-1]
         a = x.reshape(-1, self.in_features).to(self.compute_dtype).contiguous()
         T = a.shape[0]
+        # with a bias the product stays fp32 until the bias is added, so the
+        # output is rounded to the compute dtype once
+        acc = torch.float32 if self.bias is not None else self.compute_dtype
         if T == 0:
-            y = a.new_empty(0, self.out_features)
+            y = a.new_empty(0, self.out_features, dtype=acc)
         elif T <= GEMV_MAX_ROWS:
-            y = q4.gemv(a, self.state)
+            y = q4.gemv(a, self.state, acc)
         elif self._gemm_ok():
-            y = q4.gemm(a, self.state)
+            y = q4.gemm(a, self.state, acc)
         else:
-            y = torch.cat([q4.gemv(a[i:i + GEMV_MAX_ROWS].contiguous(), self.state)
+            y = torch.cat([q4.gemv(a[i:i + GEMV_MAX_ROWS].contiguous(), self.state, acc)
                            for i in range(0, T, GEMV_MAX_ROWS)])
         if self.bias is not None:
-            y = y + self.bias
+            y = (y + self.bias.float()).to(self.compute_dtype)
         return y.reshape(*lead, self.out_features)
 
     def extra_repr(self) -> str:

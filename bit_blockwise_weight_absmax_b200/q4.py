@@ -135,6 +135,22 @@ class Q4State:
         return self.packed.device
 
     def c_struct(self) -> _CState:
+        """The C view of the state, built once and rebuilt only when a buffer
+        or a field has changed."""
+        key = (self.qtype, self.src_dtype, self.rows, self.cols, self.blocksize, self.double_quant,
+               self.packed.data_ptr(), self.absmax.data_ptr(),
+               None if self.zero is None else self.zero.data_ptr(),
+               None if self.absmax_q is None else self.absmax_q.data_ptr(),
+               None if self.absmax_scale is None else self.absmax_scale.data_ptr(),
+               None if self.absmax_mean is None else self.absmax_mean.data_ptr())
+        cached = self.__dict__.get("_cs")
+        if cached is not None and cached[0] == key:
+            return cached[1]
+        s = self._build_c_struct()
+        self.__dict__["_cs"] = (key, s)
+        return s
+
+    def _build_c_struct(self) -> _CState:
         s = _CState()
         s.qtype = self.qtype
         s.src_dtype = _DT[self.src_dtype]
@@ -264,12 +280,19 @@ def dequantize(st: Q4State, dtype: torch.dtype | None = None, out: torch.Tensor 
     return out
 
 
-def _gemv_workspace(structs, M, device):
+_gemv_ws_need = {}  # (shapes and formats of the group, M) -> workspace bytes
+
+
+def _gemv_workspace(states, structs, M, device):
     arr = (ctypes.POINTER(_CState) * len(structs))(*[ctypes.pointer(s) for s in structs])
-    need = ctypes.c_size_t(0)
-    _check(library().q4_gemv_workspace_size(len(structs), arr, M, ctypes.byref(need)),
-           "q4_gemv_workspace_size")
-    return arr, _workspace(device, "gemv", need.value)
+    key = (tuple((s.rows, s.cols, s.blocksize, s.qtype, s.double_quant) for s in states), M)
+    need = _gemv_ws_need.get(key)
+    if need is None:
+        n = ctypes.c_size_t(0)
+        _check(library().q4_gemv_workspace_size(len(structs), arr, M, ctypes.byref(n)),
+               "q4_gemv_workspace_size")
+        need = _gemv_ws_need[key] = n.value
+    return arr, _workspace(device, "gemv", need)
 
 
 def gemv_grouped(As, states, out_dtype: torch.dtype | None = None, outs=None, stream=None):
@@ -279,7 +302,7 @@ def gemv_grouped(As, states, out_dtype: torch.dtype | None = None, outs=None, st
     a_dtype = As[0].dtype
     out_dtype = out_dtype or a_dtype
     structs = [s.c_struct() for s in states]
-    arr, ws = _gemv_workspace(structs, M, As[0].device)
+    arr, ws = _gemv_workspace(states, structs, M, As[0].device)
     if outs is None:
         outs = [torch.empty(M, s.rows, dtype=out_dtype, device=As[0].device) for s in states]
     a_ptrs = (ctypes.c_void_p * len(As))(*[a.data_ptr() for a in As])
