@@ -45,6 +45,11 @@ constexpr int kGemmBTile = kGemmBN * kGemmBK * 2;   // 16 KB
 constexpr int kGemmRawTile = kGemmBN * kGemmBK / 2; // 4 KB
 constexpr int kGemmStageBytes = kGemmATile + kGemmBTile + kGemmRawTile;
 constexpr int kGemmScBytes = kGemmBN * 16 * 4;     // c~ of 16 blocks per weight row
+constexpr int kGemmAccs = kGemmBM / 128;            // M=128 accumulators per tile
+constexpr int kGemmTpr = kGemmDqWarps * 32 / kGemmBN;  // dequant threads per weight row
+constexpr int kGemmCodes = kGemmBK / kGemmTpr;      // codes per thread and stage
+static_assert(kGemmBM % 128 == 0 && 2 * kGemmAccs * kGemmBN <= 512, "two accumulator sets in TMEM");
+static_assert(kGemmCodes == 16 || kGemmCodes == 32, "8 or 16 packed bytes per thread");
 constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmScBytes + 1024 /*align*/ + 256 /*barriers*/;
 
 struct alignas(64) GemmMat {
@@ -294,6 +299,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_f16(DA == Q4_BF16 ? 1 : 0, 128, kGemmBN);
+      static_assert(kGemmBN % 16 == 0 && kGemmBN <= 256, "UMMA N for M = 128");
       uint32_t it = 0, tcount = 0;
       for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++tcount) {
         const TileCoord tc = gemm_tile(p, t);
@@ -317,9 +323,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           for (int k16 = 0; k16 < kGemmBK / 16; ++k16) {
             const uint64_t db = umma_desc_sw128(b0 + 32 * k16);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t da = umma_desc_sw128(a0 + h * (kGemmATile / 2) + 32 * k16);
-              umma_f16(tmem + (uint32_t)(ab * 2 * kGemmBN + h * kGemmBN), da, db, idesc, (kb | k16) != 0);
+            for (int h = 0; h < kGemmAccs; ++h) {
+              const uint64_t da = umma_desc_sw128(a0 + h * (128 * kGemmBK * 2) + 32 * k16);
+              umma_f16(tmem + (uint32_t)((ab * kGemmAccs + h) * kGemmBN), da, db, idesc, (kb | k16) != 0);
             }
           }
           umma_commit(empty_bar(s));
@@ -337,11 +343,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
   } else {
     // ------------------------------------------------------------ dequant + epilogue
-    const int dt = tid - 64;        // 0..511
-    const int d = dt >> 2;          // weight row within the tile, 0..127
-    const int qk = dt & 3;          // k quarter of the 64-k block: codes 16 qk .. 16 qk + 15
-    const int q = warp & 3;         // TMEM lane quadrant of this warp
-    const int cc = (warp - 2) >> 2; // 32-column chunk handled in the epilogue
+    const int dt = tid - 64;           // 0..511
+    const int d = dt / kGemmTpr;       // weight row within the tile
+    const int qk = dt % kGemmTpr;      // part of the 64-k block: codes kGemmCodes qk .. + kGemmCodes - 1
+    const int q = warp & 3;            // TMEM lane quadrant of this warp
+    const int cc = (warp - 2) >> 2;    // quarter of the accumulator columns handled in the epilogue
     const uint32_t lvb = smem_u32(s_lv) + 4u * lane;
     // epilogue of a finished tile: its accumulator set -> Y
     // (the MMAs of the next tile go to the other accumulator set meanwhile)
@@ -351,11 +357,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         if (!mbar_wait_warp(accfull_bar(ab), (tcount >> 1) & 1, p.status, abort)) return false;
         tc_fence_after();
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
+        for (int piece = 0; piece < kGemmAccs * kGemmBN / 128; ++piece) {
+          const int h = piece / (kGemmBN / 128), part = piece % (kGemmBN / 128);
           const int mrow = tc.tm * kGemmBM + h * 128 + q * 32 + lane;
-          const int col0 = cc * 32;
+          const int col0 = cc * (kGemmBN / 4) + part * 32;
           uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * 2 * kGemmBN + h * kGemmBN + col0), r);
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((ab * kGemmAccs + h) * kGemmBN + col0), r);
           const int n0 = tc.tn * kGemmBN + col0;
           if (mrow < m.M && n0 < m.N) {
             if (p.y_dtype == Q4_F32) {
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const float mu = (DQ && row_ok) ? __ldg(m.absmax_mean) : 0.0f;
       const int64_t bi0 = (int64_t)min(row, m.N - 1) * nk;
       // block scales: the c~ of 16 blocks of the row at a time, computed by
-      // the row's four threads (four blocks each) from inputs requested 16
+      // the row's threads (parts of four blocks) from inputs requested 16
       // blocks ahead, kept in shared memory for the row
       struct In4 {
         uint32_t cw;     // int8 codes of four blocks (double quant)
@@ -407,8 +414,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         int bsplit;
         float f[4];      // fp32 absmax (no double quant)
       };
-      auto load4 = [&](int kb0, In4 &o) {  // blocks kb0 + 4 qk .. + 3
-        const int b0 = kb0 + 4 * qk;
+      constexpr int kParts = 4 / kGemmTpr;  // parts of four blocks per thread
+      auto load4 = [&](int kb0, int j, In4 &o) {  // blocks kb0 + 4 j .. + 3
+        const int b0 = kb0 + 4 * j;
         const int nv = max(0, min(4, nk - b0));
         const int64_t bi = bi0 + b0;
         if (nv == 0) {
@@ -437,7 +445,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         }
       };
       float *scrow = sSc + d * 16;
-      auto store4 = [&](const In4 &o) {
+      auto store4 = [&](int j, const In4 &o) {
         float v[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -449,15 +457,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           }
           if (!row_ok) v[e] = 0.0f;
         }
-        *reinterpret_cast<float4 *>(scrow + 4 * qk) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(scrow + 4 * j) = make_float4(v[0], v[1], v[2], v[3]);
       };
-      In4 nin;
+      In4 nin[kParts];
       {
-        In4 cin;
-        load4(0, cin);
-        if (nk > 16) load4(16, nin);
+        In4 cin[kParts];
+#pragma unroll
+        for (int j = 0; j < kParts; ++j) {
+          load4(0, qk * kParts + j, cin[j]);
+          if (nk > 16) load4(16, qk * kParts + j, nin[j]);
+        }
         __syncwarp();  // the row's previous c~ have been read
-        store4(cin);
+#pragma unroll
+        for (int j = 0; j < kParts; ++j) store4(qk * kParts + j, cin[j]);
         __syncwarp();
       }
       bool ok = true;
@@ -466,9 +478,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const uint32_t use = it / kGemmStages;
         if ((kb & 15) == 0 && kb > 0) {
           __syncwarp();  // the row's c~ of the previous 16 blocks have been read
-          store4(nin);
+#pragma unroll
+          for (int j = 0; j < kParts; ++j) store4(qk * kParts + j, nin[j]);
           __syncwarp();
-          if (kb + 16 < nk) load4(kb + 16, nin);
+#pragma unroll
+          for (int j = 0; j < kParts; ++j)
+            if (kb + 16 < nk) load4(kb + 16, qk * kParts + j, nin[j]);
         }
         const float sc = scrow[kb & 15];
         // lane 0 waits for the copy (acquire); the shuffle keeps the other
@@ -481,12 +496,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             break;
           }
         }
-        // 8 packed bytes = codes 16 qk .. 16 qk + 15 of row d
-        const uint2 raw = *reinterpret_cast<const uint2 *>(sR + s * kGemmRawTile + d * 32 + qk * 8);
+        // kGemmCodes / 2 packed bytes = codes kGemmCodes qk .. + kGemmCodes - 1 of row d
+        uint32_t rw[kGemmCodes / 8];
+        if constexpr (kGemmCodes == 16) {
+          const uint2 v = *reinterpret_cast<const uint2 *>(sR + s * kGemmRawTile + d * 32 + qk * 8);
+          rw[0] = v.x;
+          rw[1] = v.y;
+        } else {
+          const uint4 v = *reinterpret_cast<const uint4 *>(sR + s * kGemmRawTile + d * 32 + qk * 16);
+          rw[0] = v.x;
+          rw[1] = v.y;
+          rw[2] = v.z;
+          rw[3] = v.w;
+        }
         uint8_t *brow = sB + s * kGemmBTile + (d >> 3) * 1024 + (d & 7) * 128;
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {  // 16-byte chunk 2 qk + c2 = k 8 (2 qk + c2) .. + 7
-          const uint32_t w = c2 ? raw.y : raw.x;
+        for (int c2 = 0; c2 < kGemmCodes / 8; ++c2) {  // 16-byte chunk (kGemmCodes / 8) qk + c2
+          const uint32_t w = rw[c2];
           const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;  // codes 2j, 2j+1
           uint32_t o[4];
 #pragma unroll
@@ -496,7 +522,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             const float l1 = lds_f32((__byte_perm(hi, 0u, 0x4440u | j) << 7) + lvb);
             o[j] = Dt<DA>::pack2(__fmul_rn(sc, l0), __fmul_rn(sc, l1));
           }
-          const int c = 2 * qk + c2;
+          const int c = (kGemmCodes / 8) * qk + c2;
           *reinterpret_cast<uint4 *>(brow + ((c ^ (d & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         fence_proxy_async_smem();
