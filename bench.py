@@ -48,7 +48,7 @@ NCU_TRAFFIC = {
     "gemm": ("bit_blockwise_weight_absmax_b200/csrc/gemm.cuh",
              "cc2cae05ec917271dc3a06504db31924d52aee9ef0e71fa7e039c5ce0ab4c406", 166_176_000),
     "gemv": ("bit_blockwise_weight_absmax_b200/csrc/gemv_small.cuh",
-             "4a5865419667459d5280ac246fdeeb6ed954f677fa143dc2ec98c9f51966fe05", 112_599_552),
+             "baebb3e71f0ab0555bea7bcd0ee49bb76bee6a550cbe28753c64d8e7427d30b4", 112_599_552),
 }
 
 

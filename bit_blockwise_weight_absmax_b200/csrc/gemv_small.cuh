@@ -1,5 +1,8 @@
-// gemv_small.cuh -- fused NF4 dequant-GEMV for decode batches 1 <= M <= 16
-// (sm_100a), Y[M,N] = A[M,K] . W^[N,K]^T.
+// gemv_small.cuh -- fused 4-bit dequant-GEMV for decode batches (sm_100a),
+// Y[M,N] = A[M,K] . W^[N,K]^T for 1 <= M <= 16 activation rows per launch
+// (q4_gemv runs 16 < M <= 32 as two launches).  NF4 states use the 16-level
+// codebook and the block absmax c~; INT4 symmetric states the integers -8..7
+// and the group scale.
 //
 // What it computes: n4n.ai, "What is 4-bit quantization and why does it
 // matter?", "Why it matters for deployment" (decode at batch < 32 reads every
