@@ -87,6 +87,18 @@ def gemv_bytes(shapes, M):
     return layer_state_bytes(shapes) + sum(2 * M * K + 2 * M * N for _, N, K in shapes)
 
 
+def workload_config(L, world):
+    """The `config` of both arms' JSON lines: the 7B-layer workload."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    n_params = sum(N * K for _, N, K in wl.LAYER_7B)
+    state_b = layer_state_bytes(wl.LAYER_7B)
+    return {"workload": WORKLOAD, "decode_M": list(DECODE_M), "prefill_M": PREFILL_M,
+            "layer_copies": L, "blocksize": 64, "double_quant": True,
+            "l2": f"{L} rotating layer copies (~{L * 2 * n_params / 1e9:.1f} GB bf16 + "
+                  f"{L * state_b / 1e6:.0f} MB packed) > 126 MB L2",
+            "parallelism": f"replicas x{world}"}
+
+
 # ------------------------------------------------------------- replicas --
 def max_over_ranks(values, world, device=None):
     """Element-wise max over all ranks of per-rank device times (ms): the
@@ -222,7 +234,7 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": steps, "warmup": warm, "ms_per_step": statistics.mean(ms), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "decode_M": list(DECODE_M), "sample": "256 rows per matrix, scaled to the layer"},
+            "config": workload_config(args.copies, world),
             "quantize_gbs": statistics.mean(qs),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -505,11 +517,7 @@ def run_gpu(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic (seeded Gaussian weights of 7B-layer shapes; no checkpoint)",
-            "config": {"workload": WORKLOAD, "decode_M": list(DECODE_M), "prefill_M": PREFILL_M,
-                       "layer_copies": L, "blocksize": 64, "double_quant": True,
-                       "l2": f"{L} rotating layer copies (~{L * 2 * n_params / 1e9:.1f} GB bf16 + "
-                             f"{L * state_b / 1e6:.0f} MB packed) > 126 MB L2",
-                       "parallelism": f"replicas x{world}"},
+            "config": workload_config(L, world),
             "quantize_gbs": quant_gbs,
             "gemv_per_m": per_m,
             "phase_ms_per_step": {p: ph_ms[p] / args.steps for p in phases},
