@@ -61,3 +61,26 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks([3.5, 4.0], 1) == [3.5, 4.0]
     assert bench.whole_job_rate(5e8, 1, 2.0) == pytest.approx(2.5e11)
+
+
+def test_reference_arm_json_line(capsys):
+    """The reference arm (the oracle on the host) prints one JSON line with
+    the contract's keys and the same config as the GPU arm."""
+    import json
+
+    import bench
+
+    class A:
+        steps, warmup, copies = 1, 0, bench.N_COPIES
+    bench.run_reference(A, 0, 1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["higher_is_better"] is True and line["value"] > 0
+    assert line["config"] == bench.workload_config(bench.N_COPIES, 1)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
