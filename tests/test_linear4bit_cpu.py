@@ -43,3 +43,17 @@ def test_forward_without_gpu_fails_loudly():
         m(torch.zeros(2, 8))
     with pytest.raises(q4.Q4Error):
         m(torch.zeros(2, 7))  # wrong width is caught before any kernel call
+
+
+def test_state_c_struct_is_cached_and_rebuilt_on_change():
+    """The binding builds a state's C struct once and rebuilds it when a
+    buffer is replaced (the cache is keyed by every pointer and field)."""
+    st = _dummy_state()
+    a = st.c_struct()
+    assert st.c_struct() is a
+    assert a.packed == st.packed.data_ptr() and a.rows == 4 and a.cols == 8
+    st.packed = torch.zeros(16, dtype=torch.uint8)
+    b = st.c_struct()
+    assert b is not a and b.packed == st.packed.data_ptr()
+    st.blocksize = 32
+    assert st.c_struct().blocksize == 32
