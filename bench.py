@@ -534,6 +534,63 @@ def run_gpu(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_stack70b(args):
+    """The Llama-70B-shaped stack (80 layers; shape templates, synthetic
+    N(0, 0.015) bf16 weights generated per layer on the device, quantized to
+    NF4 blocksize 64 with double quantization, bf16 freed): decode GEMV over
+    the whole stack, one grouped launch per layer, at M = 1, 8, 32.  Prints
+    one JSON line; not part of the default step."""
+    import torch
+
+    from bit_blockwise_weight_absmax_b200 import q4
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    shapes = wl.LAYER_70B
+    t0 = time.perf_counter()
+    stack = []
+    for layer in range(wl.N_LAYERS_70B):
+        Ws = [wl.gaussian((N, K), 0.015, torch.bfloat16, 70000 + 16 * layer + i, dev)
+              for i, (_, N, K) in enumerate(shapes)]
+        stack.append([q4.quantize(w, 64, "nf4", True) for w in Ws])
+        del Ws
+    torch.cuda.synchronize()
+    load_s = time.perf_counter() - t0
+    resident = sum(st.resident_bytes() for sts in stack for st in sts)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    per_m = {}
+    for M in (1, 8, 32):
+        A = [wl.activation(M, K, torch.float16, 7 + i, dev) for i, (_, N, K) in enumerate(shapes)]
+        Y = [[torch.empty(M, N, dtype=torch.float16, device=dev) for _, N, K in shapes] for _ in stack]
+
+        def token_step():
+            for sts, ys in zip(stack, Y):
+                q4.gemv_grouped(A, sts, outs=ys)
+        token_step()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            token_step()
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+        e0, e1 = ev(), ev()
+        e0.record()
+        for _ in range(args.steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        nbytes = wl.N_LAYERS_70B * gemv_bytes(shapes, M)
+        per_m[f"M={M}"] = {"ms_per_token_step": ms, "tb_s": nbytes / (ms / 1e3) / 1e12,
+                           "bytes_per_token_step": nbytes}
+        del g, Y
+    print(json.dumps({"metric": "70B-stack decode GEMV effective HBM TB/s", "unit": "TB/s",
+                      "workload": "llama-70b-stack-80-layers-nf4-b64-dq", "resident_gb": resident / 1e9,
+                      "quantize_load_s": load_s, "steps": args.steps, "per_m": per_m,
+                      "note": "M=32 runs the decode kernel twice (the weights stream twice); "
+                              "bytes count them once"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -541,6 +598,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="q4", choices=["q4", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--stack70b", action="store_true",
+                    help="time the decode GEMV over the Llama-70B-shaped 80-layer stack instead (one JSON line)")
     ap.add_argument("--no-unfused", action="store_true",
                     help="skip timing the unfused dequantize-then-cuBLAS baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -558,6 +617,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.stack70b:
+        if rank == 0:
+            run_stack70b(args)
         return
     if world > 1:
         import datetime
