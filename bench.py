@@ -126,7 +126,8 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"q4_bench_clocks_rank{gpu_index}.csv")
 
     def start(self):
         try:

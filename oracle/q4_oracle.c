@@ -26,7 +26,7 @@
  *  [BNB]  mbrenndoerfer.com, "INT4 Quantization > Practical Implementation
  *         with bitsandbytes" (dequantize to fp16, then a 16-bit matmul).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *  - ties in nearest-level coding go to the level of smaller magnitude;
  *  - an all-zero block has c = 0, every x = 0, and dequantizes to 0;
  *  - INT4 asymmetric widens [min, max] to include 0; scale and zero-point
