@@ -130,3 +130,63 @@ def test_invalid_arguments_rejected_on_host(lib):
     assert lib.q4_state_sizes(0, 0, 64, 0, out) == -2       # empty
     with pytest.raises(q4.Q4Error):
         q4.state_sizes("int4_sym", 100, 64, True)
+
+
+def _fake_state(qtype, rows, cols, bs, dq):
+    """A q4_state whose device pointers are placeholders: the host-side
+    checks below never dereference them."""
+    from bit_blockwise_weight_absmax_b200 import q4
+    s = q4._CState()
+    s.qtype, s.src_dtype, s.rows, s.cols, s.n = qtype, 1, rows, cols, rows * cols
+    s.blocksize, s.double_quant, s.dq_group = bs, int(dq), 256
+    s.packed, s.absmax = 0x10000, 0x20000
+    s.zero = 0x30000 if qtype == 2 else None
+    if dq:
+        s.absmax_q, s.absmax_scale, s.absmax_mean = 0x40000, 0x50000, 0x60000
+    return s
+
+
+def _gemv(lib, states, M):
+    from bit_blockwise_weight_absmax_b200 import q4
+    n = len(states)
+    arr = (ctypes.POINTER(q4._CState) * n)(*[ctypes.pointer(s) for s in states])
+    ptrs = (ctypes.c_void_p * n)(*([0x70000] * n))
+    return lib.q4_gemv_grouped(n, ptrs, arr, ptrs, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None)
+
+
+def test_gemv_workspace_two_passes_share_the_sixteen_row_size(lib):
+    """16 < M <= 32 runs the decode kernel twice on one workspace: the size
+    for any such M is the size for 16 rows (slots of 16 columns), and M <= 8
+    needs less (slots of 8 columns)."""
+    from bit_blockwise_weight_absmax_b200 import q4
+    sts = [_fake_state(0, 4096, 4096, 64, True), _fake_state(0, 11008, 4096, 64, True)]
+    arr = (ctypes.POINTER(q4._CState) * 2)(*[ctypes.pointer(s) for s in sts])
+
+    def size(M):
+        out = ctypes.c_size_t(0)
+        assert lib.q4_gemv_workspace_size(2, arr, M, ctypes.byref(out)) == 0
+        return out.value
+    s16 = size(16)
+    assert all(size(M) == s16 for M in (9, 17, 24, 32))
+    assert size(1) == size(8) < s16
+    out = ctypes.c_size_t(0)
+    assert lib.q4_gemv_workspace_size(2, arr, 33, ctypes.byref(out)) == -2
+    assert lib.q4_gemv_workspace_size(2, arr, 0, ctypes.byref(out)) == -2
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_gemv_host_checks_before_the_device(lib):
+    """The GEMV's format checks run on the host, matrix by matrix, before
+    any device work: INT4 asymmetric states are rejected (Q4_ERR_ARG); NF4
+    and INT4 symmetric states pass them and stop at the missing GPU; M
+    outside 1..32 is a shape error."""
+    nf4 = _fake_state(0, 256, 512, 64, True)
+    sym = _fake_state(1, 256, 512, 128, False)
+    asym = _fake_state(2, 256, 512, 128, False)
+    assert _gemv(lib, [asym], 1) == -1
+    assert _gemv(lib, [asym], 24) == -1          # the first of the two passes rejects it too
+    assert _gemv(lib, [nf4], 1) == -4            # Q4_ERR_NO_DEVICE
+    assert _gemv(lib, [sym], 16) == -4
+    assert _gemv(lib, [nf4], 32) == -4
+    assert _gemv(lib, [nf4], 33) == -2
+    assert _gemv(lib, [nf4], 0) == -2
