@@ -208,6 +208,21 @@ def test_gemv_rejects_int4_asym(q4):
         q4.gemv(dev(torch.randn(1, 128).half()), st)
 
 
+def test_gemv_grouped_rejects_mixed_formats(q4):
+    """One grouped launch takes one format: a second matrix with another
+    double-quant flag or quantization type is rejected on the host, before
+    any launch."""
+    W = dev(torch.randn(256, 512).half())
+    a = q4.quantize(W, 64, "nf4", True)
+    b = q4.quantize(W, 64, "nf4", False)
+    c = q4.quantize(W, 64, "int4_sym", False)
+    A = [dev(torch.randn(1, 512).half()) for _ in range(2)]
+    for pair in ((a, b), (a, c), (c, a)):
+        with pytest.raises(q4.Q4Error):
+            q4.gemv_grouped(A, list(pair))
+    assert q4.last_device_status() == 0
+
+
 def test_gemv_fp32_output_tight(q4, oracle):
     """fp32 output against the unrounded reference: the fused path's own error
     (fp16 codebook values, fp32 accumulation) stays far below the tolerance."""
