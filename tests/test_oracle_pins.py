@@ -5,6 +5,7 @@ Each test names what pins it: printed values (tests/golden/), library
 routines (numpy / torch conversions and matmul), exact rational arithmetic
 (fractions.Fraction), closed forms, invariants and brute force on tiny inputs.
 """
+import os
 from fractions import Fraction
 
 import numpy as np
@@ -441,3 +442,137 @@ def test_storage_arithmetic_matches_pages(oracle):
         mib = G["meta_params"] / 1e9 * 2 ** 30 / g * 2 / 2 ** 20
         assert mib == G[key + "_mb"]
         assert round(mib / (G["meta_weights_gb"] * 1000) * 100, 1) == G[key + "_pct"]
+
+
+# ------------------------------------- INT4 asym: closed forms, exactly -----
+# robotsatlas.com, "INT4", "How it works": each group's range is fit into
+# [0, 15]; "Components" (Zero-point): an integer offset lets a group whose
+# values are not centred on zero use all 16 levels.  With the range widened
+# to include 0 (so 0 stays exactly representable), the scale is the range
+# over the 15 steps between level 0 and level 15, and the zero-point is the
+# level that 0 falls on.  These pins evaluate that closed form with exact
+# rationals on the exact 16-bit inputs, rounding to binary32 only where a
+# binary32 operation stands: the difference, the quotient by 15, -mn / s.
+
+def _rne32(x: Fraction) -> Fraction:
+    """Round an exact rational to the nearest binary32 (ties to even)."""
+    if x == 0:
+        return Fraction(0)
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, -126)  # subnormal quantum below 2^-126
+    quantum = Fraction(2) ** (e - 23)
+    r = round(a / quantum)  # Python rounds a Fraction half to even
+    return (r * quantum) if x > 0 else -(r * quantum)
+
+
+def int4_asym_pin_failures(wf: np.ndarray, st) -> list:
+    """Every closed-form check that the state of INT4 asymmetric groups
+    (rows of `wf`, the exact binary32 values of the 16-bit inputs) fails."""
+    nb, B = wf.shape
+    z = np.stack([st.zero & 0xF, st.zero >> 4], -1).reshape(-1)[:nb].astype(np.int64)
+    q = st.codes().astype(np.int64).reshape(nb, B)
+    bad = []
+    for b in range(nb):
+        vals = [Fraction(float(v)) for v in wf[b]]
+        mn, mx = min(min(vals), Fraction(0)), max(max(vals), Fraction(0))
+        s = _rne32(_rne32(mx - mn) / 15)
+        if Fraction(float(st.absmax[b])) != s:
+            bad.append(("scale", b))
+            continue
+        if s == 0:
+            if z[b] != 0 or np.any(q[b] != 0):
+                bad.append(("zero-range", b))
+            continue
+        zz = min(max(round(_rne32(-mn / s)), 0), 15)
+        if z[b] != zz:
+            bad.append(("zero-point", b))
+            continue
+        # the dequantized ends of the level range sit within s/2 (plus the
+        # binary32 roundings of s) of the widened group minimum and maximum
+        slack = s / 2 + abs(mx - mn) * Fraction(1, 2 ** 22)
+        if abs(-zz * s - mn) > slack or abs((15 - zz) * s - mx) > slack:
+            bad.append(("endpoints", b))
+        for j in range(B):
+            qq = min(max(round(_rne32(vals[j] / s)) + zz, 0), 15)
+            if q[b, j] != qq:
+                bad.append(("code", b, j))
+                break
+    return bad
+
+
+def _asym_groups(dt, seed):
+    """Groups of 32 covering the cases the rule distinguishes: centred and
+    offset Gaussians, all-positive and all-negative groups (the widening to
+    0), constant and all-zero groups, tiny and large magnitudes."""
+    g = torch.Generator().manual_seed(seed)
+    B = 32
+    rows = [torch.randn(B, generator=g) * 0.02 + off for off in (0.0, 0.01, -0.015, 0.05)]
+    rows += [torch.rand(B, generator=g) * 0.3 + 0.01, -(torch.rand(B, generator=g) * 0.3 + 0.01)]
+    rows += [torch.full((B,), 0.125), torch.zeros(B), torch.randn(B, generator=g) * 1e-4,
+             torch.randn(B, generator=g) * 300.0]
+    rows += [torch.randn(B, generator=g) * s for s in torch.rand(40, generator=g).mul(4).exp().tolist()]
+    w = torch.stack(rows).to(dt)
+    return w, B
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_int4_asym_scale_and_zero_point_closed_form(oracle, dt):
+    """s = fl32(fl32(mx - mn) / 15) and z = clamp(rint(fl32(-mn / s)), 0, 15)
+    on every group, exactly; the levels 0 and 15 dequantize to within s/2 of
+    the widened group minimum and maximum."""
+    w, B = _asym_groups(dt, 31)
+    bits = w.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    st = oracle.quantize(bits, dt == torch.bfloat16, B, oracle.QT_INT4_ASYM)
+    assert int4_asym_pin_failures(w.float().numpy(), st) == []
+
+
+def _mutated_oracle(tmp_path, old, new):
+    """The oracle source with one planted mistake, built into its own .so."""
+    import ctypes
+    import subprocess
+    src = open(os.path.join(os.path.dirname(oracle_module_file()), "q4_oracle.c")).read()
+    assert src.count(old) == 1, old
+    path = tmp_path / "mut.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "mut.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", str(path),
+                    "-o", str(so), "-lm"], check=True, capture_output=True)
+    lib = ctypes.CDLL(str(so))
+    P = ctypes.c_void_p
+    lib.oracle_quantize.argtypes = [P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, P, P, P, P, P, P]
+    lib.oracle_quantize.restype = None
+    return lib
+
+
+def oracle_module_file():
+    import oracle as o
+    return o.__file__
+
+
+@pytest.mark.parametrize("old,new", [
+    ("float s = (mx - mn) / 15.0f;", "float s = (mx - mn) / 16.0f;"),
+    ("z = clampi((int)rintf(-mn / s), 0, 15);", "z = clampi((int)floorf(-mn / s), 0, 15);"),
+    ("q = clampi((int)rintf(to_f32(w[j], is_bf16) / s) + z, 0, 15);",
+     "q = clampi((int)floorf(to_f32(w[j], is_bf16) / s) + z, 0, 15);"),
+    ("float mn = 0.0f, mx = 0.0f;", "float mn = 3e38f, mx = -3e38f;"),
+])
+def test_int4_asym_pins_catch_planted_mistakes(oracle, tmp_path, old, new):
+    """Each plausible slip in the asymmetric rule (divisor 16, floor for the
+    zero-point or the code, no widening to include 0), planted in a copy of
+    the oracle, fails the closed-form pins."""
+    import ctypes
+    w, B = _asym_groups(torch.float16, 31)
+    bits = np.ascontiguousarray(w.view(torch.int16).numpy().view(np.uint16).reshape(-1))
+    lib = _mutated_oracle(tmp_path, old, new)
+    n = bits.size
+    nb = n // B
+    st = oracle.State(oracle.QT_INT4_ASYM, n, B, 0, np.zeros(n // 2, np.uint8), np.zeros(nb, np.float32),
+                      np.zeros((nb + 1) // 2, np.uint8), None, None, None)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    lib.oracle_quantize(p(bits), 0, n, B, oracle.QT_INT4_ASYM, 0, p(st.packed), p(st.absmax),
+                        p(st.zero), None, None, None)
+    assert int4_asym_pin_failures(w.float().numpy(), st) != []
