@@ -7,13 +7,7 @@ namespace q4 {
 namespace {
 template <int DA, bool DQ>
 int go(const GemmParams &p, int sms, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(gemm_kernel<DA, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) !=
-        cudaSuccess)
-      return Q4_ERR_CUDA;
-    attr = true;
-  }
+  if (set_smem_attr_once<gemm_kernel<DA, DQ>>(kGemmSmem, false) != Q4_OK) return Q4_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(p.total_tiles, (int64_t)sms);
   launch_pdl(gemm_kernel<DA, DQ>, dim3(grid), dim3(kGemmThreads), kGemmSmem, st, p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;

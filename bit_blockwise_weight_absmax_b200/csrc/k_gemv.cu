@@ -13,15 +13,8 @@ int go_small(const GsParams &p, int sms, cudaStream_t st) {
   // 16-row groups per compute warp: M <= 8 fits 16 compute warps (+ the
   // producer) in the registers; M <= 16 uses 8 warps of 32 rows
   constexpr int R = NT == 1 ? 1 : 2;
-  auto kern = gemv_small_kernel<DA, NT, B, R>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGsSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-      return Q4_ERR_CUDA;
-    attr = true;
-  }
+  constexpr auto kern = gemv_small_kernel<DA, NT, B, R>;
+  if (set_smem_attr_once<kern>(kGsSmemBytes, true) != Q4_OK) return Q4_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(p.total_stages, (int64_t)std::min(sms, kGsMaxCtas));
   launch_pdl(kern, dim3(grid), dim3(GsShape<R>::kThreads), kGsSmemBytes, st, p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;

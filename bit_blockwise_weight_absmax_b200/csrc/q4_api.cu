@@ -431,7 +431,9 @@ int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *
   if (count < 1 || count > kGsMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
-  if (!Wq[0]) return Q4_ERR_ARG;
+  // every entry is checked before any of them is dereferenced
+  for (int i = 0; i < count; ++i)
+    if (!Wq[i] || !A[i] || !Y[i]) return Q4_ERR_ARG;
   if (M <= kGemvPassRows)
     return gemv_small_grouped(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
   // two passes of the decode kernel: activation rows 0..15, then 16..M-1
@@ -463,6 +465,8 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (y_dtype != Q4_F32 && y_dtype != a_dtype) return Q4_ERR_ARG;
   if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;
+  for (int i = 0; i < count; ++i)
+    if (!Wq[i] || !A[i] || !Y[i]) return Q4_ERR_ARG;
   const DeviceInfo di = device_info();
   static thread_local GemmParams p;  // host staging of the kernel parameters (~5 KB)
   memset(&p, 0, sizeof(p));

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <utility>
 
 #include "q4_common.cuh"
@@ -29,6 +30,30 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Raise a kernel's dynamic shared-memory limit (and, optionally, its
+// shared-memory carveout) once per device: the attribute is per device, and
+// the first calls on a device may come from several threads at once.
+constexpr int kMaxDevices = 64;
+template <auto Kern>
+int set_smem_attr_once(int bytes, bool max_carveout) {
+  static std::once_flag once[kMaxDevices];
+  static int rc[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return Q4_ERR_CUDA;
+  }
+  std::call_once(once[dev], [&] {
+    bool ok = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+    if (ok && max_carveout)
+      ok = cudaFuncSetAttribute(Kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+    if (!ok) cudaGetLastError();
+    rc[dev] = ok ? Q4_OK : Q4_ERR_CUDA;
+  });
+  return rc[dev];
 }
 
 int run_quantize(int dt, int qt, int bs, bool dq, const QuantParams &p, int grid, cudaStream_t st);

@@ -8,7 +8,8 @@ the compute dtype for the matmul; the output head and the normalisation
 layers stay in 16 bits.  Here the dequantization is fused into the kernels:
 up to 32 rows of activations run the decode GEMV, more rows the W4A16
 tcgen05 GEMM (NF4, blocksize 64, N % 16 == 0), other formats run the GEMV
-32 rows at a time.  All compute is on the GPU; there is no CPU path.
+32 rows at a time.  A format neither consumer takes is refused when the
+module is built.  All compute is on the GPU; there is no CPU path.
 """
 from __future__ import annotations
 
@@ -27,6 +28,9 @@ class Linear4bit(torch.nn.Module):
         super().__init__()
         if compute_dtype not in (torch.float16, torch.bfloat16):
             raise q4.Q4Error("compute_dtype must be torch.float16 or torch.bfloat16")
+        why = unsupported_reason(state)
+        if why:
+            raise q4.Q4Error(f"Linear4bit cannot run this state: {why}")
         self.state = state
         self.in_features = state.cols
         self.out_features = state.rows
@@ -36,12 +40,21 @@ class Linear4bit(torch.nn.Module):
 
     @classmethod
     def from_linear(cls, lin: torch.nn.Linear, blocksize: int = 64, qtype: str = "nf4",
-                    double_quant: bool = True, compute_dtype: torch.dtype = torch.float16) -> "Linear4bit":
-        """Quantize an nn.Linear's weight (on its CUDA device) once, at load time."""
+                    double_quant: bool = True, compute_dtype: torch.dtype = torch.float16,
+                    keep_absmax: bool = False) -> "Linear4bit":
+        """Quantize an nn.Linear's weight (on its CUDA device) once, at load
+        time.  With double quantization the fp32 block absmax, which no
+        consumer reads, is released unless `keep_absmax`."""
+        qt = q4.QTYPES[qtype] if isinstance(qtype, str) else int(qtype)
+        why = unsupported_reason_of(qt, blocksize, lin.in_features)
+        if why:
+            raise q4.Q4Error(f"Linear4bit cannot run this format: {why}")
         w = lin.weight.detach()
         if w.dtype not in (torch.float16, torch.bfloat16):
             w = w.to(torch.bfloat16)
-        st = q4.quantize(w.contiguous(), blocksize, qtype, double_quant)
+        st = q4.quantize(w.contiguous(), blocksize, qt, double_quant)
+        if double_quant and not keep_absmax:
+            st.release_absmax()
         return cls(st, lin.bias, compute_dtype)
 
     def _gemm_ok(self) -> bool:
@@ -77,6 +90,41 @@ class Linear4bit(torch.nn.Module):
         return (f"in_features={self.in_features}, out_features={self.out_features}, {kind}, "
                 f"blocksize={st.blocksize}, double_quant={st.double_quant}, "
                 f"compute_dtype={self.compute_dtype}")
+
+
+def unsupported_reason_of(qtype: int, blocksize: int, in_features: int) -> str | None:
+    """Why the fused consumers cannot run a format, or None when they can:
+    the GEMV needs whole blocks per row (in_features % blocksize == 0) and
+    does not take INT4 asymmetric states."""
+    if qtype == q4.INT4_ASYM:
+        return "INT4 asymmetric states have no fused consumer"
+    if qtype not in (q4.NF4, q4.INT4_SYM):
+        return f"unknown qtype {qtype}"
+    if blocksize not in (32, 64, 128, 256):
+        return f"blocksize {blocksize} is not 32, 64, 128 or 256"
+    if in_features % blocksize:
+        return f"in_features {in_features} is not a multiple of the blocksize {blocksize}"
+    return None
+
+
+def unsupported_reason(st: q4.Q4State) -> str | None:
+    return unsupported_reason_of(st.qtype, st.blocksize, st.cols)
+
+
+def memory_footprint(module: torch.nn.Module) -> int:
+    """Bytes a module holds: every distinct parameter and buffer (a weight
+    tied between two layers counts once) plus the buffers of every
+    Linear4bit's quantized state."""
+    total = 0
+    seen = set()
+    for t in list(module.parameters()) + list(module.buffers()):
+        if id(t) not in seen:
+            seen.add(id(t))
+            total += t.numel() * t.element_size()
+    for m in module.modules():
+        if isinstance(m, Linear4bit):
+            total += m.state.held_bytes()
+    return total
 
 
 def linears_to_replace(module: torch.nn.Module, skip=("lm_head",)) -> list:

@@ -120,7 +120,7 @@ class Q4State:
     blocksize: int
     double_quant: bool
     packed: torch.Tensor
-    absmax: torch.Tensor
+    absmax: torch.Tensor | None  # with double quantization no consumer reads it
     zero: torch.Tensor | None = None
     absmax_q: torch.Tensor | None = None
     absmax_scale: torch.Tensor | None = None
@@ -138,7 +138,7 @@ class Q4State:
         """The C view of the state, built once and rebuilt only when a buffer
         or a field has changed."""
         key = (self.qtype, self.src_dtype, self.rows, self.cols, self.blocksize, self.double_quant,
-               self.packed.data_ptr(), self.absmax.data_ptr(),
+               self.packed.data_ptr(), None if self.absmax is None else self.absmax.data_ptr(),
                None if self.zero is None else self.zero.data_ptr(),
                None if self.absmax_q is None else self.absmax_q.data_ptr(),
                None if self.absmax_scale is None else self.absmax_scale.data_ptr(),
@@ -161,12 +161,26 @@ class Q4State:
         s.double_quant = int(self.double_quant)
         s.dq_group = DQ_GROUP
         s.packed = self.packed.data_ptr()
-        s.absmax = self.absmax.data_ptr()
+        s.absmax = None if self.absmax is None else self.absmax.data_ptr()
         s.zero = None if self.zero is None else self.zero.data_ptr()
         s.absmax_q = None if self.absmax_q is None else self.absmax_q.data_ptr()
         s.absmax_scale = None if self.absmax_scale is None else self.absmax_scale.data_ptr()
         s.absmax_mean = None if self.absmax_mean is None else self.absmax_mean.data_ptr()
         return s
+
+    def release_absmax(self):
+        """Drop the fp32 block absmax of a double-quantized state: the
+        consumers read the 8-bit codes, their scales and the mean instead, so
+        the fp32 copy (0.5 bit per weight at blocksize 64) is only needed to
+        inspect the state."""
+        if not self.double_quant:
+            raise Q4Error("the fp32 absmax is the block scale of a state without double quantization")
+        self.absmax = None
+
+    def held_bytes(self) -> int:
+        """Device bytes of every buffer the state still holds."""
+        return sum(t.numel() * t.element_size() for t in (self.packed, self.absmax, self.zero, self.absmax_q,
+                                                         self.absmax_scale, self.absmax_mean) if t is not None)
 
     def resident_bytes(self) -> int:
         """Bytes of the format a consumer reads (codes + block state); with
@@ -249,6 +263,8 @@ def quantize(W: torch.Tensor, blocksize: int = 64, qtype="nf4", double_quant: bo
         if (out.qtype, out.rows, out.cols, out.blocksize, out.double_quant) != \
                 (qt, rows, cols, blocksize, bool(double_quant)):
             raise Q4Error("out= state has a different shape or format")
+        if out.absmax is None:
+            raise Q4Error("out= state has released its absmax buffer, which quantize writes")
         out.src_dtype = W.dtype
     st = out if out is not None else Q4State(qt, W.dtype, rows, cols, blocksize, bool(double_quant),
                  packed=torch.empty(sz[0], dtype=torch.uint8, device=dev),

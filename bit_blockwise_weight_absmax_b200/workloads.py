@@ -69,3 +69,14 @@ def layer_weights(shapes, std: float, seed: int, dtype=torch.bfloat16, device="c
 
 def activation(M: int, K: int, dtype, seed: int, device="cpu") -> torch.Tensor:
     return gaussian((M, K), 1.0, dtype, seed, device)
+
+
+# Decoder-only model layouts for the memory-footprint checks (shape templates
+# only; no weights): hidden size, MLP size, layers, attention heads, KV heads,
+# vocabulary, whether the output head shares the embedding matrix.
+# A 135M-class small model (the scale of the demo on
+# learn.pranaymahendrakar.com, "Loading a model in 4-bit", "The walkthrough":
+# 269 MB at fp16) and the Llama-70B-shaped stack of LAYER_70B.
+LAYOUT_135M = dict(hidden=576, inter=1536, layers=30, heads=9, kv_heads=3, vocab=49152, tied=True)
+LAYOUT_70B = dict(hidden=8192, inter=28672, layers=N_LAYERS_70B, heads=64, kv_heads=8, vocab=32000,
+                  tied=False)

@@ -190,3 +190,23 @@ def test_gemv_host_checks_before_the_device(lib):
     assert _gemv(lib, [nf4], 32) == -4
     assert _gemv(lib, [nf4], 33) == -2
     assert _gemv(lib, [nf4], 0) == -2
+
+
+def test_grouped_calls_reject_a_null_entry_before_any_use(lib):
+    """A NULL state, activation or output pointer in any entry of a grouped
+    call is Q4_ERR_ARG, found before the library reads any entry (a NULL
+    second state used to be dereferenced while sizing the workspace)."""
+    from bit_blockwise_weight_absmax_b200 import q4
+    good = _fake_state(0, 256, 512, 64, True)
+    P = ctypes.POINTER(q4._CState)
+    for M in (1, 24):
+        arr = (P * 2)(ctypes.pointer(good), P())
+        ptrs = (ctypes.c_void_p * 2)(0x70000, 0x70000)
+        assert lib.q4_gemv_grouped(2, ptrs, arr, ptrs, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None) == -1
+        assert lib.q4_gemm_grouped(2, ptrs, arr, ptrs, 512, 1, 1, None) == -1
+        arr = (P * 2)(ctypes.pointer(good), ctypes.pointer(good))
+        for bad in ((ctypes.c_void_p * 2)(0x70000, None),):
+            assert lib.q4_gemv_grouped(2, bad, arr, ptrs, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None) == -1
+            assert lib.q4_gemv_grouped(2, ptrs, arr, bad, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None) == -1
+            assert lib.q4_gemm_grouped(2, bad, arr, ptrs, 512, 1, 1, None) == -1
+            assert lib.q4_gemm_grouped(2, ptrs, arr, bad, 512, 1, 1, None) == -1

@@ -26,9 +26,9 @@ def test_linears_to_replace_keeps_head_embeddings_norms():
     assert "lm_head" in linear4bit.linears_to_replace(_Toy(), skip=())
 
 
-def _dummy_state():
-    z = torch.zeros(16, dtype=torch.uint8)
-    return q4.Q4State(q4.NF4, torch.float16, 4, 8, 64, False, z, torch.zeros(1))
+def _dummy_state(qtype=q4.NF4, cols=64, blocksize=64):
+    z = torch.zeros(4 * cols // 2, dtype=torch.uint8)
+    return q4.Q4State(qtype, torch.float16, 4, cols, blocksize, False, z, torch.zeros(4 * cols // blocksize))
 
 
 def test_rejects_fp32_compute_dtype():
@@ -38,11 +38,23 @@ def test_rejects_fp32_compute_dtype():
 
 def test_forward_without_gpu_fails_loudly():
     m = linear4bit.Linear4bit(_dummy_state())
-    assert m.in_features == 8 and m.out_features == 4
+    assert m.in_features == 64 and m.out_features == 4
     with pytest.raises(q4.Q4Error):
-        m(torch.zeros(2, 8))
+        m(torch.zeros(2, 64))
     with pytest.raises(q4.Q4Error):
         m(torch.zeros(2, 7))  # wrong width is caught before any kernel call
+
+
+def test_refuses_formats_no_consumer_runs():
+    """A state the GEMV/GEMM cannot consume is refused when the module is
+    built, not at its first forward pass."""
+    with pytest.raises(q4.Q4Error, match="asymmetric"):
+        linear4bit.Linear4bit(_dummy_state(q4.INT4_ASYM, 128, 128))
+    with pytest.raises(q4.Q4Error, match="multiple"):
+        linear4bit.Linear4bit(_dummy_state(q4.NF4, 96, 64))
+    with pytest.raises(q4.Q4Error, match="asymmetric"):
+        linear4bit.Linear4bit.from_linear(torch.nn.Linear(128, 8), 128, "int4_asym")
+    linear4bit.Linear4bit(_dummy_state(q4.INT4_SYM, 128, 128))
 
 
 def test_state_c_struct_is_cached_and_rebuilt_on_change():
@@ -51,7 +63,7 @@ def test_state_c_struct_is_cached_and_rebuilt_on_change():
     st = _dummy_state()
     a = st.c_struct()
     assert st.c_struct() is a
-    assert a.packed == st.packed.data_ptr() and a.rows == 4 and a.cols == 8
+    assert a.packed == st.packed.data_ptr() and a.rows == 4 and a.cols == 64
     st.packed = torch.zeros(16, dtype=torch.uint8)
     b = st.c_struct()
     assert b is not a and b.packed == st.packed.data_ptr()

@@ -71,3 +71,29 @@ def test_replace_linear_on_a_small_model(mods):
     rel16 = ((y - ref16).norm() / ref16.norm()).item()
     assert rel16 < 0.25, rel16
     assert q4.last_device_status() == 0
+
+
+def test_replace_linear_footprint_small_model(mods):
+    """learn.pranaymahendrakar.com, "Loading a model in 4-bit": the 135M demo
+    goes from 269 MB at fp16 to about 110 MB, 2.4x, because embeddings, the
+    tied output head and the norms stay 16-bit.  The same layout, quantized
+    for real by replace_linear (NF4, blocksize 64, double quantization), holds
+    exactly the bytes the planned CPU footprint gives, and still runs."""
+    linear4bit, q4 = mods
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    from model_layouts import DecoderSkeleton
+    torch.manual_seed(0)
+    model = DecoderSkeleton(wl.LAYOUT_135M, device="cuda", dtype=torch.float16)
+    fp16 = linear4bit.memory_footprint(model)
+    linear4bit.replace_linear(model, blocksize=64, qtype="nf4", double_quant=True)
+    b4 = linear4bit.memory_footprint(model)
+    assert type(model.lm_head) is torch.nn.Linear
+    assert model.lm_head.weight is model.embed_tokens.weight
+    assert round(fp16 / 1e6) == 269 and abs(b4 / 1e6 - 110) < 3
+    assert round(fp16 / b4, 1) == 2.4
+    blk = model.layers[0]
+    assert isinstance(blk.down_proj, linear4bit.Linear4bit) and blk.down_proj.state.absmax is None
+    x = torch.randn(3, 576, device="cuda").half()
+    y = blk.down_proj(blk.gate_proj(x))
+    assert y.shape == (3, 576) and torch.isfinite(y).all()
+    assert q4.last_device_status() == 0
