@@ -106,25 +106,28 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait: gives up after ~2 s, raises Q4_STATUS_TIMEOUT and sets *abort.
-// The first probe is inlined; only a phase that is not yet complete pays the
-// call into the polling loop.
+// Bounded wait: gives up after `limit_ns` (2 s unless the launch sets a
+// limit), raises Q4_STATUS_TIMEOUT and sets *abort.  The first probe is
+// inlined; only a phase that is not yet complete pays the call into the
+// polling loop.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, int *status,
-                                                   volatile int *abort) {
+                                                   volatile int *abort, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > 2000000000ull) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       raise_status(status, Q4_STATUS_TIMEOUT);
       *abort = 1;
       return false;
     }
   }
 }
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *status, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *status, volatile int *abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, status, abort);
+  return mbar_wait_slow(bar, parity, status, abort, limit_ns);
 }
 
 // Wait by a whole warp: only lane 0 polls the barrier (many polling lanes
@@ -132,9 +135,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *st
 // the result is broadcast.  Must be called by all 32 lanes.
 // After lane 0 has seen the phase complete, each other lane queries it once
 // (returns at once) so that it acquires the data the phase published itself.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int *status, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int *status, volatile int *abort,
+                                               uint64_t limit_ns = kWaitLimitNs) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort, limit_ns);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   if (ok && (threadIdx.x & 31) != 0) (void)mbar_try(bar, parity);
   return ok;

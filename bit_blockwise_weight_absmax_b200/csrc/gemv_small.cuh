@@ -11,6 +11,8 @@
 // to the compute dtype, then a 16-bit matmul); the dequantization is fused
 // into the streaming of the packed weights.
 //
+// INT4 asymmetric states run the one-pass kernel of gemv.cuh instead.
+//
 // Design (B200, decode sizes).  At M <= 16 a tcgen05 MMA (128 x 16 x 16
 // takes ~44 cycles) would cap the kernel near the HBM rate, while the
 // warp-level mma.sync path (m16n8k16) has ample headroom; what limits a
@@ -104,6 +106,8 @@ struct GsParams {
   uint32_t total_stages;  // below 2^32 / kGsMaxCtas, so c * T fits 32 bits
   float *slots;     // [grid][2][256 rows][8 NT] fp32 partial rows of each CTA's first / last tile
   int *status;
+  uint64_t wait_ns;  // bound of every mbarrier wait
+  int32_t stall_copies;  // test hook: issue no copies, so every stage wait runs out
   float levels[16];
 };
 
@@ -437,9 +441,10 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
         if (gi != g0) u = gs_next<B>(info, p.count, u, gi, g0, g1);
         const GsMat &mt = p.mat[u.mi];
         for (int q = u.q0; q < u.q1; ++q) {
-          if (!mbar_wait(sempty(s), ph ^ 1u, p.status, abort)) { ok = false; break; }
+          if (!mbar_wait(sempty(s), ph ^ 1u, p.status, abort, p.wait_ns)) { ok = false; break; }
           // the compute warps' reads of this slot (generic proxy) come before
           // the copy that overwrites it (async proxy)
+          if (p.stall_copies) continue;
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(sfull(s), tx);
           const uint32_t st = stage_addr(s);
@@ -576,7 +581,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
       // lanes' reads of the stage after it
       {
         bool ready = true;
-        if (lane == 0) ready = mbar_wait(sfull(s), ph, p.status, abort);
+        if (lane == 0) ready = mbar_wait(sfull(s), ph, p.status, abort, p.wait_ns);
         if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) { ok = false; break; }
       }
       const uint32_t st = stage_addr(s);

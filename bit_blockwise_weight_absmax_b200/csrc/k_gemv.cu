@@ -1,43 +1,18 @@
-// k_gemv.cu -- launchers of the fused dequant-GEMV (decode) kernel.
-#include <algorithm>
-
+// k_gemv.cu -- dispatch of the one-pass decode GEMV (gemv.cuh), which runs
+// INT4 asymmetric states; its instantiations live in k_gemv_{f16,bf16}_asym.cu.
 #include "q4_internal.h"
 
 namespace q4 {
-namespace {
 
-// The mma.sync kernel: one CTA per SM with all of its shared memory (the
-// kernel lays out its table, buffers and ring itself).
-template <int DA, int NT, int B>
-int go_small(const GsParams &p, int sms, cudaStream_t st) {
-  // 16-row groups per compute warp: M <= 8 fits 16 compute warps (+ the
-  // producer) in the registers; M <= 16 uses 8 warps of 32 rows
-  constexpr int R = NT == 1 ? 1 : 2;
-  constexpr auto kern = gemv_small_kernel<DA, NT, B, R>;
-  if (set_smem_attr_once<kern>(kGsSmemBytes, true) != Q4_OK) return Q4_ERR_CUDA;
-  const int grid = (int)std::min<int64_t>(p.total_stages, (int64_t)std::min(sms, kGsMaxCtas));
-  launch_pdl(kern, dim3(grid), dim3(GsShape<R>::kThreads), kGsSmemBytes, st, p);
-  return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+int gv_tile_rows(int nt) {
+  return nt == 1 ? 16 * GvShape<1>::R * GvShape<1>::WARPS
+                 : nt == 2 ? 16 * GvShape<2>::R * GvShape<2>::WARPS : 16 * GvShape<4>::R * GvShape<4>::WARPS;
 }
-template <int DA, int NT>
-int small_bs(int bs, const GsParams &p, int sms, cudaStream_t st) {
-  switch (bs) {
-    case 32: return go_small<DA, NT, 32>(p, sms, st);
-    case 64: return go_small<DA, NT, 64>(p, sms, st);
-    case 128: return go_small<DA, NT, 128>(p, sms, st);
-    case 256: return go_small<DA, NT, 256>(p, sms, st);
-  }
-  return Q4_ERR_ARG;
-}
-template <int DA>
-int small_m(int M, int bs, const GsParams &p, int sms, cudaStream_t st) {
-  if (M <= 8) return small_bs<DA, 1>(bs, p, sms, st);
-  return small_bs<DA, 2>(bs, p, sms, st);
-}
-}  // namespace
 
-int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st) {
-  return da == Q4_F16 ? small_m<Q4_F16>(M, bs, p, sms, st) : small_m<Q4_BF16>(M, bs, p, sms, st);
+int run_gemv(int da, int mode, int nt, int bs, const GvParams &p, int grid, cudaStream_t st) {
+  if (mode != kGvAsym) return Q4_ERR_ARG;
+  return da == Q4_F16 ? run_gemv_dm<Q4_F16, kGvAsym>(nt, bs, p, grid, st)
+                      : run_gemv_dm<Q4_BF16, kGvAsym>(nt, bs, p, grid, st);
 }
 
 }  // namespace q4

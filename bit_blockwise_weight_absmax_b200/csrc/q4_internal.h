@@ -10,6 +10,7 @@
 #include "q4_common.cuh"
 #include "quantize.cuh"
 #include "dequantize.cuh"
+#include "gemv.cuh"
 #include "gemv_small.cuh"
 #include "gemm.cuh"
 
@@ -61,6 +62,10 @@ int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t 
                      float *absmax_scale, cudaStream_t st);
 int run_dequantize(int qt, int dout, int bs, bool dq, const DequantParams &p, int sms,
                    cudaStream_t st);
-int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st);
 int run_gemm(int da, const GemmParams &p, int sms, cudaStream_t st);
+int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st);
+int run_gemv(int da, int mode, int nt, int bs, const GvParams &p, int grid, cudaStream_t st);
+int gv_tile_rows(int nt);
+template <int DA, int MODE>
+int run_gemv_dm(int nt, int bs, const GvParams &p, int grid, cudaStream_t st);
 }  // namespace q4

@@ -1,6 +1,7 @@
 """A Linear4bit-style module over the C ABI: an nn.Linear whose weight is held
-as blockwise 4-bit codes (NF4 absmax with optional double quantization, or
-INT4 symmetric), and whose forward pass is the fused consumer.
+as blockwise 4-bit codes (NF4 absmax with optional double quantization, INT4
+symmetric, or INT4 asymmetric with zero-points), and whose forward pass is the
+fused consumer.
 
 learn.pranaymahendrakar.com, "Loading a model in 4-bit", "Where the accuracy
 goes": a 4-bit linear layer keeps its weight quantized and dequantizes it to
@@ -94,11 +95,9 @@ class Linear4bit(torch.nn.Module):
 
 def unsupported_reason_of(qtype: int, blocksize: int, in_features: int) -> str | None:
     """Why the fused consumers cannot run a format, or None when they can:
-    the GEMV needs whole blocks per row (in_features % blocksize == 0) and
-    does not take INT4 asymmetric states."""
-    if qtype == q4.INT4_ASYM:
-        return "INT4 asymmetric states have no fused consumer"
-    if qtype not in (q4.NF4, q4.INT4_SYM):
+    the GEMV takes NF4, INT4 symmetric and INT4 asymmetric states with whole
+    blocks per row (in_features % blocksize == 0)."""
+    if qtype not in (q4.NF4, q4.INT4_SYM, q4.INT4_ASYM):
         return f"unknown qtype {qtype}"
     if blocksize not in (32, 64, 128, 256):
         return f"blocksize {blocksize} is not 32, 64, 128 or 256"

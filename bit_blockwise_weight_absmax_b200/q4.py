@@ -72,6 +72,8 @@ def library():
                                  i32, i32, P], i32),
             "q4_device_status": ([ctypes.POINTER(i32)], i32),
             "q4_clear_device_status": ([], i32),
+            "q4_set_wait_limit_ns": ([ctypes.c_uint64], i32),
+            "q4_set_copy_stall": ([i32], i32),
             "q4_check_device": ([], i32),
             "q4_nf4_levels": ([ctypes.POINTER(ctypes.c_float)], i32),
             "q4_nf4_thresholds": ([ctypes.POINTER(ctypes.c_float)], i32),
@@ -222,6 +224,24 @@ def last_device_status() -> int:
 
 def clear_device_status():
     _check(library().q4_clear_device_status(), "q4_clear_device_status")
+
+
+def set_wait_limit_ns(ns: int):
+    """Bound (ns) of every device-side wait of later launches; 0 = default 2 s."""
+    _check(library().q4_set_wait_limit_ns(int(ns)), "q4_set_wait_limit_ns")
+
+
+def set_copy_stall(on: bool):
+    """Test hook: while on, the decode GEMV issues no weight copies, so its
+    stage waits run out after the wait limit (Q4_STATUS_TIMEOUT)."""
+    _check(library().q4_set_copy_stall(int(bool(on))), "q4_set_copy_stall")
+
+
+def reset_workspaces():
+    """Zero-fill every cached workspace again (needed after a call ended with
+    Q4_STATUS_TIMEOUT, which leaves its workspace undefined)."""
+    for t in _ws.values():
+        t.zero_()
 
 
 # -------------------------------------------------------------- workspaces --

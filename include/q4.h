@@ -206,25 +206,27 @@ Q4_API int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int6
  * q4_gemv -- Y[M, N] = A[M, K] . W^[N, K]^T for 1 <= M <= 32 ([NF4] "Why it
  * matters": memory-bound decode at small batch; [BWQ]/[BNB] dequantize to
  * the compute dtype then matmul), with the dequantization fused into the
- * streaming of the packed weights and fp32 accumulation.  The kernel takes
- * 16 activation rows at a time: 16 < M <= 32 runs it twice (rows 0..15, then
- * the rest), so the weights stream twice.
+ * streaming of the packed weights and fp32 accumulation; one pass over the
+ * weights for every M.
  *   A      device, a_dtype (Q4_F16 / Q4_BF16), [M, K] row-major, 16-byte
  *          aligned, K = Wq->cols.
- *   Wq     NF4 state (with or without double quantization) or INT4 symmetric
- *          state (the codebook is then the integers -8..7 and the group scale
- *          takes the place of c~), K % blocksize == 0, blocksize in
- *          {32, 64, 128, 256}.  INT4 asymmetric states return Q4_ERR_ARG.
+ *   Wq     NF4 state (with or without double quantization), INT4 symmetric
+ *          state (the codebook is the integers -8..7 and the group scale
+ *          takes the place of c~) or INT4 asymmetric state (codes 0..15,
+ *          w^ = (q - z) s: the kernel subtracts z times each block's
+ *          activation sum); K % blocksize == 0, blocksize in {32, 64, 128,
+ *          256}.
  *   Y      device, y_dtype (Q4_F16 / Q4_BF16 / Q4_F32), [M, N] row-major.
  *   workspace  device, q4_gemv_workspace_size() bytes, zero-filled.
  * Result: within relative Frobenius error 1e-3 of the binary64 product of A
- * and the 16-bit dequantized weights (rounded once to y_dtype).
+ * and the 16-bit dequantized weights (rounded once to y_dtype).  The
+ * summation order is fixed: identical calls give identical bits.
  */
 Q4_API int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
             int32_t y_dtype, void *workspace, size_t workspace_bytes, void *stream);
 
-/* q4_gemv over `count` (1..16) independent matrices in ONE launch per 16
- * activation rows (e.g. the seven projections of a decoder layer).  A[i], Wq[i], Y[i] are host arrays
+/* q4_gemv over `count` (1..16) independent matrices in ONE launch (e.g. the
+ * seven projections of a decoder layer); one format per call.  A[i], Wq[i], Y[i] are host arrays
  * of device pointers / host structs; M, dtypes and the rules of q4_gemv
  * apply to every entry. */
 Q4_API int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
@@ -250,6 +252,22 @@ Q4_API int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream);
 
 /* ---- status and introspection ----------------------------------------- */
+
+/* Bound, in nanoseconds, of every device-side wait (a pipeline barrier
+ * between a kernel's copy and compute warps) of the kernels launched after
+ * this call, process-wide; 0 restores the default of 2 s.  A wait that runs
+ * out raises Q4_STATUS_TIMEOUT: the kernel stops, waits for its own copies
+ * in flight and returns, leaving its outputs undefined.  After a timeout the
+ * GEMV workspace must be zero-filled again before its next use.  Host only;
+ * no device needed. */
+Q4_API int q4_set_wait_limit_ns(uint64_t ns);
+
+/* Test hook for the bounded waits, process-wide: while `on` is non-zero the
+ * decode GEMV's copy warp issues no copies, so every compute warp's wait for
+ * a weight stage runs out after the wait limit (set a short one first) and
+ * the call returns with Q4_STATUS_TIMEOUT and undefined outputs.  Leave it
+ * off otherwise.  Host only. */
+Q4_API int q4_set_copy_stall(int32_t on);
 
 /* Reads (synchronously) the sticky device status word of the current
  * device: an OR of Q4_STATUS_* bits set by kernels since the last clear. */

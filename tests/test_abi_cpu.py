@@ -154,42 +154,50 @@ def _gemv(lib, states, M):
     return lib.q4_gemv_grouped(n, ptrs, arr, ptrs, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None)
 
 
-def test_gemv_workspace_two_passes_share_the_sixteen_row_size(lib):
-    """16 < M <= 32 runs the decode kernel twice on one workspace: the size
-    for any such M is the size for 16 rows (slots of 16 columns), and M <= 8
-    needs less (slots of 8 columns)."""
+def test_gemv_workspace_sizes_per_format(lib):
+    """NF4 / INT4 symmetric: 16 < M <= 32 runs the decode kernel twice on one
+    workspace, so every such M needs the 16-row size (slots of 16 columns)
+    and M <= 8 less (8 columns).  INT4 asymmetric runs one pass for every M:
+    its slots hold 8, 16 or 32 columns.  M outside 1..32 is refused."""
     from bit_blockwise_weight_absmax_b200 import q4
-    sts = [_fake_state(0, 4096, 4096, 64, True), _fake_state(0, 11008, 4096, 64, True)]
-    arr = (ctypes.POINTER(q4._CState) * 2)(*[ctypes.pointer(s) for s in sts])
 
-    def size(M):
+    def sizes(qt, bs, dq):
+        sts = [_fake_state(qt, 4096, 4096, bs, dq), _fake_state(qt, 11008, 4096, bs, dq)]
+        arr = (ctypes.POINTER(q4._CState) * 2)(*[ctypes.pointer(s) for s in sts])
+
+        def size(M):
+            out = ctypes.c_size_t(0)
+            assert lib.q4_gemv_workspace_size(2, arr, M, ctypes.byref(out)) == 0
+            return out.value
         out = ctypes.c_size_t(0)
-        assert lib.q4_gemv_workspace_size(2, arr, M, ctypes.byref(out)) == 0
-        return out.value
-    s16 = size(16)
-    assert all(size(M) == s16 for M in (9, 17, 24, 32))
-    assert size(1) == size(8) < s16
-    out = ctypes.c_size_t(0)
-    assert lib.q4_gemv_workspace_size(2, arr, 33, ctypes.byref(out)) == -2
-    assert lib.q4_gemv_workspace_size(2, arr, 0, ctypes.byref(out)) == -2
+        assert lib.q4_gemv_workspace_size(2, arr, 33, ctypes.byref(out)) == -2
+        assert lib.q4_gemv_workspace_size(2, arr, 0, ctypes.byref(out)) == -2
+        return size
+    nf4 = sizes(0, 64, True)
+    assert nf4(1) == nf4(8) < nf4(9) == nf4(16) == nf4(17) == nf4(32)
+    asym = sizes(2, 128, False)
+    assert asym(1) == asym(8) < asym(9) == asym(16) < asym(17) == asym(32)
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_gemv_host_checks_before_the_device(lib):
     """The GEMV's format checks run on the host, matrix by matrix, before
-    any device work: INT4 asymmetric states are rejected (Q4_ERR_ARG); NF4
-    and INT4 symmetric states pass them and stop at the missing GPU; M
-    outside 1..32 is a shape error."""
+    any device work: NF4, INT4 symmetric and INT4 asymmetric states pass them
+    and stop at the missing GPU; mixed formats in one group are Q4_ERR_ARG;
+    M outside 1..32 is a shape error; K not a multiple of the blocksize is
+    a shape error."""
     nf4 = _fake_state(0, 256, 512, 64, True)
     sym = _fake_state(1, 256, 512, 128, False)
     asym = _fake_state(2, 256, 512, 128, False)
-    assert _gemv(lib, [asym], 1) == -1
-    assert _gemv(lib, [asym], 24) == -1          # the first of the two passes rejects it too
-    assert _gemv(lib, [nf4], 1) == -4            # Q4_ERR_NO_DEVICE
+    assert _gemv(lib, [asym], 1) == -4           # Q4_ERR_NO_DEVICE
+    assert _gemv(lib, [asym], 24) == -4
+    assert _gemv(lib, [nf4], 1) == -4
     assert _gemv(lib, [sym], 16) == -4
     assert _gemv(lib, [nf4], 32) == -4
+    assert _gemv(lib, [nf4, sym], 4) == -1
     assert _gemv(lib, [nf4], 33) == -2
     assert _gemv(lib, [nf4], 0) == -2
+    assert _gemv(lib, [_fake_state(0, 256, 96, 64, False)], 1) == -2
 
 
 def test_grouped_calls_reject_a_null_entry_before_any_use(lib):

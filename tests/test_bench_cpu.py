@@ -71,7 +71,7 @@ def test_reference_arm_json_line(capsys):
     import bench
 
     class A:
-        steps, warmup, copies = 1, 0, bench.N_COPIES
+        steps, warmup, copies, ref_rows = 1, 0, bench.N_COPIES, 16
     bench.run_reference(A, 0, 1)
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
@@ -84,3 +84,5 @@ def test_reference_arm_json_line(capsys):
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+    # ms_per_step is the step's measured wall time, not the whole-layer estimate
+    assert 0 < line["ms_per_step"] < line["layer_gemv_ms_estimate"]

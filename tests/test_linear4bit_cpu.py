@@ -48,13 +48,14 @@ def test_forward_without_gpu_fails_loudly():
 def test_refuses_formats_no_consumer_runs():
     """A state the GEMV/GEMM cannot consume is refused when the module is
     built, not at its first forward pass."""
-    with pytest.raises(q4.Q4Error, match="asymmetric"):
-        linear4bit.Linear4bit(_dummy_state(q4.INT4_ASYM, 128, 128))
     with pytest.raises(q4.Q4Error, match="multiple"):
         linear4bit.Linear4bit(_dummy_state(q4.NF4, 96, 64))
-    with pytest.raises(q4.Q4Error, match="asymmetric"):
-        linear4bit.Linear4bit.from_linear(torch.nn.Linear(128, 8), 128, "int4_asym")
-    linear4bit.Linear4bit(_dummy_state(q4.INT4_SYM, 128, 128))
+    with pytest.raises(q4.Q4Error, match="multiple"):
+        linear4bit.Linear4bit.from_linear(torch.nn.Linear(96, 8), 64, "nf4")
+    with pytest.raises(q4.Q4Error, match="blocksize"):
+        linear4bit.Linear4bit(_dummy_state(q4.NF4, 96, 48))
+    for qt in (q4.NF4, q4.INT4_SYM, q4.INT4_ASYM):
+        linear4bit.Linear4bit(_dummy_state(qt, 128, 128))
 
 
 def test_state_c_struct_is_cached_and_rebuilt_on_change():

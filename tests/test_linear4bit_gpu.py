@@ -20,7 +20,7 @@ def mods():
 
 
 @pytest.mark.parametrize("T", [1, 8, 32, 33, 100])
-@pytest.mark.parametrize("fmt", [("nf4", 64, True), ("int4_sym", 128, False)])
+@pytest.mark.parametrize("fmt", [("nf4", 64, True), ("int4_sym", 128, False), ("int4_asym", 128, False)])
 def test_linear4bit_forward_routes(mods, oracle, T, fmt):
     linear4bit, q4 = mods
     qtype, bs, dq = fmt
@@ -35,7 +35,7 @@ def test_linear4bit_forward_routes(mods, oracle, T, fmt):
     x = torch.randn(T, K, generator=g).bfloat16()
     y = m(x.cuda().view(1, T, K))
     assert y.shape == (1, T, N) and y.dtype == torch.bfloat16
-    ost = oracle_state(oracle, lin.weight.detach().cpu(), bs, {"nf4": 0, "int4_sym": 1}[qtype], dq)
+    ost = oracle_state(oracle, lin.weight.detach().cpu(), bs, {"nf4": 0, "int4_sym": 1, "int4_asym": 2}[qtype], dq)
     ref = oracle.gemv_reference(bits(x), True, ost, N, K)
     ref = ref + lin.bias.detach().float().cpu().double().numpy()[None, :]
     assert_matmul_close(y.view(T, N), ref)

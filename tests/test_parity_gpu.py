@@ -164,11 +164,9 @@ def test_gemv_blocksizes_dtypes(q4, oracle, bs, a_dtype):
 @pytest.mark.parametrize("M", [20, 32])
 @pytest.mark.parametrize("a_dtype,out_dtype", [(torch.bfloat16, None), (torch.float16, torch.float32),
                                                (torch.bfloat16, torch.float32)])
-def test_gemv_two_pass_grouped_dtypes(q4, oracle, M, a_dtype, out_dtype):
-    """16 < M <= 32 runs the decode kernel twice (activation rows 0..15, then
-    the rest): a grouped call over two matrices of different shapes, with
-    16-bit and fp32 outputs, so the second pass's A and Y row offsets are
-    exercised for every element size."""
+def test_gemv_large_batch_grouped_dtypes(q4, oracle, M, a_dtype, out_dtype):
+    """16 < M <= 32 in one pass (four activation tiles of 8): a grouped call
+    over two matrices of different shapes, with 16-bit and fp32 outputs."""
     g = torch.Generator().manual_seed(M)
     shapes = [(384, 1024), (272, 3072)]
     Ws = [torch.randn(N, K, generator=g).mul(0.02).bfloat16() for N, K in shapes]
@@ -180,6 +178,25 @@ def test_gemv_two_pass_grouped_dtypes(q4, oracle, M, a_dtype, out_dtype):
         ost = oracle_state(oracle, W, 64, 0, True)
         ref = oracle.gemv_reference(bits(A), a_dtype == torch.bfloat16, ost, N, K)
         assert_matmul_close(y, ref)
+
+
+@pytest.mark.parametrize("M", [1, 5, 13, 29])
+def test_gemv_ragged_group_split_tiles(q4, oracle, M):
+    """Shapes that leave partial 256-row tiles, 16-row groups cut by N, K not
+    a multiple of the 128-k chunk, and tiles split across CTAs (seven
+    matrices of different shapes in one launch)."""
+    g = torch.Generator().manual_seed(300 + M)
+    shapes = [(5, 64), (17, 192), (300, 1088), (257, 2112), (1000, 960), (16, 4096), (512, 64)]
+    Ws = [torch.randn(N, K, generator=g).mul(0.05).bfloat16() for N, K in shapes]
+    As = [torch.randn(M, K, generator=g).half() for N, K in shapes]
+    sts = [q4.quantize(dev(W), 64, "nf4", True) for W in Ws]
+    for _ in range(2):  # the second call reuses the workspace the first left
+        ys = q4.gemv_grouped([dev(A) for A in As], sts)
+        for (N, K), W, A, y in zip(shapes, Ws, As, ys):
+            ost = oracle_state(oracle, W, 64, 0, True)
+            ref = oracle.gemv_reference(bits(A), False, ost, N, K)
+            assert_matmul_close(y, ref)
+    assert q4.last_device_status() == 0
 
 
 @pytest.mark.parametrize("M", [1, 16, 24])
@@ -200,12 +217,25 @@ def test_gemv_int4_sym(q4, oracle, a_dtype, M):
     assert_matmul_close(y, ref)
 
 
-def test_gemv_rejects_int4_asym(q4):
-    """The asymmetric format's per-group zero-point has no place in the
-    decode kernel's codebook: the call fails instead of computing garbage."""
-    st = q4.quantize(dev(torch.randn(64, 128).half()), 128, "int4_asym", False)
-    with pytest.raises(q4.Q4Error):
-        q4.gemv(dev(torch.randn(1, 128).half()), st)
+@pytest.mark.parametrize("M", [1, 16, 24, 32])
+@pytest.mark.parametrize("a_dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("bs", [32, 128])
+def test_gemv_int4_asym(q4, oracle, a_dtype, M, bs):
+    """INT4 asymmetric (robotsatlas.com "INT4": [0, 15] with an integer
+    zero-point), with offset weights so the zero-points vary: the kernel's
+    s (sum a q - z sum a) against the oracle's dequantize + binary64 matmul."""
+    g = torch.Generator().manual_seed(256 + M + bs)
+    N, K = 400, 4096 + 2 * bs
+    W = (torch.randn(N, K, generator=g) * 0.02 + torch.randn(N, 1, generator=g) * 0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).to(a_dtype)
+    st = q4.quantize(dev(W), bs, "int4_asym", False)
+    ost = oracle_state(oracle, W, bs, 2, False)
+    assert_state_equal(st, ost)
+    z = np.concatenate([ost.zero & 15, ost.zero >> 4])
+    assert len(np.unique(z)) > 4
+    y = q4.gemv(dev(A), st)
+    ref = oracle.gemv_reference(bits(A), a_dtype == torch.bfloat16, ost, N, K)
+    assert_matmul_close(y, ref)
 
 
 def test_gemv_grouped_rejects_mixed_formats(q4):
@@ -304,3 +334,25 @@ def test_gemv_workspace_reuse_across_batch_sizes(q4, oracle):
         y = q4.gemv(dev(A), st)
         ref = oracle.matmul(bits(A), False, w16, False, M, len(rows), K)
         assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+
+
+def test_gemv_workspace_left_zeroed_across_shapes(q4, oracle):
+    """The partial-row slots and the counters sit at offsets that depend on
+    M and on the group, so one cached workspace serves every call only if
+    each call leaves all of it zeroed: alternate batch sizes and groups of
+    different shapes on one workspace (large M first, then small)."""
+    g = torch.Generator().manual_seed(12)
+    shapes = [(1024, 2048), (256, 4096), (2048, 1024)]
+    Ws = [torch.randn(N, K, generator=g).mul(0.02).bfloat16() for N, K in shapes]
+    sts = [q4.quantize(dev(W), 64, "nf4", True) for W in Ws]
+    osts = [oracle_state(oracle, W, 64, 0, True) for W in Ws]
+    for M, idx in [(32, [0, 1, 2]), (1, [1]), (16, [2, 0]), (8, [0]), (32, [1]), (4, [0, 1, 2]), (1, [2])]:
+        As = [torch.randn(M, shapes[i][1], generator=g).half() for i in idx]
+        ys = q4.gemv_grouped([dev(a) for a in As], [sts[i] for i in idx])
+        for i, a, y in zip(idx, As, ys):
+            N, K = shapes[i]
+            ref = oracle.gemv_reference(bits(a), False, osts[i], N, K)
+            assert_matmul_close(y, ref)
+    ws = q4._ws.get((torch.cuda.current_device(), "gemv"))
+    torch.cuda.synchronize()
+    assert ws is not None and int(ws.count_nonzero().item()) == 0

@@ -1,0 +1,47 @@
+"""Failure detection without a GPU fault: every pipeline wait in the decode
+GEMVs is bounded by the launch's wait limit.  With the copy stall test hook
+on, the copy warp issues no weight copies (a flag that nothing sets), so
+every compute warp's wait for a stage must run out after the (short) wait
+limit: the call must set Q4_STATUS_TIMEOUT and return, and after switching
+the hook off, restoring the limit and re-zeroing the workspace, the next
+call is correct."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import assert_matmul_close, bits, oracle_state
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("qtype,bs,dq,N,K", [("nf4", 64, True, 4096, 8192), ("int4_asym", 128, False, 4096, 8192)])
+def test_gemv_wait_limit_times_out_and_recovers(oracle, qtype, bs, dq, N, K):
+    """Both decode kernels (NF4 and INT4 symmetric run one, INT4 asymmetric
+    the other)."""
+    from bit_blockwise_weight_absmax_b200 import build
+    build.build()
+    from bit_blockwise_weight_absmax_b200 import q4
+    g = torch.Generator().manual_seed(5)
+    M = 4
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).half()
+    st = q4.quantize(W.cuda(), bs, qtype, dq)
+    q4.clear_device_status()
+    try:
+        q4.set_wait_limit_ns(200_000)  # 0.2 ms
+        q4.set_copy_stall(True)
+        q4.gemv(A.cuda(), st)
+        torch.cuda.synchronize()
+        assert q4.last_device_status() & 2  # Q4_STATUS_TIMEOUT
+    finally:
+        q4.set_copy_stall(False)
+        q4.set_wait_limit_ns(0)
+        q4.reset_workspaces()
+        q4.clear_device_status()
+    y = q4.gemv(A.cuda(), st)
+    rows = np.arange(0, N, 61)
+    ost = oracle_state(oracle, W, bs, {"nf4": 0, "int4_asym": 2}[qtype], dq)
+    w16 = oracle.dequantize(ost, False).reshape(N, K)[rows]
+    ref = oracle.matmul(bits(A), False, w16, False, M, len(rows), K)
+    assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+    assert q4.last_device_status() == 0
