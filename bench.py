@@ -3,11 +3,12 @@
 One step = one pass of every hot-path operation over the Llama-2-7B-shaped
 decoder layer (q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008):
   1. load-time quantize of L distinct layer copies (bf16 ~ N(0, 0.02) ->
-     NF4 blocksize 64 with double quantization of the absmax);
+     NF4 blocksize 64 with double quantization of the absmax), one grouped
+     launch per layer plus its second-level launch;
   2. fused dequant-GEMV of every layer copy at decode batch M = 1, 4, 16
      (fp16 activations ~ N(0, 1), fp32 accumulate, fp16 out), one grouped
      launch per layer;
-  3. dequantize of every layer copy to bf16;
+  3. dequantize of every layer copy to bf16, one grouped launch per layer;
   4. W4A16 tcgen05 GEMM of every layer copy at prefill M = 512 (bf16).
 The L = 4 copies (~2 GB of inputs) rotate, so every kernel reads data that
 was last touched more than the 126 MB L2 ago.  `value` is the headline
@@ -283,8 +284,7 @@ def run_gpu(args, rank, world, local_rank):
     # interval; graphs replay back to back on one stream.
     def ph_quantize():
         for l in range(L):
-            for w, st in zip(Ws[l], states[l]):
-                q4.quantize(w, 64, "nf4", True, out=st)
+            q4.quantize_grouped(Ws[l], 64, "nf4", True, outs=states[l])
 
     def ph_gemv(M):
         for l in range(L):
@@ -292,8 +292,7 @@ def run_gpu(args, rank, world, local_rank):
 
     def ph_dequantize():
         for l in range(L):
-            for st, o in zip(states[l], deq_out):
-                q4.dequantize(st, torch.bfloat16, out=o)
+            q4.dequantize_grouped(states[l], torch.bfloat16, outs=deq_out)
 
     def ph_gemm():
         for l in range(L):
@@ -305,9 +304,10 @@ def run_gpu(args, rank, world, local_rank):
     fns["dequantize"] = ph_dequantize
     fns["gemm"] = ph_gemm
     phases = list(fns)
-    launches = {"quantize": L * len(shapes) * 2, "dequantize": L * len(shapes), "gemm": L}
+    # one grouped launch per layer (quantize: plus its second-level launch)
+    launches = {"quantize": L * 2, "dequantize": L, "gemm": L}
     for M in DECODE_M:
-        launches[f"gemv_m{M}"] = L
+        launches[f"gemv_m{M}"] = L * (1 if M <= 16 else 2)
     launches_per_step = sum(launches.values())
     if args.profile:
         # a short eager run of one phase for a profiler capture (no timing)
@@ -593,7 +593,7 @@ def stack70b(steps, warmup, dev):
     """The Llama-70B-shaped stack (80 layers; shape templates, synthetic
     N(0, 0.015) bf16 weights generated per layer on the device, quantized to
     NF4 blocksize 64 with double quantization, bf16 freed): load-time
-    quantize rate (CUDA events around the quantize launches only) and the
+    quantize rate (CUDA events around each layer's grouped quantize) and the
     decode GEMV over the whole stack, one grouped launch per layer, at
     M = 1, 8, 32.  Returns a dict."""
     import torch
@@ -609,7 +609,7 @@ def stack70b(steps, warmup, dev):
               for i, (_, N, K) in enumerate(shapes)]
         e0, e1 = ev(), ev()
         e0.record()
-        sts = [q4.quantize(w, 64, "nf4", True) for w in Ws]
+        sts = q4.quantize_grouped(Ws, 64, "nf4", True)
         e1.record()
         qev.append((e0, e1))
         for st in sts:

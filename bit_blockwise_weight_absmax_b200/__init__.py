@@ -8,8 +8,8 @@ streams).  Importing this package loads nothing; the first call of an op
 loads ``libq4.so`` and fails loudly if the library or a B200 is missing.
 """
 _BINDING = {
-    "Q4State", "Q4Error", "NF4", "INT4_SYM", "INT4_ASYM", "F16", "BF16", "quantize",
-    "dequantize", "gemv", "gemv_grouped", "gemm", "gemm_grouped", "state_sizes", "nf4_levels",
+    "Q4State", "Q4Error", "NF4", "INT4_SYM", "INT4_ASYM", "F16", "BF16", "quantize", "quantize_grouped",
+    "dequantize", "dequantize_grouped", "gemv", "gemv_grouped", "gemm", "gemm_grouped", "state_sizes", "nf4_levels",
     "nf4_thresholds", "last_device_status", "clear_device_status", "library",
 }
 

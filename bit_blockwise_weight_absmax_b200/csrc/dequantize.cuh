@@ -16,6 +16,8 @@
 // next span (codes, scale codes, group scales) are loaded while the current
 // one is expanded, so two spans' loads overlap.  The 16 levels sit in shared
 // memory, one copy per lane, so a warp's 32 lookups hit 32 distinct banks.
+// A grouped launch walks the spans of several matrices (one layer) at once,
+// so the launch ramp and tail are paid once per group.
 #pragma once
 #include "q4_common.cuh"
 
@@ -53,8 +55,8 @@ struct DqRaw {
   float s[kDqChunks];      // second-level scale (double quant) or the block scale
 };
 
-template <int QT, int B, bool DQ>
-__device__ __forceinline__ void dq_load(const DequantParams &p, int64_t base, int lane, DqRaw &r) {
+template <int QT, int B, bool DQ, typename PP>
+__device__ __forceinline__ void dq_load(const PP &p, int64_t base, int lane, DqRaw &r) {
   const int64_t n = p.n;
   const uint8_t *pk_base = p.packed + base / 2 + lane * 4;  // chunk u at + 128 u
   const int64_t b_base = base / B;
@@ -83,8 +85,8 @@ __device__ __forceinline__ void dq_load(const DequantParams &p, int64_t base, in
   }
 }
 
-template <int QT, int DOUT, int B, bool DQ>
-__device__ __forceinline__ void dq_emit(const DequantParams &p, int64_t base, int lane, uint32_t lb, float mu,
+template <int QT, int DOUT, int B, bool DQ, typename PP>
+__device__ __forceinline__ void dq_emit(const PP &p, int64_t base, int lane, uint32_t lb, float mu,
                                         uint16_t *out, const DqRaw &r) {
   const int64_t n = p.n;
 #pragma unroll
@@ -155,6 +157,67 @@ __global__ void __launch_bounds__(kDqThreads, dq_ctas_per_sm<QT>()) dequantize_k
     if (sp + stride < nspan) dq_load<QT, B, DQ>(p, (sp + stride) * kDqSpan, lane, nxt);
     dq_emit<QT, DOUT, B, DQ>(p, sp * kDqSpan, lane, lb, mu, out, cur);
     cur = nxt;
+  }
+}
+
+// One matrix of a grouped dequantize.
+struct DqGMat {
+  const uint8_t *packed;
+  const float *absmax;
+  const uint8_t *zero;
+  const int8_t *absmax_q;
+  const float *absmax_scale;
+  const float *absmax_mean;
+  int64_t n;
+  void *out;
+  int64_t span_begin;  // first global span of this matrix
+};
+constexpr int kDqMaxGroup = 16;
+struct DequantGroupParams {
+  DqGMat mat[kDqMaxGroup];
+  int32_t count;
+  int64_t total_spans;
+  float levels[16];
+};
+
+// Every matrix of a group in one launch: the warps walk the spans of all
+// matrices with a grid stride (the next span's loads, in whichever matrix it
+// lies, are in flight while the current one is expanded).
+template <int QT, int DOUT, int B, bool DQ>
+__global__ void __launch_bounds__(kDqThreads, dq_ctas_per_sm<QT>())
+    dequantize_grouped_kernel(const __grid_constant__ DequantGroupParams p) {
+  pdl_launch_then_wait();
+  static_assert(B % 8 == 0, "a chunk never straddles two blocks");
+  __shared__ float s_lv[16 * 32];  // [level][lane]
+  const int lane = threadIdx.x & 31;
+  if (QT == Q4_NF4) {
+    for (int i = threadIdx.x; i < 16 * 32; i += blockDim.x) s_lv[i] = p.levels[i >> 5];
+    __syncthreads();
+  }
+  const uint32_t lb = (uint32_t)__cvta_generic_to_shared(s_lv) + 4u * (uint32_t)lane;
+  const int wpb = blockDim.x >> 5;
+  const int64_t stride = (int64_t)gridDim.x * wpb;
+  int64_t sp = (int64_t)blockIdx.x * wpb + (threadIdx.x >> 5);
+  if (sp >= p.total_spans) return;
+  int mi = 0;
+  while (mi + 1 < p.count && sp >= p.mat[mi + 1].span_begin) ++mi;
+  DqRaw cur;
+  dq_load<QT, B, DQ>(p.mat[mi], (sp - p.mat[mi].span_begin) * kDqSpan, lane, cur);
+  while (sp < p.total_spans) {
+    const int64_t nsp = sp + stride;
+    int nmi = mi;
+    DqRaw nxt;
+    if (nsp < p.total_spans) {
+      while (nmi + 1 < p.count && nsp >= p.mat[nmi + 1].span_begin) ++nmi;
+      dq_load<QT, B, DQ>(p.mat[nmi], (nsp - p.mat[nmi].span_begin) * kDqSpan, lane, nxt);
+    }
+    const DqGMat &m = p.mat[mi];
+    const float mu = DQ ? __ldg(m.absmax_mean) : 0.0f;
+    dq_emit<QT, DOUT, B, DQ>(m, (sp - m.span_begin) * kDqSpan, lane, lb, mu, reinterpret_cast<uint16_t *>(m.out),
+                             cur);
+    cur = nxt;
+    sp = nsp;
+    mi = nmi;
   }
 }
 

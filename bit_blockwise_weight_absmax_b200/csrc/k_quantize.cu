@@ -3,33 +3,43 @@
 
 namespace q4 {
 namespace {
-template <int DT, int QT, int B, bool DQ>
-void go(const QuantParams &p, int grid, cudaStream_t st) {
-  launch_pdl(quantize_kernel<DT, QT, B, DQ>, dim3(grid), dim3(kQThreads), 0, st, p);
+template <int DT, int QT, int B, bool DQ, bool GROUPED, typename P>
+void go(const P &p, int grid, cudaStream_t st) {
+  launch_pdl(quantize_kernel<DT, QT, B, DQ, GROUPED>, dim3(grid), dim3(kQThreads), 0, st, p);
 }
-template <int DT, int QT, bool DQ>
-int by_bs(int bs, const QuantParams &p, int grid, cudaStream_t st) {
+template <int DT, int QT, bool DQ, bool GROUPED, typename P>
+int by_bs(int bs, const P &p, int grid, cudaStream_t st) {
   switch (bs) {
-    case 32: go<DT, QT, 32, DQ>(p, grid, st); return 0;
-    case 64: go<DT, QT, 64, DQ>(p, grid, st); return 0;
-    case 128: go<DT, QT, 128, DQ>(p, grid, st); return 0;
-    case 256: go<DT, QT, 256, DQ>(p, grid, st); return 0;
+    case 32: go<DT, QT, 32, DQ, GROUPED>(p, grid, st); return 0;
+    case 64: go<DT, QT, 64, DQ, GROUPED>(p, grid, st); return 0;
+    case 128: go<DT, QT, 128, DQ, GROUPED>(p, grid, st); return 0;
+    case 256: go<DT, QT, 256, DQ, GROUPED>(p, grid, st); return 0;
   }
   return Q4_ERR_ARG;
 }
-template <int DT>
-int by_qt(int qt, int bs, bool dq, const QuantParams &p, int grid, cudaStream_t st) {
-  if (qt == Q4_NF4) return dq ? by_bs<DT, Q4_NF4, true>(bs, p, grid, st) : by_bs<DT, Q4_NF4, false>(bs, p, grid, st);
-  if (qt == Q4_INT4_SYM) return by_bs<DT, Q4_INT4_SYM, false>(bs, p, grid, st);
-  return by_bs<DT, Q4_INT4_ASYM, false>(bs, p, grid, st);
+template <int DT, bool GROUPED, typename P>
+int by_qt(int qt, int bs, bool dq, const P &p, int grid, cudaStream_t st) {
+  if (qt == Q4_NF4)
+    return dq ? by_bs<DT, Q4_NF4, true, GROUPED>(bs, p, grid, st) : by_bs<DT, Q4_NF4, false, GROUPED>(bs, p, grid, st);
+  if (qt == Q4_INT4_SYM) return by_bs<DT, Q4_INT4_SYM, false, GROUPED>(bs, p, grid, st);
+  return by_bs<DT, Q4_INT4_ASYM, false, GROUPED>(bs, p, grid, st);
+}
+template <bool GROUPED, typename P>
+int dispatch(int dt, int qt, int bs, bool dq, const P &p, int grid, cudaStream_t st) {
+  if (dq && qt != Q4_NF4) return Q4_ERR_ARG;
+  const int rc = dt == Q4_F16 ? by_qt<Q4_F16, GROUPED>(qt, bs, dq, p, grid, st)
+                              : by_qt<Q4_BF16, GROUPED>(qt, bs, dq, p, grid, st);
+  if (rc) return rc;
+  return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 }  // namespace
 
 int run_quantize(int dt, int qt, int bs, bool dq, const QuantParams &p, int grid, cudaStream_t st) {
-  if (dq && qt != Q4_NF4) return Q4_ERR_ARG;
-  int rc = dt == Q4_F16 ? by_qt<Q4_F16>(qt, bs, dq, p, grid, st) : by_qt<Q4_BF16>(qt, bs, dq, p, grid, st);
-  if (rc) return rc;
-  return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+  return dispatch<false>(dt, qt, bs, dq, p, grid, st);
+}
+
+int run_quantize_grouped(int dt, int qt, int bs, bool dq, const QuantGroupParams &p, int grid, cudaStream_t st) {
+  return dispatch<true>(dt, qt, bs, dq, p, grid, st);
 }
 
 int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t *absmax_q,
@@ -37,6 +47,11 @@ int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t 
   const int64_t ng = (nb + Q4_DQ_GROUP - 1) / Q4_DQ_GROUP;
   launch_pdl(double_quant_kernel, dim3((unsigned)((ng + 7) / 8)), dim3(256), 0, st, absmax, nb, mean, absmax_q,
              absmax_scale);
+  return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
+}
+
+int run_double_quant_grouped(const DqGroupParams &p, cudaStream_t st) {
+  launch_pdl(double_quant_grouped_kernel, dim3((unsigned)((p.total_groups + 7) / 8)), dim3(256), 0, st, p);
   return cudaGetLastError() == cudaSuccess ? Q4_OK : Q4_ERR_CUDA;
 }
 }  // namespace q4

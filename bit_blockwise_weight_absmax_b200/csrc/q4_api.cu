@@ -491,6 +491,105 @@ int q4_quantize(const void *W, int32_t w_dtype, int64_t rows, int64_t cols, int3
   return rc;
 }
 
+int q4_quantize_grouped_workspace_size(int32_t count, const int64_t *rows, const int64_t *cols,
+                                       int32_t blocksize, int32_t qtype, int32_t double_quant, size_t *bytes) {
+  if (!bytes || !rows || !cols || count < 1 || count > kQMaxGroup) return Q4_ERR_ARG;
+  size_t total = 256;  // one arrival counter per matrix
+  for (int i = 0; i < count; ++i) {
+    if (rows[i] < 1 || cols[i] < 1) return Q4_ERR_SHAPE;
+    size_t sz[6];
+    const int rc = q4_state_sizes(qtype, rows[i] * cols[i], blocksize, double_quant, sz);
+    if (rc != Q4_OK) return rc;
+    const int64_t nb = ceil_div(rows[i] * cols[i], blocksize);
+    if (double_quant) total += align256((size_t)ceil_div(nb, kChunkBlocks) * 8);
+  }
+  *bytes = double_quant ? total : 0;
+  return Q4_OK;
+}
+
+int q4_quantize_grouped(int32_t count, const void *const *W, int32_t w_dtype, const int64_t *rows,
+                        const int64_t *cols, int32_t blocksize, int32_t qtype, int32_t double_quant,
+                        q4_state *const *out, void *workspace, size_t workspace_bytes, void *stream) {
+  if (count < 1 || count > kQMaxGroup || !W || !rows || !cols || !out || !valid_in_dtype(w_dtype)) return Q4_ERR_ARG;
+  for (int i = 0; i < count; ++i)
+    if (!W[i] || !out[i]) return Q4_ERR_ARG;
+  size_t need = 0;
+  int rc = q4_quantize_grouped_workspace_size(count, rows, cols, blocksize, qtype, double_quant, &need);
+  if (rc != Q4_OK) return rc;
+  for (int i = 0; i < count; ++i) {
+    q4_state *o = out[i];
+    if (!o->packed || !o->absmax || (qtype == Q4_INT4_ASYM && !o->zero)) return Q4_ERR_ARG;
+    if (double_quant && (!o->absmax_q || !o->absmax_scale || !o->absmax_mean)) return Q4_ERR_ARG;
+    if (!aligned16(W[i]) || !aligned16(o->packed) || ((uintptr_t)o->absmax & 3u)) return Q4_ERR_ALIGN;
+  }
+  if (need && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+  static Nf4BinTable tab;
+  static bool tab_ok = false;
+  static std::once_flag once;
+  std::call_once(once, [] { tab_ok = build_bin_table(&tab); });
+  if (!tab_ok) return Q4_ERR_ARG;
+
+  static thread_local QuantGroupParams p;
+  static thread_local DqGroupParams dp;
+  memset(&p, 0, sizeof(p));
+  memset(&dp, 0, sizeof(dp));
+  int64_t chunks = 0, groups = 0;
+  size_t ws_off = 256;
+  for (int i = 0; i < count; ++i) {
+    q4_state *o = out[i];
+    const int64_t n = rows[i] * cols[i];
+    const int64_t nb = ceil_div(n, blocksize);
+    o->qtype = qtype;
+    o->src_dtype = w_dtype;
+    o->n = n;
+    o->rows = rows[i];
+    o->cols = cols[i];
+    o->blocksize = blocksize;
+    o->double_quant = double_quant;
+    o->dq_group = Q4_DQ_GROUP;
+    o->reserved = 0;
+    if (!double_quant) o->absmax_q = nullptr, o->absmax_scale = nullptr, o->absmax_mean = nullptr;
+    if (qtype != Q4_INT4_ASYM) o->zero = nullptr;
+    QMat &m = p.mat[i];
+    m.W = reinterpret_cast<const uint16_t *>(W[i]);
+    m.n = n;
+    m.nb = nb;
+    m.n_chunks = ceil_div(nb, kChunkBlocks);
+    m.chunk_begin = chunks;
+    m.packed = o->packed;
+    m.absmax = o->absmax;
+    m.zero = o->zero;
+    if (double_quant) {
+      m.absmax_mean = o->absmax_mean;
+      m.counter = reinterpret_cast<unsigned *>((char *)workspace + 4 * i);
+      m.partials = reinterpret_cast<double *>((char *)workspace + ws_off);
+      ws_off += align256((size_t)m.n_chunks * 8);
+      DqMat &d = dp.mat[i];
+      d.absmax = o->absmax;
+      d.nb = nb;
+      d.mean = o->absmax_mean;
+      d.absmax_q = o->absmax_q;
+      d.absmax_scale = o->absmax_scale;
+      d.group_begin = groups;
+      groups += ceil_div(nb, Q4_DQ_GROUP);
+    }
+    chunks += m.n_chunks;
+  }
+  p.count = count;
+  p.total_chunks = chunks;
+  p.status = di.status;
+  p.tab = tab;
+  dp.count = count;
+  dp.total_groups = groups;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(chunks, (int64_t)di.sms * 4));
+  rc = run_quantize_grouped(w_dtype, qtype, blocksize, double_quant != 0, p, grid, st);
+  if (rc == Q4_OK && double_quant) rc = run_double_quant_grouped(dp, st);
+  return rc;
+}
+
 int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream) {
   int rc = check_state(Wq);
   if (rc != Q4_OK) return rc;
@@ -510,6 +609,44 @@ int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream
   memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
   return run_dequantize(Wq->qtype, out_dtype, Wq->blocksize, Wq->double_quant != 0, p, di.sms,
                         (cudaStream_t)stream);
+}
+
+int q4_dequantize_grouped(int32_t count, const q4_state *const *Wq, void *const *out, int32_t out_dtype,
+                          void *stream) {
+  if (count < 1 || count > kDqMaxGroup || !Wq || !out || !valid_in_dtype(out_dtype)) return Q4_ERR_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (!Wq[i] || !out[i]) return Q4_ERR_ARG;
+    const int rc = check_state(Wq[i]);
+    if (rc != Q4_OK) return rc;
+    if (Wq[i]->qtype != Wq[0]->qtype || Wq[i]->blocksize != Wq[0]->blocksize ||
+        Wq[i]->double_quant != Wq[0]->double_quant)
+      return Q4_ERR_ARG;  // one format per grouped call
+    if (!aligned16(out[i])) return Q4_ERR_ALIGN;
+  }
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+  static thread_local DequantGroupParams p;
+  memset(&p, 0, sizeof(p));
+  int64_t spans = 0;
+  for (int i = 0; i < count; ++i) {
+    const q4_state *s = Wq[i];
+    DqGMat &m = p.mat[i];
+    m.packed = s->packed;
+    m.absmax = s->absmax;
+    m.zero = s->zero;
+    m.absmax_q = s->absmax_q;
+    m.absmax_scale = s->absmax_scale;
+    m.absmax_mean = s->absmax_mean;
+    m.n = s->n;
+    m.out = out[i];
+    m.span_begin = spans;
+    spans += ceil_div(s->n, kDqSpan);
+  }
+  p.count = count;
+  p.total_spans = spans;
+  memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+  return run_dequantize_grouped(Wq[0]->qtype, out_dtype, Wq[0]->blocksize, Wq[0]->double_quant != 0, p, di.sms,
+                                (cudaStream_t)stream);
 }
 
 int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {

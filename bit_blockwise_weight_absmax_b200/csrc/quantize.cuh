@@ -11,7 +11,7 @@
 // with an integer zero-point) share the kernel.  Double quantization of the
 // absmax ("blocks of 256, to 8 bits") is a second kernel.
 //
-// Design: one streaming pass over W.  A thread owns 8 consecutive elements
+// Design: one streaming pass over W.  A thread owns 16 consecutive elements
 // (one 128-bit load); B/8 adjacent lanes own one block and reduce its absmax
 // with xor shuffles.  A CTA (256 threads) walks 256-block chunks (the
 // double-quant groups); each CTA owns a contiguous, power-of-two-aligned run
@@ -19,7 +19,11 @@
 // the double-quant mean is formed in the exact order of the definition (an
 // aligned binary tree) without atomics: lanes -> chunk (shared memory tree)
 // -> CTA run (streaming pairwise stack) -> the last CTA to finish combines the
-// per-CTA partial sums and writes the mean.
+// per-CTA partial sums and writes the mean.  A grouped launch quantizes every
+// matrix of a layer at once: CTAs walk all matrices' chunks with a grid
+// stride, each chunk's sum goes to the workspace, and the CTA that counts a
+// matrix's last chunk combines them in the same tree order; one second
+// launch quantizes every matrix's groups of absmax values.
 #pragma once
 #include <type_traits>
 
@@ -59,6 +63,29 @@ struct QuantParams {
   Nf4BinTable tab;
 };
 
+// One matrix of a grouped launch.
+struct QMat {
+  const uint16_t *W;
+  int64_t n, nb;
+  int64_t n_chunks;
+  int64_t chunk_begin;  // first global chunk of this matrix
+  uint8_t *packed;
+  float *absmax;
+  uint8_t *zero;
+  float *absmax_mean;   // double quant
+  double *partials;     // [n_chunks] fp64 pairwise sums of the chunks (double quant)
+  unsigned *counter;    // chunks done (double quant), left at 0
+};
+constexpr int kQMaxGroup = 16;
+
+struct QuantGroupParams {
+  QMat mat[kQMaxGroup];
+  int32_t count;
+  int64_t total_chunks;
+  int *status;
+  Nf4BinTable tab;
+};
+
 // Absolute value of eight 16-bit floats as a max over (bits & 0x7fff): the
 // order of magnitudes of IEEE 16-bit floats is the integer order of these
 // patterns, and NaN / Inf sort above every finite value.
@@ -81,11 +108,41 @@ __device__ __forceinline__ uint32_t nf4_code_fast(float x, uint32_t tb) {
   return (uint32_t)(base + (x >= thr ? 1 : 0));
 }
 
+// The pairwise fp64 sum of len <= kMaxRunPartials values at src (level by
+// level, adjacent pairs, an odd last value carried up), staged in shared
+// memory by the whole CTA (every thread must call it).  Returns the sum in
+// every thread.
+__device__ __forceinline__ double tree_sum_smem(const double *src, int len, double *s_red, int tid) {
+  for (int i = tid; i < len; i += kQThreads) s_red[i] = __ldcg(src + i);
+  __syncthreads();
+  while (len > 1) {
+    const int half = len >> 1;
+    double t[kMaxRunPartials / kQThreads / 2 + 1];
+    int cnt = 0;
+    for (int i = tid; i < half; i += kQThreads) t[cnt++] = s_red[2 * i] + s_red[2 * i + 1];
+    const double carry = s_red[len - 1];
+    __syncthreads();
+    cnt = 0;
+    for (int i = tid; i < half; i += kQThreads) s_red[i] = t[cnt++];
+    if ((len & 1) && tid == 0) s_red[half] = carry;
+    __syncthreads();
+    len = half + (len & 1);
+  }
+  const double r = s_red[0];
+  __syncthreads();
+  return r;
+}
+
 // Four resident CTAs of 256 threads per SM (at most 64 registers): more
 // warps to hide the division and table latencies, with four 16-byte loads
 // in flight per thread.
-template <int DT, int QT, int B, bool DQ>
-__global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
+// GROUPED: one launch over the matrices of a QuantGroupParams; every CTA
+// walks the global chunks with a grid stride, each chunk's fp64 sum goes to
+// the matrix's partials and the CTA that counts a matrix's last chunk sums
+// them.  Otherwise one matrix; each CTA owns one run of chunks.
+template <int DT, int QT, int B, bool DQ, bool GROUPED = false>
+__global__ void __launch_bounds__(kQThreads, 4)
+    quantize_kernel(const __grid_constant__ std::conditional_t<GROUPED, QuantGroupParams, QuantParams> p) {
   pdl_launch_then_wait();
   constexpr int E = 16;                          // consecutive elements per thread (one block)
   constexpr int V = E / 8;                       // 16-byte words per thread
@@ -102,6 +159,7 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
   __shared__ double s_blk[2][kChunkBlocks];      // block absmax of a chunk, by chunk parity
   __shared__ uint8_t s_zero[BLK_IT];             // INT4_ASYM zero-points of one iteration
   __shared__ double s_stack[24];                 // streaming pairwise stack (thread 0)
+  __shared__ double s_red_all[GROUPED && DQ ? kMaxRunPartials : 1];  // a matrix's chunk sums (grouped)
   __shared__ int s_last;
 
   const int tid = threadIdx.x;
@@ -119,8 +177,6 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
   int nonfinite = 0;
   int depth = 0;  // stack depth (thread 0)
   int cpar = 0;   // parity of s_blk for the current chunk
-  const int64_t c0 = (int64_t)blockIdx.x * p.run;
-  const int64_t c1 = min(c0 + p.run, p.n_chunks);
 
   // Codes of the thread's E elements (element 8k + j in bits 4j..4j+3 of
   // codes[k]) and the block's scale; lanes of one block agree on `scale`
@@ -229,14 +285,18 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
     }
   };
 
-  for (int64_t chunk = c0; chunk < c1; ++chunk) {
+  // One chunk (256 blocks) of a matrix; with double quantization returns the
+  // fp64 pairwise sum of its block absmax values (valid in thread 0).
+  auto do_chunk = [&](const uint16_t *W, int64_t n, int64_t nb, uint8_t *packed, float *absmax, uint8_t *zero,
+                      int64_t chunk) -> double {
+    double chunk_sum = 0.0;
     const int64_t chunk_e0 = chunk * CHUNK_ELEMS;
     const int64_t chunk_b0 = chunk * kChunkBlocks;
     // FULL: the whole chunk lies inside the tensor (every chunk but the last)
     auto run_chunk = [&](auto full_tag) {
       constexpr bool FULL = decltype(full_tag)::value;
-      const uint16_t *wp = p.W + chunk_e0 + tid * E;
-      uint8_t *pp = p.packed + chunk_e0 / 2 + tid * (E / 2);
+      const uint16_t *wp = W + chunk_e0 + tid * E;
+      uint8_t *pp = packed + chunk_e0 / 2 + tid * (E / 2);
       for (int it0 = 0; it0 < IT_PER_CHUNK; it0 += BATCH) {
         uint4 v[BATCH][V];
 #pragma unroll
@@ -248,12 +308,12 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
               v[b][k] = ldg_stream_v4(wp + off + 8 * k);
             } else {
               const int64_t e0 = chunk_e0 + off + tid * E + 8 * k;
-              if (e0 + 8 <= p.n) {
+              if (e0 + 8 <= n) {
                 v[b][k] = ldg_stream_v4(wp + off + 8 * k);
               } else {
                 uint16_t t[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) t[j] = (e0 + j < p.n) ? p.W[e0 + j] : (uint16_t)0;
+                for (int j = 0; j < 8; ++j) t[j] = (e0 + j < n) ? W[e0 + j] : (uint16_t)0;
                 v[b][k] = make_uint4(t[0] | (t[1] << 16), t[2] | (t[3] << 16), t[4] | (t[5] << 16),
                                      t[6] | (t[7] << 16));
               }
@@ -272,10 +332,10 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
           if (QT == Q4_INT4_ASYM && (tid % LPB) == 0) s_zero[(tid * E) / B] = (uint8_t)z;
           // ---- stores
           const int64_t e0 = chunk_e0 + off + tid * E;
-          if (FULL || e0 + E <= p.n) {
+          if (FULL || e0 + E <= n) {
             *reinterpret_cast<uint2 *>(pp + off / 2) = make_uint2(codes[0], codes[1]);
-          } else if (e0 < p.n) {
-            const int valid = (int)(p.n - e0);
+          } else if (e0 < n) {
+            const int valid = (int)(n - e0);
 #pragma unroll
             for (int j = 0; j < E / 2; ++j) {
               if (2 * j < valid) {
@@ -286,22 +346,22 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
             }
           }
           if ((tid % LPB) == 0) {
-            const bool in = FULL || chunk_b0 + bl < p.nb;
-            if (in) p.absmax[chunk_b0 + bl] = scale;
+            const bool in = FULL || chunk_b0 + bl < nb;
+            if (in) absmax[chunk_b0 + bl] = scale;
             if (DQ) s_blk[cpar][bl] = in ? (double)scale : 0.0;
           }
           if (QT == Q4_INT4_ASYM) {
             __syncthreads();
             if (tid < BLK_IT / 2) {
               const int64_t b0 = chunk_b0 + it * BLK_IT + 2 * tid;
-              if (b0 < p.nb) p.zero[b0 / 2] = (uint8_t)(s_zero[2 * tid] | (s_zero[2 * tid + 1] << 4));
+              if (b0 < nb) zero[b0 / 2] = (uint8_t)(s_zero[2 * tid] | (s_zero[2 * tid + 1] << 4));
             }
             __syncthreads();
           }
         }
       }
     };
-    if (chunk_e0 + CHUNK_ELEMS <= p.n) run_chunk(std::true_type{});
+    if (chunk_e0 + CHUNK_ELEMS <= n) run_chunk(std::true_type{});
     else run_chunk(std::false_type{});
     if (DQ) {
       // Pairwise fp64 sum of the chunk's 256 block values in tree order:
@@ -317,20 +377,81 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
         if (tid == 0) {
           // streaming pairwise stack over the CTA's run of chunks: merging
           // equal-size neighbours reproduces the aligned binary tree
-          s_stack[depth++] = s;
-          for (int64_t k = chunk - c0 + 1; (k & 1) == 0; k >>= 1) {
-            s_stack[depth - 2] = s_stack[depth - 2] + s_stack[depth - 1];
-            --depth;
-          }
+          chunk_sum = s;
         }
       }
       cpar ^= 1;
+    }
+    return chunk_sum;
+  };
+
+  if constexpr (!GROUPED) {
+    const int64_t c0 = (int64_t)blockIdx.x * p.run;
+    const int64_t c1 = min(c0 + p.run, p.n_chunks);
+    for (int64_t chunk = c0; chunk < c1; ++chunk) {
+      const double cs = do_chunk(p.W, p.n, p.nb, p.packed, p.absmax, p.zero, chunk);
+      if (DQ && tid == 0) {
+        // streaming pairwise stack over the CTA's run of chunks: merging
+        // equal-size neighbours reproduces the aligned binary tree
+        s_stack[depth++] = cs;
+        for (int64_t k = chunk - c0 + 1; (k & 1) == 0; k >>= 1) {
+          s_stack[depth - 2] = s_stack[depth - 2] + s_stack[depth - 1];
+          --depth;
+        }
+      }
+    }
+  } else {
+    int mi = 0;
+    for (int64_t gc = blockIdx.x; gc < p.total_chunks; gc += gridDim.x) {
+      while (mi + 1 < p.count && gc >= p.mat[mi + 1].chunk_begin) ++mi;
+      const QMat &m = p.mat[mi];
+      const int64_t chunk = gc - m.chunk_begin;
+      const double cs = do_chunk(m.W, m.n, m.nb, m.packed, m.absmax, m.zero, chunk);
+      if constexpr (DQ) {
+        if (tid == 0) {
+          m.partials[chunk] = cs;
+          __threadfence();
+          s_last = atomicAdd(m.counter, 1u) == (unsigned)(m.n_chunks - 1);
+        }
+        __syncthreads();
+        if (s_last) {
+          // this CTA counted the matrix's last chunk: the pairwise tree over
+          // its chunk sums, as aligned subtrees of kMaxRunPartials values
+          // (each reduced level by level, odd last carried up) and then the
+          // tree over the subtree sums -- the same order as one tree
+          __threadfence();
+          double sub[32];
+          int nsub = 0;
+          for (int64_t b0 = 0; b0 < m.n_chunks; b0 += kMaxRunPartials) {
+            const int len = (int)min((int64_t)kMaxRunPartials, m.n_chunks - b0);
+            const double t = tree_sum_smem(m.partials + b0, len, s_red_all, tid);
+            if (nsub < 32) sub[nsub] = t;
+            ++nsub;
+          }
+          // the workspace is left zeroed
+          for (int64_t i = tid; i < m.n_chunks; i += kQThreads) __stcg(m.partials + i, 0.0);
+          if (tid == 0) {
+            int len = nsub;
+            while (len > 1) {
+              const int half = len >> 1;
+              for (int i = 0; i < half; ++i) sub[i] = sub[2 * i] + sub[2 * i + 1];
+              if (len & 1) sub[half] = sub[len - 1];
+              len = half + (len & 1);
+            }
+            m.absmax_mean[0] = __double2float_rn(__ddiv_rn(sub[0], (double)m.nb));
+            *m.counter = 0u;  // leave the workspace zeroed for the next call
+          }
+          __syncthreads();
+        }
+      }
     }
   }
 
   if (nonfinite) raise_status(p.status, Q4_STATUS_NONFINITE);
 
-  if (DQ) {
+  if constexpr (DQ && !GROUPED) {
+    const int64_t c0 = (int64_t)blockIdx.x * p.run;
+    const int64_t c1 = min(c0 + p.run, p.n_chunks);
     if (tid == 0) {
       // pad the run with zero chunks up to its power-of-two length
       for (int64_t k = c1 - c0; k < p.run; ++k) {
@@ -352,7 +473,10 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
       __threadfence();
       __shared__ double s_red[kMaxRunPartials];
       int len = gridDim.x;
-      for (int i = tid; i < len; i += kQThreads) s_red[i] = __ldcg(p.partials + i);
+      for (int i = tid; i < len; i += kQThreads) {
+        s_red[i] = __ldcg(p.partials + i);
+        __stcg(p.partials + i, 0.0);  // the workspace is left zeroed
+      }
       __syncthreads();
       while (len > 1) {
         const int half = len >> 1;
@@ -376,19 +500,26 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(QuantParams p) {
   }
 }
 
-// Second-level quantization of the block absmax, one warp per group of 256:
+// One matrix's double-quant state for the grouped second-level kernel.
+struct DqMat {
+  const float *absmax;
+  int64_t nb;
+  const float *mean;
+  int8_t *absmax_q;
+  float *absmax_scale;
+  int64_t group_begin;  // first global group of this matrix
+};
+struct DqGroupParams {
+  DqMat mat[kQMaxGroup];
+  int32_t count;
+  int64_t total_groups;
+};
+
+// One group of 256 block absmax values, by one warp:
 // m2 = max|c - mu|, s2 = m2 / 127, q2 = clamp(rint((c - mu) / s2), -128, 127).
-static __global__ void __launch_bounds__(256) double_quant_kernel(const float *__restrict__ absmax,
-                                                           int64_t nb,
-                                                           const float *__restrict__ mean,
-                                                           int8_t *__restrict__ absmax_q,
-                                                           float *__restrict__ absmax_scale) {
-  pdl_launch_then_wait();
-  const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int64_t ng = (nb + Q4_DQ_GROUP - 1) / Q4_DQ_GROUP;
-  if (g >= ng) return;
-  const float mu = __ldg(mean);
+__device__ __forceinline__ void double_quant_group(const float *__restrict__ absmax, int64_t nb, float mu,
+                                                   int8_t *__restrict__ absmax_q, float *__restrict__ absmax_scale,
+                                                   int64_t g, int lane) {
   float d[8];
   float m2 = 0.0f;
 #pragma unroll
@@ -410,6 +541,32 @@ static __global__ void __launch_bounds__(256) double_quant_kernel(const float *_
       absmax_q[b] = (int8_t)q2;
     }
   }
+}
+
+// The groups of every matrix of a grouped quantize, one warp per group.
+static __global__ void __launch_bounds__(256) double_quant_grouped_kernel(const __grid_constant__ DqGroupParams p) {
+  pdl_launch_then_wait();
+  const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (g >= p.total_groups) return;
+  int mi = 0;
+  while (mi + 1 < p.count && g >= p.mat[mi + 1].group_begin) ++mi;
+  const DqMat &m = p.mat[mi];
+  double_quant_group(m.absmax, m.nb, __ldg(m.mean), m.absmax_q, m.absmax_scale, g - m.group_begin,
+                     threadIdx.x & 31);
+}
+
+// Second-level quantization of the block absmax, one warp per group of 256:
+// m2 = max|c - mu|, s2 = m2 / 127, q2 = clamp(rint((c - mu) / s2), -128, 127).
+static __global__ void __launch_bounds__(256) double_quant_kernel(const float *__restrict__ absmax,
+                                                           int64_t nb,
+                                                           const float *__restrict__ mean,
+                                                           int8_t *__restrict__ absmax_q,
+                                                           float *__restrict__ absmax_scale) {
+  pdl_launch_then_wait();
+  const int64_t g = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int64_t ng = (nb + Q4_DQ_GROUP - 1) / Q4_DQ_GROUP;
+  if (g >= ng) return;
+  double_quant_group(absmax, nb, __ldg(mean), absmax_q, absmax_scale, g, threadIdx.x & 31);
 }
 
 }  // namespace q4

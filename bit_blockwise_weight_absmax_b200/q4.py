@@ -62,7 +62,12 @@ def library():
             "q4_state_sizes": ([i32, i64, i32, i32, ctypes.POINTER(sz)], i32),
             "q4_quantize_workspace_size": ([i32, i64, i32, i32, ctypes.POINTER(sz)], i32),
             "q4_quantize": ([P, i32, i64, i64, i32, i32, i32, SP, P, sz, P], i32),
+            "q4_quantize_grouped_workspace_size": ([i32, ctypes.POINTER(i64), ctypes.POINTER(i64), i32, i32, i32,
+                                                    ctypes.POINTER(sz)], i32),
+            "q4_quantize_grouped": ([i32, ctypes.POINTER(P), i32, ctypes.POINTER(i64), ctypes.POINTER(i64), i32, i32,
+                                     i32, ctypes.POINTER(SP), P, sz, P], i32),
             "q4_dequantize": ([SP, P, i32, P], i32),
+            "q4_dequantize_grouped": ([i32, ctypes.POINTER(SP), ctypes.POINTER(P), i32, P], i32),
             "q4_gemv_workspace_size": ([i32, ctypes.POINTER(SP), i64, ctypes.POINTER(sz)], i32),
             "q4_gemv": ([P, i32, i64, SP, P, i32, P, sz, P], i32),
             "q4_gemv_grouped": ([i32, ctypes.POINTER(P), ctypes.POINTER(SP), ctypes.POINTER(P), i64,
@@ -304,6 +309,55 @@ def quantize(W: torch.Tensor, blocksize: int = 64, qtype="nf4", double_quant: bo
     return st
 
 
+def _new_state(qt, dtype, rows, cols, blocksize, double_quant, dev) -> Q4State:
+    sz = state_sizes(qt, rows * cols, blocksize, double_quant)
+    return Q4State(qt, dtype, rows, cols, blocksize, bool(double_quant),
+                   packed=torch.empty(sz[0], dtype=torch.uint8, device=dev),
+                   absmax=torch.empty(sz[1] // 4, dtype=torch.float32, device=dev),
+                   zero=torch.empty(sz[2], dtype=torch.uint8, device=dev) if sz[2] else None,
+                   absmax_q=torch.empty(sz[3], dtype=torch.int8, device=dev) if sz[3] else None,
+                   absmax_scale=torch.empty(sz[4] // 4, dtype=torch.float32, device=dev) if sz[4] else None,
+                   absmax_mean=torch.empty(1, dtype=torch.float32, device=dev) if sz[5] else None)
+
+
+def quantize_grouped(Ws, blocksize: int = 64, qtype="nf4", double_quant: bool = False, stream=None,
+                     outs=None) -> list:
+    """Quantize several 2-D weights of one dtype and one format in one launch
+    (plus one second-level launch with double quantization); the states are
+    bit for bit those of quantize() on each weight.  `outs` reuses earlier
+    states of the same shapes and format (no allocation)."""
+    _require_gpu(Ws[0])
+    qt = QTYPES[qtype] if isinstance(qtype, str) else int(qtype)
+    dtype = Ws[0].dtype
+    for W in Ws:
+        if W.dtype != dtype or W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
+            raise Q4Error("weights must be 2-D float16/bfloat16 tensors of one dtype")
+    Ws = [W.contiguous() for W in Ws]
+    dev = Ws[0].device
+    if outs is None:
+        outs = [_new_state(qt, dtype, W.shape[0], W.shape[1], blocksize, double_quant, dev) for W in Ws]
+    else:
+        for st, W in zip(outs, Ws):
+            if (st.qtype, st.rows, st.cols, st.blocksize, st.double_quant) != \
+                    (qt, W.shape[0], W.shape[1], blocksize, bool(double_quant)) or st.absmax is None:
+                raise Q4Error("outs= states have a different shape or format")
+            st.src_dtype = dtype
+    n = len(Ws)
+    rows = (ctypes.c_int64 * n)(*[W.shape[0] for W in Ws])
+    cols = (ctypes.c_int64 * n)(*[W.shape[1] for W in Ws])
+    wsz = ctypes.c_size_t(0)
+    _check(library().q4_quantize_grouped_workspace_size(n, rows, cols, blocksize, qt, int(double_quant),
+                                                         ctypes.byref(wsz)), "q4_quantize_grouped_workspace_size")
+    ws = _workspace(dev, "quantize", wsz.value)
+    structs = [st.c_struct() for st in outs]
+    arr = (ctypes.POINTER(_CState) * n)(*[ctypes.pointer(c) for c in structs])
+    wp = (ctypes.c_void_p * n)(*[W.data_ptr() for W in Ws])
+    _check(library().q4_quantize_grouped(n, wp, _DT[dtype], rows, cols, blocksize, qt, int(double_quant), arr,
+                                         _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+           "q4_quantize_grouped")
+    return outs
+
+
 def dequantize(st: Q4State, dtype: torch.dtype | None = None, out: torch.Tensor | None = None,
                stream=None) -> torch.Tensor:
     _require_gpu(st.packed)
@@ -314,6 +368,20 @@ def dequantize(st: Q4State, dtype: torch.dtype | None = None, out: torch.Tensor 
     _check(library().q4_dequantize(ctypes.byref(cs), _ptr(out), _DT[dtype], _stream(stream)),
            "q4_dequantize")
     return out
+
+
+def dequantize_grouped(states, dtype: torch.dtype | None = None, outs=None, stream=None) -> list:
+    """q4.dequantize of several states of one format in one launch."""
+    _require_gpu(states[0].packed)
+    dtype = dtype or states[0].src_dtype
+    if outs is None:
+        outs = [torch.empty(st.rows, st.cols, dtype=dtype, device=st.device) for st in states]
+    structs = [st.c_struct() for st in states]
+    n = len(states)
+    arr = (ctypes.POINTER(_CState) * n)(*[ctypes.pointer(c) for c in structs])
+    op = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
+    _check(library().q4_dequantize_grouped(n, arr, op, _DT[dtype], _stream(stream)), "q4_dequantize_grouped")
+    return outs
 
 
 _gemv_ws_need = {}  # (shapes and formats of the group, M) -> workspace bytes

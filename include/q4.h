@@ -183,6 +183,23 @@ Q4_API int q4_quantize_noalloc(const void *W, int32_t w_dtype, int64_t rows, int
                                int32_t blocksize, int32_t qtype, int32_t double_quant,
                                q4_state *out, void *stream);
 
+/*
+ * q4_quantize_grouped -- q4_quantize of `count` (1..16) matrices in one
+ * launch (plus one launch of the second-level quantization with
+ * double_quant), e.g. the seven projections of a decoder layer at load time.
+ * One format for all: w_dtype, blocksize, qtype and double_quant are
+ * shared; W[i] is [rows[i], cols[i]] and out[i] its state, with the rules
+ * and results of q4_quantize for each (bit for bit the same state).
+ *   workspace  device, q4_quantize_grouped_workspace_size() bytes,
+ *              zero-filled; every call leaves it zero-filled.
+ */
+Q4_API int q4_quantize_grouped_workspace_size(int32_t count, const int64_t *rows, const int64_t *cols,
+                                              int32_t blocksize, int32_t qtype, int32_t double_quant,
+                                              size_t *bytes);
+Q4_API int q4_quantize_grouped(int32_t count, const void *const *W, int32_t w_dtype, const int64_t *rows,
+                               const int64_t *cols, int32_t blocksize, int32_t qtype, int32_t double_quant,
+                               q4_state *const *out, void *workspace, size_t workspace_bytes, void *stream);
+
 /* ---- dequantize ------------------------------------------------------- */
 
 /*
@@ -195,6 +212,12 @@ Q4_API int q4_quantize_noalloc(const void *W, int32_t w_dtype, int64_t rows, int
  *   out  device, n elements, 16-byte aligned.
  */
 Q4_API int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream);
+
+/* q4_dequantize of `count` (1..16) states of one format (qtype, blocksize,
+ * double_quant) in one launch; out[i] receives state i (16-byte aligned,
+ * n elements of out_dtype).  Bit for bit the result of q4_dequantize. */
+Q4_API int q4_dequantize_grouped(int32_t count, const q4_state *const *Wq, void *const *out, int32_t out_dtype,
+                                 void *stream);
 
 /* ---- fused dequant-GEMV (decode, M <= 32) ------------------------------ */
 

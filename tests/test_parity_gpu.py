@@ -356,3 +356,57 @@ def test_gemv_workspace_left_zeroed_across_shapes(q4, oracle):
     ws = q4._ws.get((torch.cuda.current_device(), "gemv"))
     torch.cuda.synchronize()
     assert ws is not None and int(ws.count_nonzero().item()) == 0
+
+
+@pytest.mark.parametrize("qtype,bs,dq", [("nf4", 64, True), ("nf4", 32, False), ("nf4", 256, True),
+                                         ("int4_sym", 128, False), ("int4_asym", 128, False)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_quantize_grouped_equals_single_and_oracle(q4, oracle, qtype, bs, dq, dtype):
+    """One grouped launch over matrices of different (ragged) shapes gives,
+    bit for bit, the states q4.quantize gives for each and the oracle's;
+    twice in a row (the workspace is left zeroed)."""
+    g = torch.Generator().manual_seed(40 + bs)
+    shapes = [(300, 1024), (17, 96), (1024, 4096), (5, 7), (2048, 1088)]
+    Ws = [(torch.randn(N, K, generator=g) * 0.02).to(dtype) for N, K in shapes]
+    Ws[2].view(-1)[::997] *= 20
+    for _ in range(2):
+        sts = q4.quantize_grouped([dev(W) for W in Ws], bs, qtype, dq)
+        torch.cuda.synchronize()
+        for W, st in zip(Ws, sts):
+            assert_state_equal(st, oracle_state(oracle, W, bs, QT[qtype], dq))
+            single = q4.quantize(dev(W), bs, qtype, dq)
+            assert_state_equal(single, oracle_state(oracle, W, bs, QT[qtype], dq))
+    ws = q4._ws.get((torch.cuda.current_device(), "quantize"))
+    if ws is not None:
+        assert int(ws.count_nonzero().item()) == 0
+
+
+def test_quantize_grouped_7b_layer_mean_many_chunks(q4, oracle):
+    """The 7B layer in one grouped call: matrices of 1024 and 2752 chunks, so
+    the double-quant mean crosses subtrees of 2048 chunk sums."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    Ws = wl.layer_weights(wl.LAYER_7B, 0.02, seed=300)
+    sts = q4.quantize_grouped([dev(W) for W in Ws], 64, "nf4", True)
+    for W, st in zip(Ws, sts):
+        assert_state_equal(st, oracle_state(oracle, W, 64, 0, True))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("qtype,bs,dq", [("nf4", 64, True), ("nf4", 32, False), ("int4_sym", 128, False),
+                                         ("int4_asym", 256, False)])
+@pytest.mark.parametrize("out_dtype", [torch.float16, torch.bfloat16])
+def test_dequantize_grouped_equals_single_and_oracle(q4, oracle, qtype, bs, dq, out_dtype):
+    """One grouped dequantize launch over ragged shapes (spans that end
+    mid-matrix, matrices smaller than one span) writes, bit for bit, what
+    q4.dequantize writes for each matrix and what the oracle computes."""
+    g = torch.Generator().manual_seed(70 + bs)
+    shapes = [(3, 256), (300, 1024), (1, 256), (1024, 4096), (17, 768), (2048, 1280)]
+    Ws = [(torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16) for N, K in shapes]
+    sts = q4.quantize_grouped([dev(W) for W in Ws], bs, qtype, dq)
+    outs = q4.dequantize_grouped(sts, out_dtype)
+    torch.cuda.synchronize()
+    for W, st, o in zip(Ws, sts, outs):
+        single = q4.dequantize(st, out_dtype)
+        assert torch.equal(o.view(torch.int16), single.view(torch.int16))
+        ost = oracle_state(oracle, W, bs, QT[qtype], dq)
+        assert np.array_equal(bits(o), oracle.dequantize(ost, out_dtype == torch.bfloat16))
