@@ -109,10 +109,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Bounded wait: gives up after `limit_ns` (2 s unless the launch sets a
 // limit), raises Q4_STATUS_TIMEOUT and sets *abort.  The first probe is
 // inlined; only a phase that is not yet complete pays the call into the
-// polling loop.
+// polling loop.  A warp that waits for long (a copy warp ahead of its
+// consumers, a reducer between chunks) passes `sleep_ns` > 0: it sleeps
+// between probes instead of taking issue slots from the working warps of
+// its scheduler.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, int *status,
-                                                   volatile int *abort, uint64_t limit_ns) {
+                                                   volatile int *abort, uint64_t limit_ns, uint32_t sleep_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try(bar, parity)) return true;
@@ -122,12 +125,13 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
       *abort = 1;
       return false;
     }
+    if (sleep_ns) __nanosleep(sleep_ns);
   }
 }
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *status, volatile int *abort,
-                                          uint64_t limit_ns = kWaitLimitNs) {
+                                          uint64_t limit_ns = kWaitLimitNs, uint32_t sleep_ns = 0) {
   if (mbar_try(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, status, abort, limit_ns);
+  return mbar_wait_slow(bar, parity, status, abort, limit_ns, sleep_ns);
 }
 
 // Wait by a whole warp: only lane 0 polls the barrier (many polling lanes
@@ -136,9 +140,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *st
 // After lane 0 has seen the phase complete, each other lane queries it once
 // (returns at once) so that it acquires the data the phase published itself.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, int *status, volatile int *abort,
-                                               uint64_t limit_ns = kWaitLimitNs) {
+                                               uint64_t limit_ns = kWaitLimitNs, uint32_t sleep_ns = 0) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort, limit_ns);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, abort, limit_ns, sleep_ns);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   if (ok && (threadIdx.x & 31) != 0) (void)mbar_try(bar, parity);
   return ok;

@@ -501,6 +501,8 @@ int q4_quantize_grouped_workspace_size(int32_t count, const int64_t *rows, const
     const int rc = q4_state_sizes(qtype, rows[i] * cols[i], blocksize, double_quant, sz);
     if (rc != Q4_OK) return rc;
     const int64_t nb = ceil_div(rows[i] * cols[i], blocksize);
+    // the grouped kernel sums at most 65536 chunk sums per matrix
+    if (double_quant && ceil_div(nb, kChunkBlocks) > kQgMaxChunks) return Q4_ERR_SHAPE;
     if (double_quant) total += align256((size_t)ceil_div(nb, kChunkBlocks) * 8);
   }
   *bytes = double_quant ? total : 0;
@@ -580,11 +582,13 @@ int q4_quantize_grouped(int32_t count, const void *const *W, int32_t w_dtype, co
   p.count = count;
   p.total_chunks = chunks;
   p.status = di.status;
+  p.wait_ns = g_wait_limit_ns.load();
+  p.stall_copies = g_copy_stall.load();
   p.tab = tab;
   dp.count = count;
   dp.total_groups = groups;
   const cudaStream_t st = (cudaStream_t)stream;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(chunks, (int64_t)di.sms * 4));
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(chunks, (int64_t)di.sms));
   rc = run_quantize_grouped(w_dtype, qtype, blocksize, double_quant != 0, p, grid, st);
   if (rc == Q4_OK && double_quant) rc = run_double_quant_grouped(dp, st);
   return rc;

@@ -13,6 +13,7 @@
 #include "gemv.cuh"
 #include "gemv_small.cuh"
 #include "gemm.cuh"
+#include "quantize_grouped.cuh"
 
 namespace q4 {
 // Launch with programmatic stream serialization (the kernel calls

@@ -19,13 +19,11 @@
 // the double-quant mean is formed in the exact order of the definition (an
 // aligned binary tree) without atomics: lanes -> chunk (shared memory tree)
 // -> CTA run (streaming pairwise stack) -> the last CTA to finish combines the
-// per-CTA partial sums and writes the mean.  A grouped launch quantizes every
-// matrix of a layer at once: CTAs walk all matrices' chunks with a grid
-// stride, each chunk's sum goes to the workspace, and the CTA that counts a
-// matrix's last chunk combines them in the same tree order; one second
-// launch quantizes every matrix's groups of absmax values.
+// per-CTA partial sums and writes the mean.  The grouped launch over every
+// matrix of a layer (quantize_grouped.cuh) shares the per-thread step,
+// quant16; one second launch then quantizes every matrix's groups of absmax
+// values.
 #pragma once
-#include <type_traits>
 
 #include "q4_common.cuh"
 
@@ -81,7 +79,9 @@ constexpr int kQMaxGroup = 16;
 struct QuantGroupParams {
   QMat mat[kQMaxGroup];
   int32_t count;
+  int32_t stall_copies;  // test hook: the producer never fills a stage
   int64_t total_chunks;
+  uint64_t wait_ns;      // bound of every mbarrier wait
   int *status;
   Nf4BinTable tab;
 };
@@ -108,41 +108,140 @@ __device__ __forceinline__ uint32_t nf4_code_fast(float x, uint32_t tb) {
   return (uint32_t)(base + (x >= thr ? 1 : 0));
 }
 
-// The pairwise fp64 sum of len <= kMaxRunPartials values at src (level by
-// level, adjacent pairs, an odd last value carried up), staged in shared
-// memory by the whole CTA (every thread must call it).  Returns the sum in
-// every thread.
-__device__ __forceinline__ double tree_sum_smem(const double *src, int len, double *s_red, int tid) {
-  for (int i = tid; i < len; i += kQThreads) s_red[i] = __ldcg(src + i);
-  __syncthreads();
-  while (len > 1) {
-    const int half = len >> 1;
-    double t[kMaxRunPartials / kQThreads / 2 + 1];
-    int cnt = 0;
-    for (int i = tid; i < half; i += kQThreads) t[cnt++] = s_red[2 * i] + s_red[2 * i + 1];
-    const double carry = s_red[len - 1];
-    __syncthreads();
-    cnt = 0;
-    for (int i = tid; i < half; i += kQThreads) s_red[i] = t[cnt++];
-    if ((len & 1) && tid == 0) s_red[half] = carry;
-    __syncthreads();
-    len = half + (len & 1);
+// Codes of a thread's 16 consecutive elements (element 8k + j in bits
+// 4j..4j+3 of codes[k]) and its block's scale; the B/16 lanes of one block
+// (adjacent lanes) agree on `scale` and `z`.  Must be called by all 32 lanes.
+// tb: this lane's bin-table address minus 2^30; s_tab: the lane-private
+// bin tables ([bin][lane]); nonfinite is set when the block holds Inf / NaN.
+template <int DT, int QT, int B>
+__device__ __forceinline__ void quant16(const uint4 (&v)[2], float &scale, int &z, uint32_t (&codes)[2], int lane,
+                                        uint32_t tb, const float2 *s_tab, int &nonfinite) {
+  constexpr int E = 16, V = 2, LPB = B / E;
+  float f[E];
+#pragma unroll
+  for (int k = 0; k < V; ++k) {
+    const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[8 * k + 2 * j] = lo16<DT>(w[j]);
+      f[8 * k + 2 * j + 1] = hi16<DT>(w[j]);
+    }
+    codes[k] = 0;
   }
-  const double r = s_red[0];
-  __syncthreads();
-  return r;
+  if (QT == Q4_NF4 || QT == Q4_INT4_SYM) {
+    uint32_t m = absmax_bits8(v[0]);
+#pragma unroll
+    for (int k = 1; k < V; ++k) m = max(m, absmax_bits8(v[k]));
+#pragma unroll
+    for (int o = LPB / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float c = Dt<DT>::to_f((uint16_t)m);
+    if (!(c <= 3.4028235e38f)) nonfinite = 1;
+    if (QT == Q4_NF4) {
+      scale = c;
+      if (__all_sync(0xffffffffu, markstein_ok(c))) {
+        // every lane: finite weights with |w| <= c, so |x| <= 1
+        const float y = __frcp_rn(c);
+#pragma unroll
+        for (int k = 0; k < V; ++k)
+#pragma unroll
+          for (int j = 7; j >= 0; --j)
+            codes[k] = (codes[k] << 4) + nf4_code_fast(div_markstein(f[8 * k + j], c, y), tb);
+      } else {
+        const bool fast = markstein_ok(c);
+        const float y = fast ? __frcp_rn(c) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+          float x = fast ? div_markstein(f[j], c, y) : (c == 0.0f ? 0.0f : __fdiv_rn(f[j], c));
+          const float2 e = s_tab[nf4_bin(x) * 32 + lane];
+          const int code = __float_as_int(e.y) + (x >= e.x ? 1 : 0);
+          codes[j >> 3] |= (uint32_t)code << (4 * (j & 7));
+        }
+      }
+    } else {
+      const float s = __fdiv_rn(c, 7.0f);
+      scale = s;
+      if (__all_sync(0xffffffffu, markstein_ok(s))) {
+        // |w / s| <= 7 / (1 - 2^-24): rint never leaves [-7, 7], and adding
+        // 1.5 * 2^23 rounds to the nearest integer, ties to even, leaving
+        // its 4-bit two's complement in the low nibble
+        const float y = __frcp_rn(s);
+#pragma unroll
+        for (int k = 0; k < V; ++k)
+#pragma unroll
+          for (int j = 7; j >= 0; --j)
+            codes[k] = (codes[k] << 4) |
+                       (__float_as_uint(__fadd_rn(div_markstein(f[8 * k + j], s, y), 12582912.0f)) & 15u);
+      } else {
+        const bool fast = markstein_ok(s);
+        const float y = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+          int q = 0;
+          if (s != 0.0f) {
+            float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
+            q = min(max(__float2int_rn(x), -8), 7);
+          }
+          codes[j >> 3] |= (uint32_t)(q & 15) << (4 * (j & 7));
+        }
+      }
+    }
+  } else {  // Q4_INT4_ASYM
+    float mn = 0.0f, mx = 0.0f;
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      mn = fminf(mn, f[j]);
+      mx = fmaxf(mx, f[j]);
+    }
+    uint32_t m = absmax_bits8(v[0]);
+#pragma unroll
+    for (int k = 1; k < V; ++k) m = max(m, absmax_bits8(v[k]));
+#pragma unroll
+    for (int o = LPB / 2; o >= 1; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    }
+    if (!(Dt<DT>::to_f((uint16_t)m) <= 3.4028235e38f)) nonfinite = 1;
+    const float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+    scale = s;
+    z = 0;
+    if (__all_sync(0xffffffffu, markstein_ok(s))) {
+      // mn <= 0 <= mx and s = (mx - mn) / 15, so |w / s| <= 15 (1 + 2^-23):
+      // adding 1.5 * 2^23 rounds the quotient to the nearest integer, ties
+      // to even, with the integer in the low bits of the sum's pattern
+      const float y = __frcp_rn(s);
+      z = min(max(__float2int_rn(div_markstein(-mn, s, y)), 0), 15);
+#pragma unroll
+      for (int k = 0; k < V; ++k)
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+          const int r = (int)(__float_as_uint(__fadd_rn(div_markstein(f[8 * k + j], s, y), 12582912.0f)) -
+                              0x4B400000u);
+          codes[k] = (codes[k] << 4) | (uint32_t)min(max(r + z, 0), 15);
+        }
+    } else {
+      if (s != 0.0f) z = min(max(__float2int_rn(__fdiv_rn(-mn, s)), 0), 15);
+      const bool fast = markstein_ok(s);
+      const float y = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+      for (int j = 0; j < E; ++j) {
+        int q = 0;
+        if (s != 0.0f) {
+          float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
+          q = min(max(__float2int_rn(x) + z, 0), 15);
+        }
+        codes[j >> 3] |= (uint32_t)q << (4 * (j & 7));
+      }
+    }
+  }
 }
 
 // Four resident CTAs of 256 threads per SM (at most 64 registers): more
 // warps to hide the division and table latencies, with four 16-byte loads
 // in flight per thread.
-// GROUPED: one launch over the matrices of a QuantGroupParams; every CTA
-// walks the global chunks with a grid stride, each chunk's fp64 sum goes to
-// the matrix's partials and the CTA that counts a matrix's last chunk sums
-// them.  Otherwise one matrix; each CTA owns one run of chunks.
-template <int DT, int QT, int B, bool DQ, bool GROUPED = false>
-__global__ void __launch_bounds__(kQThreads, 4)
-    quantize_kernel(const __grid_constant__ std::conditional_t<GROUPED, QuantGroupParams, QuantParams> p) {
+// One matrix; each CTA owns one run of chunks.
+template <int DT, int QT, int B, bool DQ>
+__global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(const __grid_constant__ QuantParams p) {
   pdl_launch_then_wait();
   constexpr int E = 16;                          // consecutive elements per thread (one block)
   constexpr int V = E / 8;                       // 16-byte words per thread
@@ -159,7 +258,6 @@ __global__ void __launch_bounds__(kQThreads, 4)
   __shared__ double s_blk[2][kChunkBlocks];      // block absmax of a chunk, by chunk parity
   __shared__ uint8_t s_zero[BLK_IT];             // INT4_ASYM zero-points of one iteration
   __shared__ double s_stack[24];                 // streaming pairwise stack (thread 0)
-  __shared__ double s_red_all[GROUPED && DQ ? kMaxRunPartials : 1];  // a matrix's chunk sums (grouped)
   __shared__ int s_last;
 
   const int tid = threadIdx.x;
@@ -177,113 +275,6 @@ __global__ void __launch_bounds__(kQThreads, 4)
   int nonfinite = 0;
   int depth = 0;  // stack depth (thread 0)
   int cpar = 0;   // parity of s_blk for the current chunk
-
-  // Codes of the thread's E elements (element 8k + j in bits 4j..4j+3 of
-  // codes[k]) and the block's scale; lanes of one block agree on `scale`
-  // and `z`.
-  auto quantE = [&](const uint4 (&v)[V], float &scale, int &z, uint32_t (&codes)[V]) {
-    float f[E];
-#pragma unroll
-    for (int k = 0; k < V; ++k) {
-      const uint32_t w[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        f[8 * k + 2 * j] = lo16<DT>(w[j]);
-        f[8 * k + 2 * j + 1] = hi16<DT>(w[j]);
-      }
-      codes[k] = 0;
-    }
-    if (QT == Q4_NF4 || QT == Q4_INT4_SYM) {
-      uint32_t m = absmax_bits8(v[0]);
-#pragma unroll
-      for (int k = 1; k < V; ++k) m = max(m, absmax_bits8(v[k]));
-#pragma unroll
-      for (int o = LPB / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const float c = Dt<DT>::to_f((uint16_t)m);
-      if (!(c <= 3.4028235e38f)) nonfinite = 1;
-      if (QT == Q4_NF4) {
-        scale = c;
-        if (__all_sync(0xffffffffu, markstein_ok(c))) {
-          // every lane: finite weights with |w| <= c, so |x| <= 1
-          const float y = __frcp_rn(c);
-#pragma unroll
-          for (int k = 0; k < V; ++k)
-#pragma unroll
-            for (int j = 7; j >= 0; --j)
-              codes[k] = (codes[k] << 4) + nf4_code_fast(div_markstein(f[8 * k + j], c, y), tb);
-        } else {
-          const bool fast = markstein_ok(c);
-          const float y = fast ? __frcp_rn(c) : 0.0f;
-#pragma unroll
-          for (int j = 0; j < E; ++j) {
-            float x = fast ? div_markstein(f[j], c, y) : (c == 0.0f ? 0.0f : __fdiv_rn(f[j], c));
-            const float2 e = s_tab[nf4_bin(x) * 32 + lane];
-            const int code = __float_as_int(e.y) + (x >= e.x ? 1 : 0);
-            codes[j >> 3] |= (uint32_t)code << (4 * (j & 7));
-          }
-        }
-      } else {
-        const float s = __fdiv_rn(c, 7.0f);
-        scale = s;
-        if (__all_sync(0xffffffffu, markstein_ok(s))) {
-          // |w / s| <= 7 / (1 - 2^-24): rint never leaves [-7, 7], and adding
-          // 1.5 * 2^23 rounds to the nearest integer, ties to even, leaving
-          // its 4-bit two's complement in the low nibble
-          const float y = __frcp_rn(s);
-#pragma unroll
-          for (int k = 0; k < V; ++k)
-#pragma unroll
-            for (int j = 7; j >= 0; --j)
-              codes[k] = (codes[k] << 4) |
-                         (__float_as_uint(__fadd_rn(div_markstein(f[8 * k + j], s, y), 12582912.0f)) & 15u);
-        } else {
-          const bool fast = markstein_ok(s);
-          const float y = fast ? __frcp_rn(s) : 0.0f;
-#pragma unroll
-          for (int j = 0; j < E; ++j) {
-            int q = 0;
-            if (s != 0.0f) {
-              float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
-              q = min(max(__float2int_rn(x), -8), 7);
-            }
-            codes[j >> 3] |= (uint32_t)(q & 15) << (4 * (j & 7));
-          }
-        }
-      }
-    } else {  // Q4_INT4_ASYM
-      float mn = 0.0f, mx = 0.0f;
-#pragma unroll
-      for (int j = 0; j < E; ++j) {
-        mn = fminf(mn, f[j]);
-        mx = fmaxf(mx, f[j]);
-      }
-      uint32_t m = absmax_bits8(v[0]);
-#pragma unroll
-      for (int k = 1; k < V; ++k) m = max(m, absmax_bits8(v[k]));
-#pragma unroll
-      for (int o = LPB / 2; o >= 1; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      }
-      if (!(Dt<DT>::to_f((uint16_t)m) <= 3.4028235e38f)) nonfinite = 1;
-      const float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-      scale = s;
-      z = 0;
-      if (s != 0.0f) z = min(max(__float2int_rn(__fdiv_rn(-mn, s)), 0), 15);
-      const bool fast = markstein_ok(s);
-      const float y = fast ? __frcp_rn(s) : 0.0f;
-#pragma unroll
-      for (int j = 0; j < E; ++j) {
-        int q = 0;
-        if (s != 0.0f) {
-          float x = fast ? div_markstein(f[j], s, y) : __fdiv_rn(f[j], s);
-          q = min(max(__float2int_rn(x) + z, 0), 15);
-        }
-        codes[j >> 3] |= (uint32_t)q << (4 * (j & 7));
-      }
-    }
-  };
 
   // One chunk (256 blocks) of a matrix; with double quantization returns the
   // fp64 pairwise sum of its block absmax values (valid in thread 0).
@@ -328,7 +319,7 @@ __global__ void __launch_bounds__(kQThreads, 4)
           float scale = 0.0f;
           int z = 0;
           uint32_t codes[V];
-          quantE(v[b], scale, z, codes);
+          quant16<DT, QT, B>(v[b], scale, z, codes, lane, tb, s_tab, nonfinite);
           if (QT == Q4_INT4_ASYM && (tid % LPB) == 0) s_zero[(tid * E) / B] = (uint8_t)z;
           // ---- stores
           const int64_t e0 = chunk_e0 + off + tid * E;
@@ -385,7 +376,7 @@ __global__ void __launch_bounds__(kQThreads, 4)
     return chunk_sum;
   };
 
-  if constexpr (!GROUPED) {
+  {
     const int64_t c0 = (int64_t)blockIdx.x * p.run;
     const int64_t c1 = min(c0 + p.run, p.n_chunks);
     for (int64_t chunk = c0; chunk < c1; ++chunk) {
@@ -400,56 +391,11 @@ __global__ void __launch_bounds__(kQThreads, 4)
         }
       }
     }
-  } else {
-    int mi = 0;
-    for (int64_t gc = blockIdx.x; gc < p.total_chunks; gc += gridDim.x) {
-      while (mi + 1 < p.count && gc >= p.mat[mi + 1].chunk_begin) ++mi;
-      const QMat &m = p.mat[mi];
-      const int64_t chunk = gc - m.chunk_begin;
-      const double cs = do_chunk(m.W, m.n, m.nb, m.packed, m.absmax, m.zero, chunk);
-      if constexpr (DQ) {
-        if (tid == 0) {
-          m.partials[chunk] = cs;
-          __threadfence();
-          s_last = atomicAdd(m.counter, 1u) == (unsigned)(m.n_chunks - 1);
-        }
-        __syncthreads();
-        if (s_last) {
-          // this CTA counted the matrix's last chunk: the pairwise tree over
-          // its chunk sums, as aligned subtrees of kMaxRunPartials values
-          // (each reduced level by level, odd last carried up) and then the
-          // tree over the subtree sums -- the same order as one tree
-          __threadfence();
-          double sub[32];
-          int nsub = 0;
-          for (int64_t b0 = 0; b0 < m.n_chunks; b0 += kMaxRunPartials) {
-            const int len = (int)min((int64_t)kMaxRunPartials, m.n_chunks - b0);
-            const double t = tree_sum_smem(m.partials + b0, len, s_red_all, tid);
-            if (nsub < 32) sub[nsub] = t;
-            ++nsub;
-          }
-          // the workspace is left zeroed
-          for (int64_t i = tid; i < m.n_chunks; i += kQThreads) __stcg(m.partials + i, 0.0);
-          if (tid == 0) {
-            int len = nsub;
-            while (len > 1) {
-              const int half = len >> 1;
-              for (int i = 0; i < half; ++i) sub[i] = sub[2 * i] + sub[2 * i + 1];
-              if (len & 1) sub[half] = sub[len - 1];
-              len = half + (len & 1);
-            }
-            m.absmax_mean[0] = __double2float_rn(__ddiv_rn(sub[0], (double)m.nb));
-            *m.counter = 0u;  // leave the workspace zeroed for the next call
-          }
-          __syncthreads();
-        }
-      }
-    }
   }
 
   if (nonfinite) raise_status(p.status, Q4_STATUS_NONFINITE);
 
-  if constexpr (DQ && !GROUPED) {
+  if constexpr (DQ) {
     const int64_t c0 = (int64_t)blockIdx.x * p.run;
     const int64_t c1 = min(c0 + p.run, p.n_chunks);
     if (tid == 0) {
@@ -517,29 +463,56 @@ struct DqGroupParams {
 
 // One group of 256 block absmax values, by one warp:
 // m2 = max|c - mu|, s2 = m2 / 127, q2 = clamp(rint((c - mu) / s2), -128, 127).
+// Lane l owns blocks 8l..8l+7 of the group: two 16-byte loads and one 8-byte
+// store when the group is whole and the arrays are aligned for them.  The
+// quotients are correctly rounded (Markstein's correction where the divisor
+// allows it, as in the first-level quantizer; IEEE division otherwise).
 __device__ __forceinline__ void double_quant_group(const float *__restrict__ absmax, int64_t nb, float mu,
                                                    int8_t *__restrict__ absmax_q, float *__restrict__ absmax_scale,
                                                    int64_t g, int lane) {
+  const int64_t b0 = g * Q4_DQ_GROUP + lane * 8;
+  const bool vec = g * Q4_DQ_GROUP + Q4_DQ_GROUP <= nb && ((uintptr_t)absmax & 15u) == 0 &&
+                   ((uintptr_t)absmax_q & 7u) == 0;
   float d[8];
   float m2 = 0.0f;
+  if (vec) {
+    const float4 x0 = __ldg(reinterpret_cast<const float4 *>(absmax + b0));
+    const float4 x1 = __ldg(reinterpret_cast<const float4 *>(absmax + b0 + 4));
+    const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int64_t b = g * Q4_DQ_GROUP + lane * 8 + j;
-    d[j] = (b < nb) ? __fsub_rn(__ldg(absmax + b), mu) : 0.0f;
-    if (b < nb) m2 = fmaxf(m2, fabsf(d[j]));
+    for (int j = 0; j < 8; ++j) {
+      d[j] = __fsub_rn(x[j], mu);
+      m2 = fmaxf(m2, fabsf(d[j]));
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      d[j] = (b0 + j < nb) ? __fsub_rn(__ldg(absmax + b0 + j), mu) : 0.0f;
+      if (b0 + j < nb) m2 = fmaxf(m2, fabsf(d[j]));
+    }
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, o));
   const float s2 = __fdiv_rn(m2, 127.0f);
   if (lane == 0) absmax_scale[g] = s2;
+  const bool fast = markstein_ok(s2);
+  const float y = fast ? __frcp_rn(s2) : 0.0f;
+  uint32_t q[2] = {0u, 0u};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const int64_t b = g * Q4_DQ_GROUP + lane * 8 + j;
-    if (b < nb) {
-      int q2 = 0;
-      if (s2 != 0.0f) q2 = min(max(__float2int_rn(__fdiv_rn(d[j], s2)), -128), 127);
-      absmax_q[b] = (int8_t)q2;
+    int q2 = 0;
+    if (s2 != 0.0f) {
+      const float x = fast ? div_markstein(d[j], s2, y) : __fdiv_rn(d[j], s2);
+      q2 = min(max(__float2int_rn(x), -128), 127);
     }
+    q[j >> 2] |= (uint32_t)(q2 & 0xFF) << (8 * (j & 3));
+  }
+  if (vec) {
+    *reinterpret_cast<uint2 *>(absmax_q + b0) = make_uint2(q[0], q[1]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (b0 + j < nb) absmax_q[b0 + j] = (int8_t)(q[j >> 2] >> (8 * (j & 3)));
   }
 }
 

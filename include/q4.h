@@ -190,8 +190,13 @@ Q4_API int q4_quantize_noalloc(const void *W, int32_t w_dtype, int64_t rows, int
  * One format for all: w_dtype, blocksize, qtype and double_quant are
  * shared; W[i] is [rows[i], cols[i]] and out[i] its state, with the rules
  * and results of q4_quantize for each (bit for bit the same state).
+ * Runs one CTA per SM over the 256-block chunks of all matrices; W[i] must
+ * be 16-byte aligned (its pieces are copied by the bulk-copy engine).
+ * With double_quant, a matrix may hold at most 65536 groups of 256 blocks
+ * (Q4_ERR_SHAPE otherwise: e.g. 2^30 weights at blocksize 64).
  *   workspace  device, q4_quantize_grouped_workspace_size() bytes,
- *              zero-filled; every call leaves it zero-filled.
+ *              zero-filled; every call leaves it zero-filled (after a
+ *              Q4_STATUS_TIMEOUT it must be zero-filled again).
  */
 Q4_API int q4_quantize_grouped_workspace_size(int32_t count, const int64_t *rows, const int64_t *cols,
                                               int32_t blocksize, int32_t qtype, int32_t double_quant,
@@ -281,15 +286,16 @@ Q4_API int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *
  * this call, process-wide; 0 restores the default of 2 s.  A wait that runs
  * out raises Q4_STATUS_TIMEOUT: the kernel stops, waits for its own copies
  * in flight and returns, leaving its outputs undefined.  After a timeout the
- * GEMV workspace must be zero-filled again before its next use.  Host only;
- * no device needed. */
+ * GEMV or grouped-quantize workspace must be zero-filled again before its
+ * next use.  Host only; no device needed. */
 Q4_API int q4_set_wait_limit_ns(uint64_t ns);
 
 /* Test hook for the bounded waits, process-wide: while `on` is non-zero the
- * decode GEMV's copy warp issues no copies, so every compute warp's wait for
- * a weight stage runs out after the wait limit (set a short one first) and
- * the call returns with Q4_STATUS_TIMEOUT and undefined outputs.  Leave it
- * off otherwise.  Host only. */
+ * copy warp of the decode GEMV and of the grouped quantize issues no
+ * copies, so every compute warp's wait for a stage runs out after the wait
+ * limit (set a short one first) and the call returns with
+ * Q4_STATUS_TIMEOUT and undefined outputs.  Leave it off otherwise.  Host
+ * only. */
 Q4_API int q4_set_copy_stall(int32_t on);
 
 /* Reads (synchronously) the sticky device status word of the current

@@ -179,6 +179,27 @@ def test_gemv_workspace_sizes_per_format(lib):
     assert asym(1) == asym(8) < asym(9) == asym(16) < asym(17) == asym(32)
 
 
+def test_quantize_grouped_workspace_sizes(lib):
+    """The grouped quantize needs a workspace only with double quantization:
+    256 bytes of counters plus one fp64 sum per 256-block chunk of each
+    matrix (256-byte aligned); a matrix of more than 65536 chunks is a shape
+    error there (2^30 weights at blocksize 64), and fine without it."""
+    def size(shapes, bs, dq):
+        n = len(shapes)
+        rows = (ctypes.c_int64 * n)(*[r for r, _ in shapes])
+        cols = (ctypes.c_int64 * n)(*[c for _, c in shapes])
+        out = ctypes.c_size_t(0)
+        rc = lib.q4_quantize_grouped_workspace_size(n, rows, cols, bs, 0, int(dq), ctypes.byref(out))
+        return rc, out.value
+    assert size([(4096, 4096), (11008, 4096)], 64, False) == (0, 0)
+    # 1024 and 2752 chunks -> 8192 and 22016 bytes
+    assert size([(4096, 4096), (11008, 4096)], 64, True) == (0, 256 + 8192 + 22016)
+    assert size([(1, 5)], 64, True) == (0, 256 + 256)
+    assert size([(65536, 65536 * 256 * 64 // 65536)], 64, True)[0] == 0          # 65536 chunks
+    assert size([(65537, 65536 * 256 * 64 // 65536)], 64, True)[0] == -2         # one row more
+    assert size([(65537, 65536 * 256 * 64 // 65536)], 64, False) == (0, 0)
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_gemv_host_checks_before_the_device(lib):
     """The GEMV's format checks run on the host, matrix by matrix, before

@@ -1,10 +1,10 @@
 """Failure detection without a GPU fault: every pipeline wait in the decode
-GEMVs is bounded by the launch's wait limit.  With the copy stall test hook
-on, the copy warp issues no weight copies (a flag that nothing sets), so
-every compute warp's wait for a stage must run out after the (short) wait
-limit: the call must set Q4_STATUS_TIMEOUT and return, and after switching
-the hook off, restoring the limit and re-zeroing the workspace, the next
-call is correct."""
+GEMVs and the grouped quantize is bounded by the launch's wait limit.  With
+the copy stall test hook on, the copy warp issues no copies (a flag that
+nothing sets), so every compute warp's wait for a stage must run out after
+the (short) wait limit: the call must set Q4_STATUS_TIMEOUT and return, and
+after switching the hook off, restoring the limit and re-zeroing the
+workspace, the next call is correct."""
 import numpy as np
 import pytest
 import torch
@@ -44,4 +44,32 @@ def test_gemv_wait_limit_times_out_and_recovers(oracle, qtype, bs, dq, N, K):
     w16 = oracle.dequantize(ost, False).reshape(N, K)[rows]
     ref = oracle.matmul(bits(A), False, w16, False, M, len(rows), K)
     assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+    assert q4.last_device_status() == 0
+
+
+@pytest.mark.parametrize("dq", [True, False])
+def test_grouped_quantize_wait_limit_times_out_and_recovers(oracle, dq):
+    """The grouped quantize's consumer warps wait for ring stages that the
+    stalled producer never fills: Q4_STATUS_TIMEOUT, then a correct call."""
+    from bit_blockwise_weight_absmax_b200 import build
+    build.build()
+    from bit_blockwise_weight_absmax_b200 import q4
+    from gpu_helpers import assert_state_equal
+    g = torch.Generator().manual_seed(6)
+    Ws = [torch.randn(N, K, generator=g).mul(0.02).bfloat16() for N, K in [(1024, 4096), (3000, 1024)]]
+    q4.clear_device_status()
+    try:
+        q4.set_wait_limit_ns(200_000)
+        q4.set_copy_stall(True)
+        q4.quantize_grouped([W.cuda() for W in Ws], 64, "nf4", dq)
+        torch.cuda.synchronize()
+        assert q4.last_device_status() & 2
+    finally:
+        q4.set_copy_stall(False)
+        q4.set_wait_limit_ns(0)
+        q4.reset_workspaces()
+        q4.clear_device_status()
+    sts = q4.quantize_grouped([W.cuda() for W in Ws], 64, "nf4", dq)
+    for W, st in zip(Ws, sts):
+        assert_state_equal(st, oracle_state(oracle, W, 64, 0, dq))
     assert q4.last_device_status() == 0
