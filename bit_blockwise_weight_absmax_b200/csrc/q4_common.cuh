@@ -91,6 +91,39 @@ __device__ __forceinline__ float div_markstein(float a, float b, float y) {
   return __fmaf_rn(r, y, q);
 }
 
+// Two binary32 values in one 64-bit register for the packed f32x2 ALU ops
+// of sm_100 (each lane of a pair is computed and rounded exactly as the
+// scalar instruction would).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// div_markstein on a pair: yy = {y, y}, nb = {-b, -b}.
+__device__ __forceinline__ uint64_t div_markstein2(uint64_t a, uint64_t nb, uint64_t yy) {
+  const uint64_t q = f2_mul(a, yy);
+  const uint64_t r = f2_fma(q, nb, a);
+  return f2_fma(r, yy, q);
+}
+
 __device__ __forceinline__ bool markstein_ok(float b) {
   float ab = fabsf(b);
   return ab >= 8.0779356e-28f /* 2^-90 */ && ab <= 4.2535296e37f /* 2^125 */;

@@ -96,12 +96,12 @@ __device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
   return max(m & 0xFFFFu, m >> 16);
 }
 
-// NF4 code of x = RN(w / c) for |x| <= 1 (w finite): the bin is the low byte
-// of fmaf(x, 15, 1.5 * 2^23 + 15) (0..30), whose pattern is 0x4B4000jj, so
-// (pattern << 8) = 0x40000000 + 256 j and `tb` = table address of this lane
-// minus 0x40000000 gives the entry of bin j (32-bit shared addresses wrap).
-__device__ __forceinline__ uint32_t nf4_code_fast(float x, uint32_t tb) {
-  const uint32_t bits = __float_as_uint(__fmaf_rn(x, 15.0f, 12582927.0f));
+// NF4 code of x = RN(w / c) for |x| <= 1 (w finite) from `bits`, the
+// pattern of fmaf(x, 15, 1.5 * 2^23 + 15): the bin is its low byte (0..30),
+// the pattern is 0x4B4000jj, so (bits << 8) = 0x40000000 + 256 j and `tb` =
+// table address of this lane minus 0x40000000 gives the entry of bin j
+// (32-bit shared addresses wrap).
+__device__ __forceinline__ uint32_t nf4_code_bits(uint32_t bits, float x, uint32_t tb) {
   float thr;
   int base;
   asm("ld.shared.v2.b32 {%0,%1}, [%2];" : "=f"(thr), "=r"(base) : "r"((bits << 8) + tb));
@@ -139,13 +139,23 @@ __device__ __forceinline__ void quant16(const uint4 (&v)[2], float &scale, int &
     if (QT == Q4_NF4) {
       scale = c;
       if (__all_sync(0xffffffffu, markstein_ok(c))) {
-        // every lane: finite weights with |w| <= c, so |x| <= 1
+        // every lane: finite weights with |w| <= c, so |x| <= 1; the
+        // quotients and bins of two weights per packed instruction
         const float y = __frcp_rn(c);
+        const uint64_t yy = f2_pack(y, y), nc = f2_pack(-c, -c);
+        const uint64_t k15 = f2_pack(15.0f, 15.0f), kbin = f2_pack(12582927.0f, 12582927.0f);
 #pragma unroll
         for (int k = 0; k < V; ++k)
 #pragma unroll
-          for (int j = 7; j >= 0; --j)
-            codes[k] = (codes[k] << 4) + nf4_code_fast(div_markstein(f[8 * k + j], c, y), tb);
+          for (int j = 3; j >= 0; --j) {
+            const uint64_t x2 = div_markstein2(f2_pack(f[8 * k + 2 * j], f[8 * k + 2 * j + 1]), nc, yy);
+            const uint64_t b2 = f2_fma(x2, k15, kbin);
+            float x0, x1, b0, b1;
+            f2_unpack(x2, x0, x1);
+            f2_unpack(b2, b0, b1);
+            codes[k] = (codes[k] << 4) + nf4_code_bits(__float_as_uint(b1), x1, tb);
+            codes[k] = (codes[k] << 4) + nf4_code_bits(__float_as_uint(b0), x0, tb);
+          }
       } else {
         const bool fast = markstein_ok(c);
         const float y = fast ? __frcp_rn(c) : 0.0f;
@@ -165,12 +175,17 @@ __device__ __forceinline__ void quant16(const uint4 (&v)[2], float &scale, int &
         // 1.5 * 2^23 rounds to the nearest integer, ties to even, leaving
         // its 4-bit two's complement in the low nibble
         const float y = __frcp_rn(s);
+        const uint64_t yy = f2_pack(y, y), ns = f2_pack(-s, -s);
+        const uint64_t kr = f2_pack(12582912.0f, 12582912.0f);
 #pragma unroll
         for (int k = 0; k < V; ++k)
 #pragma unroll
-          for (int j = 7; j >= 0; --j)
-            codes[k] = (codes[k] << 4) |
-                       (__float_as_uint(__fadd_rn(div_markstein(f[8 * k + j], s, y), 12582912.0f)) & 15u);
+          for (int j = 3; j >= 0; --j) {
+            const uint64_t r2 = f2_add(div_markstein2(f2_pack(f[8 * k + 2 * j], f[8 * k + 2 * j + 1]), ns, yy), kr);
+            float r0, r1;
+            f2_unpack(r2, r0, r1);
+            codes[k] = (codes[k] << 8) | ((__float_as_uint(r1) & 15u) << 4) | (__float_as_uint(r0) & 15u);
+          }
       } else {
         const bool fast = markstein_ok(s);
         const float y = fast ? __frcp_rn(s) : 0.0f;
@@ -211,13 +226,18 @@ __device__ __forceinline__ void quant16(const uint4 (&v)[2], float &scale, int &
       // to even, with the integer in the low bits of the sum's pattern
       const float y = __frcp_rn(s);
       z = min(max(__float2int_rn(div_markstein(-mn, s, y)), 0), 15);
+      const uint64_t yy = f2_pack(y, y), ns = f2_pack(-s, -s);
+      const uint64_t kr = f2_pack(12582912.0f, 12582912.0f);
 #pragma unroll
       for (int k = 0; k < V; ++k)
 #pragma unroll
-        for (int j = 7; j >= 0; --j) {
-          const int r = (int)(__float_as_uint(__fadd_rn(div_markstein(f[8 * k + j], s, y), 12582912.0f)) -
-                              0x4B400000u);
-          codes[k] = (codes[k] << 4) | (uint32_t)min(max(r + z, 0), 15);
+        for (int j = 3; j >= 0; --j) {
+          const uint64_t r2 = f2_add(div_markstein2(f2_pack(f[8 * k + 2 * j], f[8 * k + 2 * j + 1]), ns, yy), kr);
+          float r0, r1;
+          f2_unpack(r2, r0, r1);
+          const int q0 = min(max((int)(__float_as_uint(r0) - 0x4B400000u) + z, 0), 15);
+          const int q1 = min(max((int)(__float_as_uint(r1) - 0x4B400000u) + z, 0), 15);
+          codes[k] = (codes[k] << 8) | ((uint32_t)q1 << 4) | (uint32_t)q0;
         }
     } else {
       if (s != 0.0f) z = min(max(__float2int_rn(__fdiv_rn(-mn, s)), 0), 15);
