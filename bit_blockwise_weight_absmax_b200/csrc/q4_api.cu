@@ -595,24 +595,7 @@ int q4_quantize_grouped(int32_t count, const void *const *W, int32_t w_dtype, co
 }
 
 int q4_dequantize(const q4_state *Wq, void *out, int32_t out_dtype, void *stream) {
-  int rc = check_state(Wq);
-  if (rc != Q4_OK) return rc;
-  if (!out || !valid_in_dtype(out_dtype)) return Q4_ERR_ARG;
-  if (!aligned16(out)) return Q4_ERR_ALIGN;
-  const DeviceInfo di = device_info();
-  if (di.ok != Q4_OK) return di.ok;
-  DequantParams p;
-  p.packed = Wq->packed;
-  p.absmax = Wq->absmax;
-  p.zero = Wq->zero;
-  p.absmax_q = Wq->absmax_q;
-  p.absmax_scale = Wq->absmax_scale;
-  p.absmax_mean = Wq->absmax_mean;
-  p.n = Wq->n;
-  p.out = out;
-  memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
-  return run_dequantize(Wq->qtype, out_dtype, Wq->blocksize, Wq->double_quant != 0, p, di.sms,
-                        (cudaStream_t)stream);
+  return q4_dequantize_grouped(1, &Wq, &out, out_dtype, stream);  // the same kernel, a group of one
 }
 
 int q4_dequantize_grouped(int32_t count, const q4_state *const *Wq, void *const *out, int32_t out_dtype,
@@ -649,8 +632,8 @@ int q4_dequantize_grouped(int32_t count, const q4_state *const *Wq, void *const 
   p.count = count;
   p.total_spans = spans;
   memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
-  return run_dequantize_grouped(Wq[0]->qtype, out_dtype, Wq[0]->blocksize, Wq[0]->double_quant != 0, p, di.sms,
-                                (cudaStream_t)stream);
+  return run_dequantize(Wq[0]->qtype, out_dtype, Wq[0]->blocksize, Wq[0]->double_quant != 0, p, di.sms,
+                        (cudaStream_t)stream);
 }
 
 int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {
