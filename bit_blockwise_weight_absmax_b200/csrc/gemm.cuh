@@ -26,7 +26,8 @@
 //               block scales come 16 blocks per load.  Then the epilogue:
 //               tcgen05.ld of the accumulators, convert, store.
 // Every mbarrier wait is bounded in time; a timeout sets Q4_STATUS_TIMEOUT,
-// stops the pipeline, waits for issued copies and frees TMEM.
+// stops the pipeline, waits for issued copies and for the issued MMAs, and
+// frees TMEM.
 #pragma once
 #include <cuda.h>
 
@@ -71,8 +72,9 @@ struct GemmParams {
   int32_t count;
   int32_t y_dtype;
   int32_t dq;
-  int32_t pad;
+  int32_t stall_copies;  // test hook: the producer issues no copies
   int64_t total_tiles;
+  uint64_t wait_ns;      // bound of every mbarrier wait
   int *status;
   float levels[16];
 };
@@ -290,14 +292,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kGemmStages;
           const uint32_t use = it / kGemmStages;
-          if (!mbar_wait(empty_bar(s), (use & 1) ^ 1, p.status, abort)) break;
+          if (!mbar_wait(empty_bar(s), (use & 1) ^ 1, p.status, abort, p.wait_ns)) break;
+          if (p.stall_copies) continue;  // test hook: the stage is never filled
           mbar_arrive_expect_tx(full_bar(s), kGemmATile + kGemmRawTile);
           tma_load_2d(smem_u32(sA + s * kGemmATile), &m.tmA, full_bar(s), kb * kGemmBK, tc.tm * kGemmBM);
           tma_load_2d(smem_u32(sR + s * kGemmRawTile), &m.tmW, full_bar(s), kb * (kGemmBK / 2), tc.tn * kGemmBN);
         }
       }
       // every issued copy completes before the CTA may exit
-      for (uint32_t j = (it > kGemmStages ? it - kGemmStages : 0); j < it; ++j) {
+      for (uint32_t j = (it > kGemmStages ? it - kGemmStages : 0); j < it && !p.stall_copies; ++j) {
         int dummy = 0;
         volatile int no_abort = 0;
         mbar_wait(full_bar(j % kGemmStages), (j / kGemmStages) & 1, &dummy, &no_abort);
@@ -309,18 +312,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const uint32_t idesc = umma_idesc_f16(DA == Q4_BF16 ? 1 : 0, 128, kGemmBN);
       static_assert(kGemmBN % 16 == 0 && kGemmBN <= 256, "UMMA N for M = 128");
       uint32_t it = 0, tcount = 0;
+      uint32_t last_bar = 0, last_par = 0;  // the barrier and phase of the last commit issued
+      bool committed = false;
       for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++tcount) {
         const TileCoord tc = gemm_tile(p, t);
         const int nk = p.mat[tc.mi].K / kGemmBK;
         const int ab = tcount & 1;  // accumulator set of this tile
-        if (!mbar_wait(accempty_bar(ab), ((tcount >> 1) & 1) ^ 1, p.status, abort)) break;
+        if (!mbar_wait(accempty_bar(ab), ((tcount >> 1) & 1) ^ 1, p.status, abort, p.wait_ns)) break;
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % kGemmStages;
           const uint32_t use = it / kGemmStages;
-          if (!mbar_wait(full_bar(s), use & 1, p.status, abort) ||
-              !mbar_wait(bfull_bar(s), use & 1, p.status, abort)) {
+          if (!mbar_wait(full_bar(s), use & 1, p.status, abort, p.wait_ns) ||
+              !mbar_wait(bfull_bar(s), use & 1, p.status, abort, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -337,16 +342,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             }
           }
           umma_commit(empty_bar(s));
+          last_bar = empty_bar(s), last_par = use & 1, committed = true;
         }
         if (!ok) break;
         umma_commit(accfull_bar(ab));
+        last_bar = accfull_bar(ab), last_par = (tcount >> 1) & 1, committed = true;
       }
-      // the last commits land before the CTA may exit
-      if (tcount > 0 && !*abort) {
+      // Every MMA issued completes before the CTA may free its TMEM, also
+      // after a timeout: a commit's arrival covers all earlier MMAs of this
+      // thread, so waiting for the last one is enough (nothing else arrives
+      // on that barrier phase, so it completes).
+      if (committed) {
         int dummy = 0;
         volatile int no_abort = 0;
-        const uint32_t last = tcount - 1;
-        mbar_wait(accfull_bar(last & 1), (last >> 1) & 1, &dummy, &no_abort);
+        mbar_wait(last_bar, last_par, &dummy, &no_abort);
       }
     }
   } else {
@@ -362,7 +371,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     auto epilogue = [&](const TileCoord &tc, uint32_t tcount) -> bool {
       const GemmMat &m = p.mat[tc.mi];
         const int ab = tcount & 1;
-        if (!mbar_wait_warp(accfull_bar(ab), (tcount >> 1) & 1, p.status, abort)) return false;
+        if (!mbar_wait_warp(accfull_bar(ab), (tcount >> 1) & 1, p.status, abort, p.wait_ns)) return false;
         tc_fence_after();
 #pragma unroll 1
         for (int piece = 0; piece < kGemmAccs * kGemmBN / 128; ++piece) {
@@ -498,7 +507,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         // lanes' reads of the stage after it
         {
           bool ready = true;
-          if (lane == 0) ready = mbar_wait(full_bar(s), use & 1, p.status, abort);
+          if (lane == 0) ready = mbar_wait(full_bar(s), use & 1, p.status, abort, p.wait_ns);
           if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) {
             ok = false;
             break;

@@ -752,6 +752,8 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     p.total_tiles = tiles;
     p.status = di.status;
     memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+    p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
     rc = run_gemm(a_dtype, p, di.sms, (cudaStream_t)stream);
   }
   return rc;

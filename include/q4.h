@@ -291,7 +291,7 @@ Q4_API int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *
 Q4_API int q4_set_wait_limit_ns(uint64_t ns);
 
 /* Test hook for the bounded waits, process-wide: while `on` is non-zero the
- * copy warp of the decode GEMV and of the grouped quantize issues no
+ * copy warp of the decode GEMV, the GEMM and the grouped quantize issues no
  * copies, so every compute warp's wait for a stage runs out after the wait
  * limit (set a short one first) and the call returns with
  * Q4_STATUS_TIMEOUT and undefined outputs.  Leave it off otherwise.  Host

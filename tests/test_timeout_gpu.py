@@ -73,3 +73,36 @@ def test_grouped_quantize_wait_limit_times_out_and_recovers(oracle, dq):
     for W, st in zip(Ws, sts):
         assert_state_equal(st, oracle_state(oracle, W, 64, 0, dq))
     assert q4.last_device_status() == 0
+
+
+def test_gemm_wait_limit_times_out_and_recovers(oracle):
+    """The GEMM's MMA and dequant warps wait for tiles that the stalled
+    producer never copies: Q4_STATUS_TIMEOUT, the kernel returns (waiting
+    for its issued MMAs before it frees the tensor memory), and a following
+    call is correct."""
+    from bit_blockwise_weight_absmax_b200 import build
+    build.build()
+    from bit_blockwise_weight_absmax_b200 import q4
+    g = torch.Generator().manual_seed(7)
+    M, N, K = 512, 1024, 2048
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).bfloat16()
+    st = q4.quantize(W.cuda(), 64, "nf4", True)
+    q4.clear_device_status()
+    try:
+        q4.set_wait_limit_ns(200_000)
+        q4.set_copy_stall(True)
+        q4.gemm(A.cuda(), st)
+        torch.cuda.synchronize()
+        assert q4.last_device_status() & 2
+    finally:
+        q4.set_copy_stall(False)
+        q4.set_wait_limit_ns(0)
+        q4.clear_device_status()
+    y = q4.gemm(A.cuda(), st)
+    rows = np.arange(0, N, 37)
+    ost = oracle_state(oracle, W, 64, 0, True)
+    w16 = oracle.dequantize(ost, True).reshape(N, K)[rows]
+    ref = oracle.matmul(bits(A), True, w16, True, M, len(rows), K)
+    assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+    assert q4.last_device_status() == 0
