@@ -56,6 +56,7 @@ constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmScBytes + 1024 /*
 struct alignas(64) GemmMat {
   CUtensorMap tmA;  // A [M, K] 16-bit, box {64, 256}, 128B swizzle
   CUtensorMap tmW;  // packed [N, K/2] bytes, box {32, 128}
+  const uint8_t *zero;  // INT4 asymmetric zero-points, two per byte
   const int8_t *absmax_q;
   const float *absmax_scale;
   const float *absmax_mean;
@@ -73,6 +74,8 @@ struct GemmParams {
   int32_t y_dtype;
   int32_t dq;
   int32_t stall_copies;  // test hook: the producer issues no copies
+  int32_t log2_bs;       // blocksize B = 2^log2_bs (32 .. 256)
+  int32_t pad2;
   int64_t total_tiles;
   uint64_t wait_ns;      // bound of every mbarrier wait
   int *status;
@@ -232,9 +235,15 @@ __device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t t) {
   return TileCoord{mi, (int)(local % tm_count), (int)(local / tm_count)};
 }
 
-// DA: activation dtype; DQ: double-quantized block scales.
-template <int DA, bool DQ>
+// Block-scale modes of the GEMM: absmax as stored (NF4, INT4 symmetric),
+// double-quantized (NF4), or scale plus zero-point (INT4 asymmetric).
+constexpr int kGemmPlain = 0, kGemmDq = 1, kGemmAsym = 2;
+
+// DA: activation dtype; MODE: block-scale mode.  The blocksize is a launch
+// parameter: it only decides which block scale a thread's 16 codes take.
+template <int DA, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  constexpr bool DQ = MODE == kGemmDq, ASYM = MODE == kGemmAsym;
   pdl_launch_then_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -247,6 +256,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ float s_lv[16 * 32];
+  __shared__ __align__(16) uint8_t s_z[ASYM ? kGemmBN * 16 : 4];  // zero-points of each row's window
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t bar0 = smem_u32(bars);
@@ -418,31 +428,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const TileCoord tc = gemm_tile(p, t);
       const GemmMat &m = p.mat[tc.mi];
       const int nk = m.K / kGemmBK;
+      const int lbs = p.log2_bs;
+      const int nblk = m.K >> lbs;  // blocks per weight row
       const int row = tc.tn * kGemmBN + d;
       const bool row_ok = row < m.N;
       const float mu = (DQ && row_ok) ? __ldg(m.absmax_mean) : 0.0f;
-      const int64_t bi0 = (int64_t)min(row, m.N - 1) * nk;
-      // block scales: the c~ of 16 blocks of the row at a time, computed by
-      // the row's threads (parts of four blocks) from inputs requested 16
-      // blocks ahead, kept in shared memory for the row
+      const int64_t bi0 = (int64_t)min(row, m.N - 1) * nblk;
+      // block scales: the c~ (and zero-points) of a window of 16 blocks of
+      // the row at a time, computed by the row's four threads (four blocks
+      // each) from inputs requested a window ahead, kept in shared memory
+      // for the row
       struct In4 {
-        uint32_t cw;     // int8 codes of four blocks (double quant)
+        uint32_t cw;     // int8 codes of four blocks (double quant) / their zero-points (asymmetric)
         float s2a, s2b;  // second-level scales of their (at most two) 256-groups
         int bsplit;
         float f[4];      // fp32 absmax (no double quant)
       };
-      constexpr int kParts = 4 / kGemmTpr;  // parts of four blocks per thread
-      auto load4 = [&](int kb0, int j, In4 &o) {  // blocks kb0 + 4 j .. + 3
-        const int b0 = kb0 + 4 * j;
-        const int nv = max(0, min(4, nk - b0));
+      auto load4 = [&](int b0, In4 &o) {  // blocks b0 .. b0 + 3 of the row
+        const int nv = max(0, min(4, nblk - b0));
         const int64_t bi = bi0 + b0;
-        if (nv == 0) {
-          o.cw = 0;
-          o.s2a = o.s2b = 0.0f;
-          o.bsplit = 4;
-          o.f[0] = o.f[1] = o.f[2] = o.f[3] = 0.0f;
-          return;
-        }
+        o.cw = 0;
+        o.s2a = o.s2b = 0.0f;
+        o.bsplit = 4;
+        o.f[0] = o.f[1] = o.f[2] = o.f[3] = 0.0f;
+        if (nv == 0) return;
         if constexpr (DQ) {
           o.s2a = __ldg(m.absmax_scale + (bi >> 8));
           o.s2b = __ldg(m.absmax_scale + ((bi + nv - 1) >> 8));
@@ -459,10 +468,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         } else {
 #pragma unroll
           for (int e = 0; e < 4; ++e) o.f[e] = e < nv ? __ldg(m.absmax + bi + e) : 0.0f;
+          if constexpr (ASYM) {
+            uint32_t w = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (e < nv) w |= ((uint32_t)(__ldg(m.zero + ((bi + e) >> 1)) >> (((bi + e) & 1) * 4)) & 15u) << (8 * e);
+            o.cw = w;
+          }
         }
       };
       float *scrow = sSc + d * 16;
-      auto store4 = [&](int j, const In4 &o) {
+      uint8_t *zrow = s_z + (ASYM ? d * 16 : 0);
+      auto store4 = [&](const In4 &o) {  // this thread's four blocks of the window
         float v[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -474,35 +491,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           }
           if (!row_ok) v[e] = 0.0f;
         }
-        *reinterpret_cast<float4 *>(scrow + 4 * j) = make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4 *>(scrow + 4 * qk) = make_float4(v[0], v[1], v[2], v[3]);
+        if constexpr (ASYM) *reinterpret_cast<uint32_t *>(zrow + 4 * qk) = o.cw;
       };
-      In4 nin[kParts];
+      In4 nin;
       {
-        In4 cin[kParts];
-#pragma unroll
-        for (int j = 0; j < kParts; ++j) {
-          load4(0, qk * kParts + j, cin[j]);
-          if (nk > 16) load4(16, qk * kParts + j, nin[j]);
-        }
+        In4 cin;
+        load4(4 * qk, cin);
+        load4(16 + 4 * qk, nin);  // zeros past the row's end
         __syncwarp();  // the row's previous c~ have been read
-#pragma unroll
-        for (int j = 0; j < kParts; ++j) store4(qk * kParts + j, cin[j]);
+        store4(cin);
         __syncwarp();
       }
+      int wnext = 16;  // first block of the window held in nin
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % kGemmStages;
         const uint32_t use = it / kGemmStages;
-        if ((kb & 15) == 0 && kb > 0) {
-          __syncwarp();  // the row's c~ of the previous 16 blocks have been read
-#pragma unroll
-          for (int j = 0; j < kParts; ++j) store4(qk * kParts + j, nin[j]);
+        const int kk = kb * kGemmBK;
+        if (kb > 0 && (kk & ((16 << lbs) - 1)) == 0) {
+          // a new window of 16 blocks starts at this k-block
+          __syncwarp();  // the row's c~ of the previous window have been read
+          store4(nin);
           __syncwarp();
-#pragma unroll
-          for (int j = 0; j < kParts; ++j)
-            if (kb + 16 < nk) load4(kb + 16, qk * kParts + j, nin[j]);
+          wnext += 16;
+          load4(wnext + 4 * qk, nin);
         }
-        const float sc = scrow[kb & 15];
+        const int blk = ((kk + kGemmCodes * qk) >> lbs) & 15;  // this thread's block in the window
+        const float sc = scrow[blk];
+        const float zf = ASYM ? (float)zrow[blk] : 0.0f;
         // lane 0 waits for the copy (acquire); the shuffle keeps the other
         // lanes' reads of the stage after it
         {
@@ -535,8 +552,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             // level table: entry e of this lane at lvb + e * 128
-            const float l0 = lds_f32((__byte_perm(lo, 0u, 0x4440u | j) << 7) + lvb);
-            const float l1 = lds_f32((__byte_perm(hi, 0u, 0x4440u | j) << 7) + lvb);
+            float l0 = lds_f32((__byte_perm(lo, 0u, 0x4440u | j) << 7) + lvb);
+            float l1 = lds_f32((__byte_perm(hi, 0u, 0x4440u | j) << 7) + lvb);
+            if constexpr (ASYM) l0 = __fsub_rn(l0, zf), l1 = __fsub_rn(l1, zf);  // q - z, exact
             o[j] = Dt<DA>::pack2(__fmul_rn(sc, l0), __fmul_rn(sc, l1));
           }
           const int c = (kGemmCodes / 8) * qk + c2;

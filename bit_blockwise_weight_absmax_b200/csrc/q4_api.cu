@@ -713,17 +713,24 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
   int rc = Q4_OK;
   int64_t tiles = 0;
   int dq = -1;
-  for (int i = 0; i < count && rc == Q4_OK; ++i) {
+  // every matrix's format and shape first (host only), then the device
+  for (int i = 0; i < count; ++i) {
     const q4_state *s = Wq[i];
     rc = check_state(s);
-    if (rc != Q4_OK) break;
-    if (s->qtype != Q4_NF4 || s->blocksize != 64) { rc = Q4_ERR_ARG; break; }
-    if (dq < 0) dq = s->double_quant;
-    if (s->double_quant != dq) { rc = Q4_ERR_ARG; break; }
-    if (s->cols % 64 || s->rows % 16 || s->rows > INT32_MAX || s->cols > INT32_MAX) { rc = Q4_ERR_SHAPE; break; }
-    if (!A[i] || !Y[i]) { rc = Q4_ERR_ARG; break; }
-    if (!aligned16(A[i]) || !aligned16(Y[i])) { rc = Q4_ERR_ALIGN; break; }
-    if (di.ok != Q4_OK) { rc = di.ok; break; }
+    if (rc != Q4_OK) return rc;
+    // one format per grouped call
+    if (s->qtype != Wq[0]->qtype || s->blocksize != Wq[0]->blocksize ||
+        s->double_quant != Wq[0]->double_quant)
+      return Q4_ERR_ARG;
+    // whole 64-k blocks of whole quantization blocks
+    if (s->cols % 64 || s->cols % s->blocksize || s->rows % 16 || s->rows > INT32_MAX || s->cols > INT32_MAX)
+      return Q4_ERR_SHAPE;
+    if (!aligned16(A[i]) || !aligned16(Y[i])) return Q4_ERR_ALIGN;
+  }
+  if (di.ok != Q4_OK) return di.ok;
+  dq = Wq[0]->double_quant;
+  for (int i = 0; i < count && rc == Q4_OK; ++i) {
+    const q4_state *s = Wq[i];
     GemmMat &m = p.mat[i];
     const CUtensorMapDataType adt = a_dtype == Q4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     if (!make_map(&m.tmA, adt, A[i], M, s->cols, 2, kGemmBK, kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -736,6 +743,7 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     m.absmax_scale = s->absmax_scale;
     m.absmax_mean = s->absmax_mean;
     m.absmax = s->absmax;
+    m.zero = s->zero;
     m.Y = Y[i];
     m.M = (int32_t)M;
     m.N = (int32_t)s->rows;
@@ -751,10 +759,20 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     p.dq = dq;
     p.total_tiles = tiles;
     p.status = di.status;
-    memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+    const int qt = Wq[0]->qtype;
+    int mode = dq ? kGemmDq : kGemmPlain;
+    if (qt == Q4_NF4) {
+      memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
+    } else if (qt == Q4_INT4_SYM) {
+      for (int j = 0; j < 16; ++j) p.levels[j] = (float)((j ^ 8) - 8);  // two's-complement nibble q: w^ = q s
+    } else {
+      for (int j = 0; j < 16; ++j) p.levels[j] = (float)j;  // w^ = (q - z) s
+      mode = kGemmAsym;
+    }
+    p.log2_bs = __builtin_ctz((unsigned)Wq[0]->blocksize);
     p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
-    rc = run_gemm(a_dtype, p, di.sms, (cudaStream_t)stream);
+    rc = run_gemm(a_dtype, mode, p, di.sms, (cudaStream_t)stream);
   }
   return rc;
 }

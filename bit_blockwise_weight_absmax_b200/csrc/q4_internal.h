@@ -64,7 +64,7 @@ int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t 
 int run_quantize_grouped(int dt, int qt, int bs, bool dq, const QuantGroupParams &p, int grid, cudaStream_t st);
 int run_double_quant_grouped(const DqGroupParams &p, cudaStream_t st);
 int run_dequantize(int qt, int dout, int bs, bool dq, const DequantGroupParams &p, int sms, cudaStream_t st);
-int run_gemm(int da, const GemmParams &p, int sms, cudaStream_t st);
+int run_gemm(int da, int mode, const GemmParams &p, int sms, cudaStream_t st);
 int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st);
 int run_gemv(int da, int mode, int nt, int bs, const GvParams &p, int grid, cudaStream_t st);
 int gv_tile_rows(int nt);

@@ -8,9 +8,9 @@ goes": a 4-bit linear layer keeps its weight quantized and dequantizes it to
 the compute dtype for the matmul; the output head and the normalisation
 layers stay in 16 bits.  Here the dequantization is fused into the kernels:
 up to 32 rows of activations run the decode GEMV, more rows the W4A16
-tcgen05 GEMM (NF4, blocksize 64, N % 16 == 0), other formats run the GEMV
-32 rows at a time.  A format neither consumer takes is refused when the
-module is built.  All compute is on the GPU; there is no CPU path.
+tcgen05 GEMM (every format and blocksize; N % 16 == 0 and K % 64 == 0),
+other shapes run the GEMV 32 rows at a time.  A format neither consumer
+takes is refused when the module is built.  All compute is on the GPU; there is no CPU path.
 """
 from __future__ import annotations
 
@@ -60,8 +60,7 @@ class Linear4bit(torch.nn.Module):
 
     def _gemm_ok(self) -> bool:
         st = self.state
-        return (st.qtype == q4.NF4 and st.blocksize == 64 and st.rows % 16 == 0
-                and st.cols % 64 == 0)
+        return st.rows % 16 == 0 and st.cols % 64 == 0 and st.cols % st.blocksize == 0
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         if x.shape[-1] != self.in_features:

@@ -268,9 +268,15 @@ Q4_API int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *
  * weight tiles into shared memory (bit-exact w^ in a_dtype) and feeding
  * tcgen05 tensor-core MMAs with fp32 accumulators in tensor memory.
  *   A   device, a_dtype (Q4_BF16 / Q4_F16), [M, K] row-major, 16-byte aligned.
- *   Wq  NF4 state, blocksize 64, K % 64 == 0, N % 16 == 0.
+ *   Wq  any state (NF4 with or without double quantization, INT4
+ *       symmetric, INT4 asymmetric; blocksize 32, 64, 128 or 256) with
+ *       K % 64 == 0 (and K a multiple of the blocksize), N % 16 == 0.
+ *       The weight tile is w^ = cvt(c~ * level) for NF4, cvt(s * q) for
+ *       INT4 symmetric and cvt(s * (q - z)) for INT4 asymmetric: bit for
+ *       bit what q4_dequantize gives.
  *   Y   device, y_dtype (a_dtype or Q4_F32), [M, N] row-major.
- * Same tolerance as q4_gemv.
+ * Same tolerance as q4_gemv.  A grouped call takes one format (qtype,
+ * blocksize, double_quant) for all its matrices (Q4_ERR_ARG otherwise).
  */
 Q4_API int q4_gemm(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
             int32_t y_dtype, void *stream);

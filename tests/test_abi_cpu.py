@@ -221,6 +221,30 @@ def test_gemv_host_checks_before_the_device(lib):
     assert _gemv(lib, [_fake_state(0, 256, 96, 64, False)], 1) == -2
 
 
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
+def test_gemm_host_checks_before_the_device(lib):
+    """The GEMM takes every format and blocksize: each passes the host checks
+    and stops at the missing GPU; a grouped call of mixed formats or
+    blocksizes is Q4_ERR_ARG; K not a multiple of 64 or of the blocksize,
+    or N not a multiple of 16, is a shape error."""
+    from bit_blockwise_weight_absmax_b200 import q4
+    P = ctypes.POINTER(q4._CState)
+
+    def gemm(states, M=512):
+        n = len(states)
+        arr = (P * n)(*[ctypes.pointer(st) for st in states])
+        ptrs = (ctypes.c_void_p * n)(*([0x70000] * n))
+        return lib.q4_gemm_grouped(n, ptrs, arr, ptrs, M, 1, 1, None)
+    for qt, dq in ((0, False), (0, True), (1, False), (2, False)):
+        for bs in (32, 64, 128, 256):
+            assert gemm([_fake_state(qt, 256, 1024, bs, dq)]) == -4  # Q4_ERR_NO_DEVICE
+    assert gemm([_fake_state(0, 256, 1024, 64, True), _fake_state(1, 256, 1024, 64, False)]) == -1
+    assert gemm([_fake_state(1, 256, 1024, 64, False), _fake_state(1, 256, 1024, 128, False)]) == -1
+    assert gemm([_fake_state(1, 256, 96, 32, False)]) == -2      # K % 64
+    assert gemm([_fake_state(1, 256, 384, 256, False)]) == -2    # K % B
+    assert gemm([_fake_state(2, 250, 1024, 128, False)]) == -2   # N % 16
+
+
 def test_grouped_calls_reject_a_null_entry_before_any_use(lib):
     """A NULL state, activation or output pointer in any entry of a grouped
     call is Q4_ERR_ARG, found before the library reads any entry (a NULL

@@ -103,3 +103,48 @@ def test_gemm_prefill_7b_layer_large_m(q4, oracle, M):
         ref = oracle.matmul(a16, True, w16, True, len(toks), len(rows), K)
         sub = y[torch.from_numpy(toks).cuda()][:, torch.from_numpy(rows).cuda()]
         assert_matmul_close(sub, ref)
+
+
+@pytest.mark.parametrize("qtype,dq", [("nf4", False), ("nf4", True), ("int4_sym", False), ("int4_asym", False)])
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+def test_gemm_formats_and_blocksizes(q4, oracle, qtype, dq, bs):
+    """Every state format the quantizer makes, at every blocksize: ragged M
+    and N (a partial 256-row and 128-column tile), K = 4608 so that the
+    row's window of 16 block scales turns over (144 blocks at B = 32, 18 at
+    B = 256); against the oracle's binary64 product of its dequantized
+    weights (w^ exactly as q4_dequantize gives it)."""
+    QT = {"nf4": 0, "int4_sym": 1, "int4_asym": 2}[qtype]
+    g = torch.Generator().manual_seed(bs + 7 * QT)
+    M, N, K = 300, 272, 4608
+    W = torch.randn(N, K, generator=g).mul(0.02)
+    W.view(-1)[::701] *= 15  # outliers: wide block ranges
+    W = W.bfloat16()
+    A = torch.randn(M, K, generator=g).bfloat16()
+    st = q4.quantize(W.cuda(), bs, qtype, dq)
+    ost = oracle_state(oracle, W, bs, QT, dq)
+    y = q4.gemm(A.cuda(), st)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    w16 = oracle.dequantize(ost, True).reshape(N, K)
+    ref = oracle.matmul(bits(A), True, w16, True, M, N, K)
+    assert_matmul_close(y, ref)
+
+
+def test_gemm_grouped_int4_asym_layer(q4, oracle):
+    """One grouped launch over the 7B layer's shapes in INT4 asymmetric
+    group-128 (the format the decode GEMV also takes), M = 512; sampled
+    output columns against the oracle."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    Ws = wl.layer_weights(wl.LAYER_7B, 0.02, seed=320)
+    sts = [q4.quantize(W.cuda(), 128, "int4_asym", False) for W in Ws]
+    rng = np.random.default_rng(3)
+    M = 512
+    As = [wl.activation(M, K, torch.bfloat16, seed=420 + i) for i, (_, N, K) in enumerate(wl.LAYER_7B)]
+    ys = q4.gemm_grouped([a.cuda() for a in As], sts)
+    torch.cuda.synchronize()
+    for W, (name, N, K), a, y in zip(Ws, wl.LAYER_7B, As, ys):
+        ost = oracle_state(oracle, W, 128, 2, False)
+        rows = np.sort(rng.choice(N, 64, replace=False))
+        w16 = oracle.dequantize(ost, True).reshape(N, K)[rows]
+        ref = oracle.matmul(bits(a), True, w16, True, M, len(rows), K)
+        assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
