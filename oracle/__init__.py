@@ -66,6 +66,8 @@ def lib():
         i64, i32 = ctypes.c_int64, ctypes.c_int
         _lib.oracle_quantize.argtypes = [P, i32, i64, i32, i32, i32, P, P, P, P, P, P]
         _lib.oracle_quantize.restype = None
+        _lib.oracle_quantize_s.argtypes = [P, i32, i64, i32, i32, i32, i32, P, P, P, P, P, P]
+        _lib.oracle_quantize_s.restype = None
         _lib.oracle_dequantize.argtypes = [P, P, P, P, P, P, i64, i32, i32, i32, i32, P]
         _lib.oracle_dequantize.restype = None
         _lib.oracle_dequantize_f32.argtypes = [P, P, P, P, P, P, i64, i32, i32, i32, P]
@@ -126,6 +128,11 @@ class State:
     absmax_q: np.ndarray | None    # int8 [nb] (double_quant)
     absmax_scale: np.ndarray | None  # float32 [ceil(nb/256)]
     absmax_mean: np.ndarray | None   # float32 [1]
+    scale_f16: int = 0               # INT4: the scale is a binary16 value (absmax holds it as fp32)
+
+    def scale_f16_bits(self) -> np.ndarray:
+        """The stored binary16 scales (uint16 [nb]) of a scale_f16 state."""
+        return np.array([lib().oracle_float_to_half(float(v)) for v in self.absmax], dtype=np.uint16)
 
     @property
     def nb(self) -> int:
@@ -140,8 +147,9 @@ class State:
 
 
 def quantize(w_bits: np.ndarray, is_bf16: bool, blocksize: int, qtype: int,
-             double_quant: bool = False) -> State:
-    """Quantize n 16-bit floats given as raw uint16 bit patterns (flattened)."""
+             double_quant: bool = False, scale_f16: bool = False) -> State:
+    """Quantize n 16-bit floats given as raw uint16 bit patterns (flattened).
+    scale_f16 (INT4 only): binary16 scales, codes against the rounded scale."""
     w = np.ascontiguousarray(w_bits.reshape(-1).view(np.uint16))
     n = w.size
     nb = (n + blocksize - 1) // blocksize
@@ -153,11 +161,12 @@ def quantize(w_bits: np.ndarray, is_bf16: bool, blocksize: int, qtype: int,
     absmax_q = np.zeros(nb, dtype=np.int8) if dq else None
     absmax_scale = np.zeros(ng, dtype=np.float32) if dq else None
     absmax_mean = np.zeros(1, dtype=np.float32) if dq else None
-    lib().oracle_quantize(_ptr(w), int(is_bf16), n, blocksize, qtype, int(dq), _ptr(packed),
-                          _ptr(absmax), _ptr(zero), _ptr(absmax_q), _ptr(absmax_scale),
-                          _ptr(absmax_mean))
+    sf = int(bool(scale_f16) and qtype != QT_NF4)
+    lib().oracle_quantize_s(_ptr(w), int(is_bf16), n, blocksize, qtype, int(dq), sf, _ptr(packed),
+                            _ptr(absmax), _ptr(zero), _ptr(absmax_q), _ptr(absmax_scale),
+                            _ptr(absmax_mean))
     return State(qtype, n, blocksize, int(dq), packed, absmax, zero, absmax_q, absmax_scale,
-                 absmax_mean)
+                 absmax_mean, sf)
 
 
 def dequantize(st: State, out_bf16: bool) -> np.ndarray:
@@ -218,18 +227,19 @@ def float_to_bf16(f: float) -> int:
 
 
 def storage_bits_per_param(qtype: int, blocksize: int, double_quant: bool,
-                           n: int | None = None) -> float:
+                           n: int | None = None, scale_f16: bool = False) -> float:
     """Bits per parameter of the resident format (codes + block state).
 
     Asymptotic (n None): 4 + per-block state / blocksize.  NF4 without double
     quantization keeps one fp32 absmax per block (learn.pranaymahendrakar.com,
     "Block-wise quantisation, stated exactly": 32/64 = 0.5 bits); with it,
     one int8 per block plus one fp32 scale per 256 blocks and one fp32 mean.
+    INT4 with scale_f16 keeps one binary16 scale per block.
     """
     if n is None:
         if qtype == QT_NF4 and double_quant:
             return 4.0 + 8.0 / blocksize + 32.0 / (blocksize * DQ_GROUP)
-        extra = 32.0 / blocksize
+        extra = (16.0 if scale_f16 else 32.0) / blocksize
         if qtype == QT_INT4_ASYM:
             extra += 4.0 / blocksize
         return 4.0 + extra
@@ -238,7 +248,7 @@ def storage_bits_per_param(qtype: int, blocksize: int, double_quant: bool,
     if qtype == QT_NF4 and double_quant:
         bits += 8 * nb + 32 * ((nb + DQ_GROUP - 1) // DQ_GROUP) + 32
     else:
-        bits += 32 * nb
+        bits += (16 if scale_f16 else 32) * nb
         if qtype == QT_INT4_ASYM:
             bits += 8 * ((nb + 1) // 2)
     return bits / n

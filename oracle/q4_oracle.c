@@ -195,6 +195,10 @@ double oracle_pairwise_sum(double *v, int64_t n) {
  *            max(max w, 0); s = (mx - mn) / 15; z = clamp(rint(-mn / s), 0,
  *            15); q = clamp(rint(w / s) + z, 0, 15); absmax[b] = s and the
  *            zero-point nibble b of `zero` = z.
+ *  scale_f16 (INT4 only, [INT4] "Components": the per-group scale is
+ *            "usually stored in FP16"): s is rounded to binary16 (IEEE,
+ *            ties to even) as soon as it is formed, and z and every q are
+ *            computed against that rounded s; absmax[b] holds its value.
  *  double_quant (NF4 only, [BWQ] "quantises the per-block scales
  *            themselves (blocks of 256, to 8 bits)"): mu = fp32(S / nb) with
  *            S the pairwise fp64 sum of all c; per group g of 256 blocks:
@@ -205,9 +209,9 @@ double oracle_pairwise_sum(double *v, int64_t n) {
  * Outputs must be sized by the caller; packed must hold ceil(n/2) bytes and
  * is fully written (an odd n leaves the final high nibble 0).
  */
-void oracle_quantize(const uint16_t *w, int is_bf16, int64_t n, int blocksize, int qtype,
-                     int double_quant, uint8_t *packed, float *absmax, uint8_t *zero,
-                     int8_t *absmax_q, float *absmax_scale, float *absmax_mean) {
+void oracle_quantize_s(const uint16_t *w, int is_bf16, int64_t n, int blocksize, int qtype,
+                       int double_quant, int scale_f16, uint8_t *packed, float *absmax, uint8_t *zero,
+                       int8_t *absmax_q, float *absmax_scale, float *absmax_mean) {
   int64_t nb = (n + blocksize - 1) / blocksize;
   memset(packed, 0, (size_t)((n + 1) / 2));
   if (qtype == QT_INT4_ASYM) memset(zero, 0, (size_t)((nb + 1) / 2));
@@ -235,6 +239,7 @@ void oracle_quantize(const uint16_t *w, int is_bf16, int64_t n, int blocksize, i
         if (a > c) c = a;
       }
       float s = c / 7.0f;
+      if (scale_f16) s = oracle_half_to_float(oracle_float_to_half(s));
       absmax[b] = s;
       for (int64_t j = lo; j < hi; j++) {
         int q = 0;
@@ -249,6 +254,7 @@ void oracle_quantize(const uint16_t *w, int is_bf16, int64_t n, int blocksize, i
         if (v > mx) mx = v;
       }
       float s = (mx - mn) / 15.0f;
+      if (scale_f16) s = oracle_half_to_float(oracle_float_to_half(s));
       int z = 0;
       if (s != 0.0f) z = clampi((int)rintf(-mn / s), 0, 15);
       absmax[b] = s;
@@ -294,6 +300,14 @@ void oracle_quantize(const uint16_t *w, int is_bf16, int64_t n, int blocksize, i
       }
     }
   }
+}
+
+/* oracle_quantize_s with binary32 scales. */
+void oracle_quantize(const uint16_t *w, int is_bf16, int64_t n, int blocksize, int qtype,
+                     int double_quant, uint8_t *packed, float *absmax, uint8_t *zero,
+                     int8_t *absmax_q, float *absmax_scale, float *absmax_mean) {
+  oracle_quantize_s(w, is_bf16, n, blocksize, qtype, double_quant, 0, packed, absmax, zero, absmax_q,
+                    absmax_scale, absmax_mean);
 }
 
 /* ------------------------------------------------------------------------ */

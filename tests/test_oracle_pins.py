@@ -468,9 +468,22 @@ def _rne32(x: Fraction) -> Fraction:
     return (r * quantum) if x > 0 else -(r * quantum)
 
 
-def int4_asym_pin_failures(wf: np.ndarray, st) -> list:
+def _keep(x: Fraction) -> Fraction:
+    return x
+
+
+def _to_half(x: Fraction) -> Fraction:
+    """The binary16 value nearest to the binary32 value x (numpy's IEEE
+    conversion, ties to even, overflow to infinity)."""
+    h = np.float16(float(x))
+    return Fraction(float(h)) if np.isfinite(h) else h
+
+
+def int4_asym_pin_failures(wf: np.ndarray, st, scale_round=_keep) -> list:
     """Every closed-form check that the state of INT4 asymmetric groups
-    (rows of `wf`, the exact binary32 values of the 16-bit inputs) fails."""
+    (rows of `wf`, the exact binary32 values of the 16-bit inputs) fails.
+    scale_round: the storage rounding of s (binary16 scales: codes and
+    zero-points are formed against the rounded s)."""
     nb, B = wf.shape
     z = np.stack([st.zero & 0xF, st.zero >> 4], -1).reshape(-1)[:nb].astype(np.int64)
     q = st.codes().astype(np.int64).reshape(nb, B)
@@ -478,7 +491,11 @@ def int4_asym_pin_failures(wf: np.ndarray, st) -> list:
     for b in range(nb):
         vals = [Fraction(float(v)) for v in wf[b]]
         mn, mx = min(min(vals), Fraction(0)), max(max(vals), Fraction(0))
-        s = _rne32(_rne32(mx - mn) / 15)
+        s = scale_round(_rne32(_rne32(mx - mn) / 15))
+        if not isinstance(s, Fraction):  # binary16 overflow: every quotient is 0
+            if not np.isinf(st.absmax[b]) or z[b] != 0 or np.any(q[b] != 0):
+                bad.append(("inf-scale", b))
+            continue
         if Fraction(float(st.absmax[b])) != s:
             bad.append(("scale", b))
             continue
@@ -491,8 +508,11 @@ def int4_asym_pin_failures(wf: np.ndarray, st) -> list:
             bad.append(("zero-point", b))
             continue
         # the dequantized ends of the level range sit within s/2 (plus the
-        # binary32 roundings of s) of the widened group minimum and maximum
+        # binary32 roundings of s) of the widened group minimum and maximum;
+        # a binary16 s may be off by half its ulp, 15 times over
         slack = s / 2 + abs(mx - mn) * Fraction(1, 2 ** 22)
+        if scale_round is not _keep:
+            slack += 15 * s / 2 ** 11 + Fraction(15, 2 ** 25)
         if abs(-zz * s - mn) > slack or abs((15 - zz) * s - mx) > slack:
             bad.append(("endpoints", b))
         for j in range(B):
@@ -576,3 +596,124 @@ def test_int4_asym_pins_catch_planted_mistakes(oracle, tmp_path, old, new):
     lib.oracle_quantize(p(bits), 0, n, B, oracle.QT_INT4_ASYM, 0, p(st.packed), p(st.absmax),
                         p(st.zero), None, None, None)
     assert int4_asym_pin_failures(w.float().numpy(), st) != []
+
+
+
+# ---------------------------------------------------------------- fp16 scales --
+# robotsatlas.com, "INT4", "Components": the per-group scale is usually stored
+# in FP16.  Reading: s is rounded to binary16 when formed and the codes (and
+# the zero-point) are computed against the rounded s.
+
+def test_oracle_binary16_rounding_is_ieee(oracle):
+    """The oracle's own binary32 -> binary16 conversion (written from the
+    format's definition) equals numpy's IEEE conversion on random patterns
+    over the whole binary32 range and on the cases that decide rounding:
+    exact halfway points between neighbouring binary16 values (both
+    parities), the subnormal range, and the overflow threshold."""
+    rng = np.random.default_rng(12)
+    f = rng.integers(0, 2 ** 32, 60000, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    f = f[np.isfinite(f)]
+    h = np.arange(0, 0x7C00, 37, dtype=np.uint16).view(np.float16).astype(np.float64)
+    halves = (h[:-1] + h[1:]) / 2  # exact in binary32 for these magnitudes
+    edge = np.array([65504.0, 65519.99, 65520.0, 65536.0, 2.0 ** -24, 2.0 ** -25, 2.0 ** -25 * 1.5,
+                     2.0 ** -26, 6.1e-5, 6.097555e-05, 1e-8, 0.0], dtype=np.float64)
+    vals = np.concatenate([f.astype(np.float64), halves, edge, -halves, -edge]).astype(np.float32)
+    want = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.float_to_half(float(v)) for v in vals], dtype=np.uint16)
+    assert np.array_equal(got, want)
+
+
+def int4_sym_pin_failures(wf: np.ndarray, st, scale_round=_keep) -> list:
+    """Closed-form checks of INT4 symmetric groups: s = round(fl32(c / 7)),
+    q = clamp(rint(fl32(w / s)), -8, 7) as a two's-complement nibble."""
+    nb, B = wf.shape
+    q = st.codes().astype(np.int64).reshape(nb, B)
+    bad = []
+    for b in range(nb):
+        vals = [Fraction(float(v)) for v in wf[b]]
+        c = max(abs(v) for v in vals)
+        s = scale_round(_rne32(c / 7))
+        if not isinstance(s, Fraction):
+            if not np.isinf(st.absmax[b]) or np.any(q[b] != 0):
+                bad.append(("inf-scale", b))
+            continue
+        if Fraction(float(st.absmax[b])) != s:
+            bad.append(("scale", b))
+            continue
+        for j in range(B):
+            qq = 0 if s == 0 else min(max(round(_rne32(vals[j] / s)), -8), 7)
+            if q[b, j] != (qq & 15):
+                bad.append(("code", b, j))
+                break
+    return bad
+
+
+def _fp16_scale_groups(dt, seed):
+    """_asym_groups plus groups whose scale leaves the binary16 range: tiny
+    ones (s rounds to a subnormal or to 0) and, for bf16, huge ones (s
+    overflows to infinity)."""
+    w, B = _asym_groups(dt, seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    extra = [torch.randn(B, generator=g) * 1e-6, torch.randn(B, generator=g) * 3e-8]
+    if dt == torch.bfloat16:
+        extra += [torch.randn(B, generator=g) * 1e6]
+    return torch.cat([w, torch.stack(extra).to(dt)]), B
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_int4_fp16_scale_closed_forms(oracle, dt):
+    """With binary16 scales, every group's stored scale is the binary16
+    rounding of the binary32 rule, and its codes (and zero-point) are the
+    closed forms computed against that rounded scale; the stored patterns
+    are the binary16 of the stored values."""
+    w, B = _fp16_scale_groups(dt, 37)
+    bits = w.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    wf = w.float().numpy()
+    sym = oracle.quantize(bits, dt == torch.bfloat16, B, oracle.QT_INT4_SYM, scale_f16=True)
+    assert int4_sym_pin_failures(wf, sym, _to_half) == []
+    asym = oracle.quantize(bits, dt == torch.bfloat16, B, oracle.QT_INT4_ASYM, scale_f16=True)
+    assert int4_asym_pin_failures(wf, asym, _to_half) == []
+    for st in (sym, asym):
+        assert np.array_equal(st.scale_f16_bits(), st.absmax.astype(np.float16).view(np.uint16))
+    # and the binary32 pins still hold without the option
+    assert int4_sym_pin_failures(wf, oracle.quantize(bits, dt == torch.bfloat16, B, oracle.QT_INT4_SYM)) == []
+
+
+@pytest.mark.parametrize("old,new", [
+    # codes against the unrounded s, only the stored scale rounded
+    ("      if (scale_f16) s = oracle_half_to_float(oracle_float_to_half(s));\n      absmax[b] = s;",
+     "      absmax[b] = scale_f16 ? oracle_half_to_float(oracle_float_to_half(s)) : s;"),
+    # the option ignored in the asymmetric rule
+    ("      if (scale_f16) s = oracle_half_to_float(oracle_float_to_half(s));\n      int z = 0;",
+     "      int z = 0;"),
+])
+def test_fp16_scale_pins_catch_planted_mistakes(oracle, tmp_path, old, new):
+    """A planted slip in the binary16-scale rule fails the closed-form pins."""
+    import ctypes
+    import subprocess
+    src = open(os.path.join(os.path.dirname(oracle_module_file()), "q4_oracle.c")).read()
+    assert src.count(old) == 1, old
+    path = tmp_path / "mut.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "mut.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", str(path),
+                    "-o", str(so), "-lm"], check=True, capture_output=True)
+    lib = ctypes.CDLL(str(so))
+    P = ctypes.c_void_p
+    lib.oracle_quantize_s.argtypes = [P, ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, P, P, P, P, P, P]
+    lib.oracle_quantize_s.restype = None
+    w, B = _fp16_scale_groups(torch.float16, 37)
+    bits = np.ascontiguousarray(w.view(torch.int16).numpy().view(np.uint16).reshape(-1))
+    n = bits.size
+    nb = n // B
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    fails = 0
+    for qt in (oracle.QT_INT4_SYM, oracle.QT_INT4_ASYM):
+        st = oracle.State(qt, n, B, 0, np.zeros(n // 2, np.uint8), np.zeros(nb, np.float32),
+                          np.zeros((nb + 1) // 2, np.uint8), None, None, None, 1)
+        lib.oracle_quantize_s(p(bits), 0, n, B, qt, 0, 1, p(st.packed), p(st.absmax), p(st.zero), None,
+                              None, None)
+        pin = int4_sym_pin_failures if qt == oracle.QT_INT4_SYM else int4_asym_pin_failures
+        fails += len(pin(w.float().numpy(), st, _to_half))
+    assert fails > 0
