@@ -53,6 +53,7 @@ constexpr int kDqMaxGroup = 16;
 struct DequantGroupParams {
   DqGMat mat[kDqMaxGroup];
   int32_t count;
+  int32_t scale_f16;  // INT4: binary16 scales
   int64_t total_spans;
   float levels[16];
 };
@@ -67,7 +68,7 @@ struct DqRaw {
 // Raw inputs of the span starting at element `base` of matrix m; WHOLE: the
 // span lies inside the matrix (no bounds checks).
 template <int QT, int B, bool DQ, bool WHOLE>
-__device__ __forceinline__ void dq_load(const DqGMat &m, int64_t base, int lane, DqRaw &r) {
+__device__ __forceinline__ void dq_load(const DqGMat &m, int64_t base, int lane, bool sf16, DqRaw &r) {
   const int64_t n = m.n;
   const uint8_t *pk_base = m.packed + base / 2 + lane * 4;  // chunk u at + 128 u
   const int64_t b_base = base / B;
@@ -94,7 +95,7 @@ __device__ __forceinline__ void dq_load(const DqGMat &m, int64_t base, int lane,
       r.q[u] = __ldg(m.absmax_q + b);
       r.s[u] = __ldg(m.absmax_scale + b / Q4_DQ_GROUP);
     } else {
-      r.s[u] = __ldg(m.absmax + b);
+      r.s[u] = ld_scale(m.absmax, b, sf16);
       if (QT == Q4_INT4_ASYM) r.q[u] = __ldg(m.zero + (b >> 1)) >> ((b & 1) * 4);
     }
   }
@@ -173,11 +174,12 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequantize_kernel(const __grid_
   if (sp >= p.total_spans) return;
   int mi = 0;
   while (mi + 1 < p.count && sp >= p.mat[mi + 1].span_begin) ++mi;
+  const bool sf16 = p.scale_f16 != 0;
   auto load = [&](int k, int64_t s, DqRaw &r) {
     const DqGMat &m = p.mat[k];
     const int64_t base = (s - m.span_begin) * kDqSpan;
-    if (base + kDqSpan <= m.n) dq_load<QT, B, DQ, true>(m, base, lane, r);
-    else dq_load<QT, B, DQ, false>(m, base, lane, r);
+    if (base + kDqSpan <= m.n) dq_load<QT, B, DQ, true>(m, base, lane, sf16, r);
+    else dq_load<QT, B, DQ, false>(m, base, lane, sf16, r);
   };
   DqRaw cur;
   load(mi, sp, cur);

@@ -75,7 +75,7 @@ struct GemmParams {
   int32_t dq;
   int32_t stall_copies;  // test hook: the producer issues no copies
   int32_t log2_bs;       // blocksize B = 2^log2_bs (32 .. 256)
-  int32_t pad2;
+  int32_t scale_f16;     // INT4: binary16 scales
   int64_t total_tiles;
   uint64_t wait_ns;      // bound of every mbarrier wait
   int *status;
@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o.f[e] = e < nv ? __ldg(m.absmax + bi + e) : 0.0f;
+          for (int e = 0; e < 4; ++e) o.f[e] = e < nv ? ld_scale(m.absmax, bi + e, p.scale_f16 != 0) : 0.0f;
           if constexpr (ASYM) {
             uint32_t w = 0;
 #pragma unroll

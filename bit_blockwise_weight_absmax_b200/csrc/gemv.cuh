@@ -105,6 +105,7 @@ struct GvParams {
   int *status;
   uint64_t wait_ns;      // bound of every mbarrier wait
   int32_t stall_copies;  // test hook: issue no copies, so every stage wait runs out
+  int32_t scale_f16;     // INT4: binary16 scales
   float levels[16];      // the value of each 4-bit code (NF4 levels, or integers)
 };
 
@@ -411,7 +412,8 @@ template <> struct GvScaleIn<kGvAsym> {
 
 // Load the c~ inputs of row `row` (< N, else nothing), blocks b0 .. b0+7.
 template <int MODE>
-__device__ __forceinline__ void gv_scale_load(const GvInfo &mt, int B, int row, int b0, GvScaleIn<MODE> &in) {
+__device__ __forceinline__ void gv_scale_load(const GvInfo &mt, int B, int row, int b0, bool sf16,
+                                              GvScaleIn<MODE> &in) {
   const int nbk = mt.K / B;
   in.nvalid = (row < mt.N) ? max(0, min(8, nbk - b0)) : 0;
   if constexpr (MODE == kGvDq) {
@@ -443,15 +445,12 @@ __device__ __forceinline__ void gv_scale_load(const GvInfo &mt, int B, int row, 
     if constexpr (MODE == kGvAsym) in.z = 0;
     if (in.nvalid == 0) return;
     const int64_t bi0 = (int64_t)row * nbk + b0;
-    if (in.nvalid == 8 && ((uintptr_t)(mt.absmax + bi0) & 15u) == 0) {
-      const float4 x = __ldg(reinterpret_cast<const float4 *>(mt.absmax + bi0));
-      const float4 y = __ldg(reinterpret_cast<const float4 *>(mt.absmax + bi0) + 1);
-      in.f[0] = x.x; in.f[1] = x.y; in.f[2] = x.z; in.f[3] = x.w;
-      in.f[4] = y.x; in.f[5] = y.y; in.f[6] = y.z; in.f[7] = y.w;
+    if (in.nvalid == 8) {
+      ld_scales8(mt.absmax, bi0, sf16, in.f);
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j < in.nvalid) in.f[j] = __ldg(mt.absmax + bi0 + j);
+        if (j < in.nvalid) in.f[j] = ld_scale(mt.absmax, bi0 + j, sf16);
     }
     if constexpr (MODE == kGvAsym) {
 #pragma unroll
@@ -651,7 +650,7 @@ __global__ void __launch_bounds__((GvShape<NT>::WARPS + 1) * 32, 1) gemv_kernel(
     const int wb0 = (chunk / WC) * kGvWin + (lane >> 4) * 8;
 #pragma unroll
     for (int rt = 0; rt < R; ++rt)
-      gv_scale_load<MODE>(mt, B, tile * TR + wrow + rt * 16 + (lane & 15), wb0, sin[rt]);
+      gv_scale_load<MODE>(mt, B, tile * TR + wrow + rt * 16 + (lane & 15), wb0, p.scale_f16 != 0, sin[rt]);
   };
   // byte o of c~ buffer (row group rt, parity par): contiguous, or spread
   // over the table's 128-byte gaps

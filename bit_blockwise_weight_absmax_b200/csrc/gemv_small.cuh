@@ -108,6 +108,7 @@ struct GsParams {
   int *status;
   uint64_t wait_ns;  // bound of every mbarrier wait
   int32_t stall_copies;  // test hook: issue no copies, so every stage wait runs out
+  int32_t scale_f16;     // INT4: binary16 scales
   float levels[16];
 };
 
@@ -269,7 +270,7 @@ struct GsScaleIn {
 };
 
 template <int B>
-__device__ __forceinline__ void gs_scale_load(const GsInfo *info, bool dq, const GsUnit &u, int r0, int lane,
+__device__ __forceinline__ void gs_scale_load(const GsInfo *info, bool dq, bool sf16, const GsUnit &u, int r0, int lane,
                                               GsScaleIn &in) {
   constexpr int W = kGsWinBlocks * B / kGsStageK;
   const GsInfo &mt = info[u.mi];
@@ -303,15 +304,12 @@ __device__ __forceinline__ void gs_scale_load(const GsInfo *info, bool dq, const
       }
     }
   } else {
-    if (in.nvalid == 8 && (bi0 & 3) == 0) {
-      const float4 x = __ldg(reinterpret_cast<const float4 *>(mt.absmax + bi0));
-      const float4 y = __ldg(reinterpret_cast<const float4 *>(mt.absmax + bi0) + 1);
-      in.f[0] = x.x; in.f[1] = x.y; in.f[2] = x.z; in.f[3] = x.w;
-      in.f[4] = y.x; in.f[5] = y.y; in.f[6] = y.z; in.f[7] = y.w;
+    if (in.nvalid == 8) {
+      ld_scales8(mt.absmax, bi0, sf16, in.f);
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        if (j < in.nvalid) in.f[j] = __ldg(mt.absmax + bi0 + j);
+        if (j < in.nvalid) in.f[j] = ld_scale(mt.absmax, bi0 + j, sf16);
     }
   }
 }
@@ -404,6 +402,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   const uint32_t g0 = gs_range_begin(blockIdx.x, T, G);  // this CTA's stages [g0, g1)
   const uint32_t g1 = gs_range_begin(blockIdx.x + 1, T, G);
   const bool dq = p.dq != 0;
+  const bool sf16 = p.scale_f16 != 0;
   if (tid < p.count) {
     const GsMat &m = p.mat[tid];
     GsInfo &d = info[tid];
@@ -480,7 +479,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   if (g0 < g1) {
     u = gs_describe<B>(info, p.count, mi, g0, g0, g1);
 #pragma unroll
-    for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, u, (warp * R + rt) * 16, lane, sin[rt]);
+    for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
   }
   for (int i = tid; i < 256 * 32; i += WARPS * 32) {
     const int b = i >> 5, l = i & 31;
@@ -560,7 +559,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
     if (gn < g1) {  // next unit: issue its c~ loads now, use them a unit later
       u = gs_next<B>(info, p.count, cu, gn, g0, g1);
 #pragma unroll
-      for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, u, (warp * R + rt) * 16, lane, sin[rt]);
+      for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
     }
     const GsInfo &mt = info[cu.mi];
     const int K = mt.K, N = mt.N;

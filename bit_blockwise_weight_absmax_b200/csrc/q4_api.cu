@@ -128,6 +128,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 int check_state(const q4_state *s) {
   if (!s || !s->packed) return Q4_ERR_ARG;
   if (s->qtype < 0 || s->qtype > 2 || !valid_bs(s->blocksize)) return Q4_ERR_ARG;
+  if (s->scale_f16 != 0 && (s->scale_f16 != 1 || s->qtype == Q4_NF4)) return Q4_ERR_ARG;
   if (s->double_quant) {
     if (s->qtype != Q4_NF4 || !s->absmax_q || !s->absmax_scale || !s->absmax_mean) return Q4_ERR_ARG;
   } else if (!s->absmax) {
@@ -276,6 +277,7 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
   p.status = di.status;
   p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
+  p.scale_f16 = Wq[0]->scale_f16;
   if (qt == Q4_NF4) {
     memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
   } else {
@@ -350,6 +352,7 @@ int gemv_grouped_impl(int32_t count, const void *const *A, const q4_state *const
   p.status = di.status;
   p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
+  p.scale_f16 = Wq[0]->scale_f16;
   int mode = kGvPlain;
   if (qt == Q4_NF4) {
     memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
@@ -399,15 +402,25 @@ int q4_nf4_thresholds(float out[15]) {
 
 int q4_check_device(void) { return device_info().ok; }
 
-int q4_state_sizes(int32_t qtype, int64_t n, int32_t blocksize, int32_t double_quant,
+// qtype with an optional Q4_SCALE_F16: the plain qtype and the flag, or -1.
+static int split_qtype(int32_t qtype, bool *f16) {
+  *f16 = (qtype & Q4_SCALE_F16) != 0;
+  const int32_t q = qtype & ~Q4_SCALE_F16;
+  if (q < 0 || q > 2 || (*f16 && q == Q4_NF4)) return -1;
+  return q;
+}
+
+int q4_state_sizes(int32_t qtype_in, int64_t n, int32_t blocksize, int32_t double_quant,
                    size_t sizes_out[6]) {
-  if (!sizes_out || qtype < 0 || qtype > 2 || !valid_bs(blocksize) ||
+  bool f16 = false;
+  const int qtype = split_qtype(qtype_in, &f16);
+  if (!sizes_out || qtype < 0 || !valid_bs(blocksize) ||
       (double_quant != 0 && double_quant != 1) || (double_quant && qtype != Q4_NF4))
     return Q4_ERR_ARG;
   if (n < 1) return Q4_ERR_SHAPE;
   const int64_t nb = ceil_div(n, blocksize);
   sizes_out[0] = (size_t)((n + 1) / 2);
-  sizes_out[1] = (size_t)nb * 4;
+  sizes_out[1] = (size_t)nb * (f16 ? 2 : 4);
   sizes_out[2] = qtype == Q4_INT4_ASYM ? (size_t)((nb + 1) / 2) : 0;
   sizes_out[3] = double_quant ? (size_t)nb : 0;
   sizes_out[4] = double_quant ? (size_t)ceil_div(nb, Q4_DQ_GROUP) * 4 : 0;
@@ -426,17 +439,19 @@ int q4_quantize_workspace_size(int32_t qtype, int64_t n, int32_t blocksize, int3
 }
 
 int q4_quantize(const void *W, int32_t w_dtype, int64_t rows, int64_t cols, int32_t blocksize,
-                int32_t qtype, int32_t double_quant, q4_state *out, void *workspace,
+                int32_t qtype_in, int32_t double_quant, q4_state *out, void *workspace,
                 size_t workspace_bytes, void *stream) {
   if (!W || !out || !valid_in_dtype(w_dtype)) return Q4_ERR_ARG;
   if (rows < 1 || cols < 1) return Q4_ERR_SHAPE;
   const int64_t n = rows * cols;
   size_t sz[6];
-  int rc = q4_state_sizes(qtype, n, blocksize, double_quant, sz);
+  int rc = q4_state_sizes(qtype_in, n, blocksize, double_quant, sz);
   if (rc != Q4_OK) return rc;
+  bool f16 = false;
+  const int qtype = split_qtype(qtype_in, &f16);
   if (!out->packed || !out->absmax || (qtype == Q4_INT4_ASYM && !out->zero)) return Q4_ERR_ARG;
   if (double_quant && (!out->absmax_q || !out->absmax_scale || !out->absmax_mean)) return Q4_ERR_ARG;
-  if (!aligned16(W) || !aligned16(out->packed) || ((uintptr_t)out->absmax & 3u)) return Q4_ERR_ALIGN;
+  if (!aligned16(W) || !aligned16(out->packed) || ((uintptr_t)out->absmax & (f16 ? 1u : 3u))) return Q4_ERR_ALIGN;
   size_t need = 0;
   q4_quantize_workspace_size(qtype, n, blocksize, double_quant, &need);
   if (need && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
@@ -457,7 +472,7 @@ int q4_quantize(const void *W, int32_t w_dtype, int64_t rows, int64_t cols, int3
   out->blocksize = blocksize;
   out->double_quant = double_quant;
   out->dq_group = Q4_DQ_GROUP;
-  out->reserved = 0;
+  out->scale_f16 = f16 ? 1 : 0;
   if (!double_quant) out->absmax_q = nullptr, out->absmax_scale = nullptr, out->absmax_mean = nullptr;
   if (qtype != Q4_INT4_ASYM) out->zero = nullptr;
 
@@ -483,6 +498,7 @@ int q4_quantize(const void *W, int32_t w_dtype, int64_t rows, int64_t cols, int3
     p.absmax_mean = out->absmax_mean;
   }
   p.status = di.status;
+  p.scale_f16 = f16 ? 1 : 0;
   p.tab = tab;
   cudaStream_t st = (cudaStream_t)stream;
   rc = run_quantize(w_dtype, qtype, blocksize, double_quant != 0, p, grid, st);
@@ -510,19 +526,21 @@ int q4_quantize_grouped_workspace_size(int32_t count, const int64_t *rows, const
 }
 
 int q4_quantize_grouped(int32_t count, const void *const *W, int32_t w_dtype, const int64_t *rows,
-                        const int64_t *cols, int32_t blocksize, int32_t qtype, int32_t double_quant,
+                        const int64_t *cols, int32_t blocksize, int32_t qtype_in, int32_t double_quant,
                         q4_state *const *out, void *workspace, size_t workspace_bytes, void *stream) {
   if (count < 1 || count > kQMaxGroup || !W || !rows || !cols || !out || !valid_in_dtype(w_dtype)) return Q4_ERR_ARG;
   for (int i = 0; i < count; ++i)
     if (!W[i] || !out[i]) return Q4_ERR_ARG;
   size_t need = 0;
-  int rc = q4_quantize_grouped_workspace_size(count, rows, cols, blocksize, qtype, double_quant, &need);
+  int rc = q4_quantize_grouped_workspace_size(count, rows, cols, blocksize, qtype_in, double_quant, &need);
   if (rc != Q4_OK) return rc;
+  bool f16 = false;
+  const int qtype = split_qtype(qtype_in, &f16);
   for (int i = 0; i < count; ++i) {
     q4_state *o = out[i];
     if (!o->packed || !o->absmax || (qtype == Q4_INT4_ASYM && !o->zero)) return Q4_ERR_ARG;
     if (double_quant && (!o->absmax_q || !o->absmax_scale || !o->absmax_mean)) return Q4_ERR_ARG;
-    if (!aligned16(W[i]) || !aligned16(o->packed) || ((uintptr_t)o->absmax & 3u)) return Q4_ERR_ALIGN;
+    if (!aligned16(W[i]) || !aligned16(o->packed) || ((uintptr_t)o->absmax & (f16 ? 1u : 3u))) return Q4_ERR_ALIGN;
   }
   if (need && (!workspace || workspace_bytes < need)) return Q4_ERR_WORKSPACE;
   const DeviceInfo di = device_info();
@@ -551,7 +569,7 @@ int q4_quantize_grouped(int32_t count, const void *const *W, int32_t w_dtype, co
     o->blocksize = blocksize;
     o->double_quant = double_quant;
     o->dq_group = Q4_DQ_GROUP;
-    o->reserved = 0;
+    o->scale_f16 = f16 ? 1 : 0;
     if (!double_quant) o->absmax_q = nullptr, o->absmax_scale = nullptr, o->absmax_mean = nullptr;
     if (qtype != Q4_INT4_ASYM) o->zero = nullptr;
     QMat &m = p.mat[i];
@@ -584,6 +602,7 @@ int q4_quantize_grouped(int32_t count, const void *const *W, int32_t w_dtype, co
   p.status = di.status;
   p.wait_ns = g_wait_limit_ns.load();
   p.stall_copies = g_copy_stall.load();
+  p.scale_f16 = f16 ? 1 : 0;
   p.tab = tab;
   dp.count = count;
   dp.total_groups = groups;
@@ -606,7 +625,7 @@ int q4_dequantize_grouped(int32_t count, const q4_state *const *Wq, void *const 
     const int rc = check_state(Wq[i]);
     if (rc != Q4_OK) return rc;
     if (Wq[i]->qtype != Wq[0]->qtype || Wq[i]->blocksize != Wq[0]->blocksize ||
-        Wq[i]->double_quant != Wq[0]->double_quant)
+        Wq[i]->double_quant != Wq[0]->double_quant || Wq[i]->scale_f16 != Wq[0]->scale_f16)
       return Q4_ERR_ARG;  // one format per grouped call
     if (!aligned16(out[i])) return Q4_ERR_ALIGN;
   }
@@ -631,6 +650,7 @@ int q4_dequantize_grouped(int32_t count, const q4_state *const *Wq, void *const 
   }
   p.count = count;
   p.total_spans = spans;
+  p.scale_f16 = Wq[0]->scale_f16;
   memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
   return run_dequantize(Wq[0]->qtype, out_dtype, Wq[0]->blocksize, Wq[0]->double_quant != 0, p, di.sms,
                         (cudaStream_t)stream);
@@ -670,8 +690,8 @@ int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *
   // every entry is checked before any of them is dereferenced
   for (int i = 0; i < count; ++i)
     if (!Wq[i] || !A[i] || !Y[i]) return Q4_ERR_ARG;
-  for (int i = 0; i < count; ++i)
-    if (Wq[i]->qtype != Wq[0]->qtype) return Q4_ERR_ARG;  // one format per grouped call
+  for (int i = 0; i < count; ++i)  // one format per grouped call
+    if (Wq[i]->qtype != Wq[0]->qtype || Wq[i]->scale_f16 != Wq[0]->scale_f16) return Q4_ERR_ARG;
   if (Wq[0]->qtype == Q4_INT4_ASYM)
     return gemv_grouped_impl(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
   if (M <= kGemvPassRows)
@@ -720,7 +740,7 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     if (rc != Q4_OK) return rc;
     // one format per grouped call
     if (s->qtype != Wq[0]->qtype || s->blocksize != Wq[0]->blocksize ||
-        s->double_quant != Wq[0]->double_quant)
+        s->double_quant != Wq[0]->double_quant || s->scale_f16 != Wq[0]->scale_f16)
       return Q4_ERR_ARG;
     // whole 64-k blocks of whole quantization blocks
     if (s->cols % 64 || s->cols % s->blocksize || s->rows % 16 || s->rows > INT32_MAX || s->cols > INT32_MAX)
@@ -770,6 +790,7 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
       mode = kGemmAsym;
     }
     p.log2_bs = __builtin_ctz((unsigned)Wq[0]->blocksize);
+    p.scale_f16 = Wq[0]->scale_f16;
     p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
     rc = run_gemm(a_dtype, mode, p, di.sms, (cudaStream_t)stream);

@@ -91,6 +91,43 @@ __device__ __forceinline__ float div_markstein(float a, float b, float y) {
   return __fmaf_rn(r, y, q);
 }
 
+// The per-block scale buffer of a state (`absmax`): binary32, or binary16
+// when the state's scales are stored as binary16 (INT4 with Q4_SCALE_F16).
+__device__ __forceinline__ float ld_scale(const float *absmax, int64_t b, bool f16) {
+  if (f16) return __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short *>(absmax) + b)));
+  return __ldg(absmax + b);
+}
+// Scales b0 .. b0 + 7 (all inside the buffer), vector loads when aligned.
+__device__ __forceinline__ void ld_scales8(const float *absmax, int64_t b0, bool f16, float (&f)[8]) {
+  if (f16) {
+    const unsigned short *h = reinterpret_cast<const unsigned short *>(absmax) + b0;
+    if (((uintptr_t)h & 15u) == 0) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(h));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f[2 * j] = __half2float(__ushort_as_half((unsigned short)(w[j] & 0xFFFFu)));
+        f[2 * j + 1] = __half2float(__ushort_as_half((unsigned short)(w[j] >> 16)));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] = __half2float(__ushort_as_half(__ldg(h + j)));
+    }
+  } else if (((uintptr_t)(absmax + b0) & 15u) == 0) {
+    const float4 x = __ldg(reinterpret_cast<const float4 *>(absmax + b0));
+    const float4 y = __ldg(reinterpret_cast<const float4 *>(absmax + b0) + 1);
+    f[0] = x.x, f[1] = x.y, f[2] = x.z, f[3] = x.w, f[4] = y.x, f[5] = y.y, f[6] = y.z, f[7] = y.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = __ldg(absmax + b0 + j);
+  }
+}
+// Stores scale v (already a binary16 value when f16) of block b.
+__device__ __forceinline__ void st_scale(float *absmax, int64_t b, float v, bool f16) {
+  if (f16) reinterpret_cast<unsigned short *>(absmax)[b] = __half_as_ushort(__float2half_rn(v));
+  else absmax[b] = v;
+}
+
 // Two binary32 values in one 64-bit register for the packed f32x2 ALU ops
 // of sm_100 (each lane of a pair is computed and rounded exactly as the
 // scalar instruction would).

@@ -58,6 +58,7 @@ struct QuantParams {
   unsigned *counter;      // arrival counter (double quant), left at 0
   float *absmax_mean;     // mean output (double quant)
   int *status;            // sticky status word
+  int32_t scale_f16;      // INT4: binary16 scales
   Nf4BinTable tab;
 };
 
@@ -83,6 +84,7 @@ struct QuantGroupParams {
   int64_t total_chunks;
   uint64_t wait_ns;      // bound of every mbarrier wait
   int *status;
+  int32_t scale_f16;     // INT4: binary16 scales
   Nf4BinTable tab;
 };
 
@@ -113,9 +115,11 @@ __device__ __forceinline__ uint32_t nf4_code_bits(uint32_t bits, float x, uint32
 // (adjacent lanes) agree on `scale` and `z`.  Must be called by all 32 lanes.
 // tb: this lane's bin-table address minus 2^30; s_tab: the lane-private
 // bin tables ([bin][lane]); nonfinite is set when the block holds Inf / NaN.
+// sf16 (INT4): the scale is rounded to binary16 as soon as it is formed and
+// the codes are computed against the rounded value.
 template <int DT, int QT, int B>
 __device__ __forceinline__ void quant16(const uint4 (&v)[2], float &scale, int &z, uint32_t (&codes)[2], int lane,
-                                        uint32_t tb, const float2 *s_tab, int &nonfinite) {
+                                        uint32_t tb, const float2 *s_tab, int &nonfinite, bool sf16 = false) {
   constexpr int E = 16, V = 2, LPB = B / E;
   float f[E];
 #pragma unroll
@@ -168,24 +172,44 @@ __device__ __forceinline__ void quant16(const uint4 (&v)[2], float &scale, int &
         }
       }
     } else {
-      const float s = __fdiv_rn(c, 7.0f);
+      float s = __fdiv_rn(c, 7.0f);
+      if (sf16) s = __half2float(__float2half_rn(s));
       scale = s;
       if (__all_sync(0xffffffffu, markstein_ok(s))) {
-        // |w / s| <= 7 / (1 - 2^-24): rint never leaves [-7, 7], and adding
-        // 1.5 * 2^23 rounds to the nearest integer, ties to even, leaving
-        // its 4-bit two's complement in the low nibble
+        // binary32 s: |w / s| <= 7 / (1 - 2^-24), so rint never leaves
+        // [-7, 7], and adding 1.5 * 2^23 rounds to the nearest integer, ties
+        // to even, leaving its 4-bit two's complement in the low nibble
         const float y = __frcp_rn(s);
         const uint64_t yy = f2_pack(y, y), ns = f2_pack(-s, -s);
         const uint64_t kr = f2_pack(12582912.0f, 12582912.0f);
+        if (!sf16) {
 #pragma unroll
-        for (int k = 0; k < V; ++k)
+          for (int k = 0; k < V; ++k)
 #pragma unroll
-          for (int j = 3; j >= 0; --j) {
-            const uint64_t r2 = f2_add(div_markstein2(f2_pack(f[8 * k + 2 * j], f[8 * k + 2 * j + 1]), ns, yy), kr);
-            float r0, r1;
-            f2_unpack(r2, r0, r1);
-            codes[k] = (codes[k] << 8) | ((__float_as_uint(r1) & 15u) << 4) | (__float_as_uint(r0) & 15u);
-          }
+            for (int j = 3; j >= 0; --j) {
+              const uint64_t r2 =
+                  f2_add(div_markstein2(f2_pack(f[8 * k + 2 * j], f[8 * k + 2 * j + 1]), ns, yy), kr);
+              float r0, r1;
+              f2_unpack(r2, r0, r1);
+              codes[k] = (codes[k] << 8) | ((__float_as_uint(r1) & 15u) << 4) | (__float_as_uint(r0) & 15u);
+            }
+        } else {
+          // a binary16 s can lie well below c / 7 (a subnormal keeps few
+          // bits), so the rounded quotient is clamped to [-8, 7]; it stays
+          // far below 2^22, where the 1.5 * 2^23 rounding holds
+#pragma unroll
+          for (int k = 0; k < V; ++k)
+#pragma unroll
+            for (int j = 3; j >= 0; --j) {
+              const uint64_t r2 =
+                  f2_add(div_markstein2(f2_pack(f[8 * k + 2 * j], f[8 * k + 2 * j + 1]), ns, yy), kr);
+              float r0, r1;
+              f2_unpack(r2, r0, r1);
+              const int q0 = min(max((int)(__float_as_uint(r0) - 0x4B400000u), -8), 7);
+              const int q1 = min(max((int)(__float_as_uint(r1) - 0x4B400000u), -8), 7);
+              codes[k] = (codes[k] << 8) | ((uint32_t)(q1 & 15) << 4) | (uint32_t)(q0 & 15);
+            }
+        }
       } else {
         const bool fast = markstein_ok(s);
         const float y = fast ? __frcp_rn(s) : 0.0f;
@@ -217,13 +241,16 @@ __device__ __forceinline__ void quant16(const uint4 (&v)[2], float &scale, int &
       m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     }
     if (!(Dt<DT>::to_f((uint16_t)m) <= 3.4028235e38f)) nonfinite = 1;
-    const float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+    float s = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+    if (sf16) s = __half2float(__float2half_rn(s));
     scale = s;
     z = 0;
     if (__all_sync(0xffffffffu, markstein_ok(s))) {
-      // mn <= 0 <= mx and s = (mx - mn) / 15, so |w / s| <= 15 (1 + 2^-23):
-      // adding 1.5 * 2^23 rounds the quotient to the nearest integer, ties
-      // to even, with the integer in the low bits of the sum's pattern
+      // mn <= 0 <= mx and s = (mx - mn) / 15, so |w / s| <= 15 (1 + 2^-23)
+      // (a few times that for a binary16 s rounded to a subnormal; the code
+      // is clamped): adding 1.5 * 2^23 rounds the quotient to the nearest
+      // integer, ties to even, with the integer in the low bits of the
+      // sum's pattern
       const float y = __frcp_rn(s);
       z = min(max(__float2int_rn(div_markstein(-mn, s, y)), 0), 15);
       const uint64_t yy = f2_pack(y, y), ns = f2_pack(-s, -s);
@@ -339,7 +366,7 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(const __grid_con
           float scale = 0.0f;
           int z = 0;
           uint32_t codes[V];
-          quant16<DT, QT, B>(v[b], scale, z, codes, lane, tb, s_tab, nonfinite);
+          quant16<DT, QT, B>(v[b], scale, z, codes, lane, tb, s_tab, nonfinite, p.scale_f16 != 0);
           if (QT == Q4_INT4_ASYM && (tid % LPB) == 0) s_zero[(tid * E) / B] = (uint8_t)z;
           // ---- stores
           const int64_t e0 = chunk_e0 + off + tid * E;
@@ -358,7 +385,7 @@ __global__ void __launch_bounds__(kQThreads, 4) quantize_kernel(const __grid_con
           }
           if ((tid % LPB) == 0) {
             const bool in = FULL || chunk_b0 + bl < nb;
-            if (in) absmax[chunk_b0 + bl] = scale;
+            if (in) st_scale(absmax, chunk_b0 + bl, scale, p.scale_f16 != 0);
             if (DQ) s_blk[cpar][bl] = in ? (double)scale : 0.0;
           }
           if (QT == Q4_INT4_ASYM) {

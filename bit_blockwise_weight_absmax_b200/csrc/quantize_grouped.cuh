@@ -262,7 +262,9 @@ __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const _
     int left = 0;                  // weights of the current chunk (CHUNK when whole)
     const uint16_t *W = nullptr;   // the current chunk's weights, packed codes, scales, zero-points
     uint8_t *pk = nullptr, *zc = nullptr;
-    float *am = nullptr, *sb = nullptr;
+    float *am = nullptr, *sb = nullptr;  // am: the matrix's scales; block b of the chunk at ab0 + b
+    int64_t ab0 = 0;
+    const bool sf16 = p.scale_f16 != 0;
     // One 16-weight group of a slice: weights g0..g0+15 of the chunk, read
     // at shared address src.
     auto group = [&](int g0, uint32_t src, int pe0) {
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const _
       if (left == (int)CHUNK) {
         v[0] = lds_v4(src);
         v[1] = lds_v4(src + 16);
-        quant16<DT, QT, B>(v, scale, z, codes, lane, tb, s_tab, nonfinite);
+        quant16<DT, QT, B>(v, scale, z, codes, lane, tb, s_tab, nonfinite, sf16);
         *reinterpret_cast<uint2 *>(pk + g0 / 2) = make_uint2(codes[0], codes[1]);
         if (QT == Q4_INT4_ASYM) {
           // the zero-points of blocks 2k, 2k+1 share a byte; 512 weights
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const _
           if ((lane % (2 * LPB)) == 0) zc[bl >> 1] = (uint8_t)(z | (zn << 4));
         }
         if ((lane % LPB) == 0) {
-          am[bl] = scale;
+          st_scale(am, ab0 + bl, scale, sf16);
           if (DQ) sb[bl] = scale;
         }
       } else {
@@ -316,7 +318,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const _
           v[0] = make_uint4(w[0], w[1], w[2], w[3]);
           v[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
-        quant16<DT, QT, B>(v, scale, z, codes, lane, tb, s_tab, nonfinite);
+        quant16<DT, QT, B>(v, scale, z, codes, lane, tb, s_tab, nonfinite, sf16);
         const int nv = min(16, left - g0);  // this lane's weights (<= 0: none)
         if (nv >= 16) {
           *reinterpret_cast<uint2 *>(pk + g0 / 2) = make_uint2(codes[0], codes[1]);
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const _
           if ((lane % (2 * LPB)) == 0 && nv > 0) zc[bl >> 1] = (uint8_t)(z | (zn << 4));
         }
         if ((lane % LPB) == 0 && nv > 0) {
-          am[bl] = scale;
+          st_scale(am, ab0 + bl, scale, sf16);
           if (DQ) sb[bl] = scale;
         }
       }
@@ -356,7 +358,8 @@ __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const _
         left = (int)min(CHUNK, m.n - ce0);
         W = m.W + ce0;
         pk = m.packed + ce0 / 2;
-        am = m.absmax + chunk * kChunkBlocks;
+        am = m.absmax;
+        ab0 = chunk * kChunkBlocks;
         zc = QT == Q4_INT4_ASYM ? m.zero + chunk * (kChunkBlocks / 2) : nullptr;
         sb = s_blk + (k % kQgBufs) * kChunkBlocks;
       }

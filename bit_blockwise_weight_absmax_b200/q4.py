@@ -19,6 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libq4.so")
 
 NF4, INT4_SYM, INT4_ASYM = 0, 1, 2
+SCALE_F16 = 0x100  # OR into an INT4 qtype: binary16 group scales
 F16, BF16, F32 = 0, 1, 2
 QTYPES = {"nf4": NF4, "int4_sym": INT4_SYM, "int4_asym": INT4_ASYM}
 _DT = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
@@ -34,7 +35,7 @@ class _CState(ctypes.Structure):
     _fields_ = [("qtype", ctypes.c_int32), ("src_dtype", ctypes.c_int32), ("n", ctypes.c_int64),
                 ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
                 ("blocksize", ctypes.c_int32), ("double_quant", ctypes.c_int32),
-                ("dq_group", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("dq_group", ctypes.c_int32), ("scale_f16", ctypes.c_int32),
                 ("packed", ctypes.c_void_p), ("absmax", ctypes.c_void_p), ("zero", ctypes.c_void_p),
                 ("absmax_q", ctypes.c_void_p), ("absmax_scale", ctypes.c_void_p),
                 ("absmax_mean", ctypes.c_void_p)]
@@ -132,6 +133,7 @@ class Q4State:
     absmax_q: torch.Tensor | None = None
     absmax_scale: torch.Tensor | None = None
     absmax_mean: torch.Tensor | None = None
+    scale_f16: bool = False  # INT4: absmax holds binary16 scales
 
     @property
     def n(self) -> int:
@@ -144,7 +146,7 @@ class Q4State:
     def c_struct(self) -> _CState:
         """The C view of the state, built once and rebuilt only when a buffer
         or a field has changed."""
-        key = (self.qtype, self.src_dtype, self.rows, self.cols, self.blocksize, self.double_quant,
+        key = (self.qtype, self.src_dtype, self.rows, self.cols, self.blocksize, self.double_quant, self.scale_f16,
                self.packed.data_ptr(), None if self.absmax is None else self.absmax.data_ptr(),
                None if self.zero is None else self.zero.data_ptr(),
                None if self.absmax_q is None else self.absmax_q.data_ptr(),
@@ -167,6 +169,7 @@ class Q4State:
         s.blocksize = self.blocksize
         s.double_quant = int(self.double_quant)
         s.dq_group = DQ_GROUP
+        s.scale_f16 = int(self.scale_f16)
         s.packed = self.packed.data_ptr()
         s.absmax = None if self.absmax is None else self.absmax.data_ptr()
         s.zero = None if self.zero is None else self.zero.data_ptr()
@@ -196,7 +199,7 @@ class Q4State:
         if self.double_quant:
             b += self.absmax_q.numel() + 4 * self.absmax_scale.numel() + 4
         else:
-            b += 4 * self.absmax.numel()
+            b += self.absmax.numel() * self.absmax.element_size()
             if self.zero is not None:
                 b += self.zero.numel()
         return b
@@ -270,64 +273,62 @@ def _workspace(device, kind: str, nbytes: int) -> torch.Tensor | None:
 # ------------------------------------------------------------------- ops ----
 
 def quantize(W: torch.Tensor, blocksize: int = 64, qtype="nf4", double_quant: bool = False,
-             stream=None, out: Q4State | None = None) -> Q4State:
+             stream=None, out: Q4State | None = None, scale_f16: bool = False) -> Q4State:
     """Blockwise 4-bit quantization of a 2-D fp16/bf16 CUDA tensor.
 
     `out` reuses the buffers of an earlier state of the same shape and format
-    (no allocation: the call can be captured in a CUDA graph)."""
+    (no allocation: the call can be captured in a CUDA graph).  scale_f16
+    (INT4 only): binary16 group scales, the codes taken against them."""
     _require_gpu(W)
     if W.dtype not in (torch.float16, torch.bfloat16) or W.dim() != 2:
         raise Q4Error("W must be a 2-D float16/bfloat16 tensor")
     W = W.contiguous()
     qt = QTYPES[qtype] if isinstance(qtype, str) else int(qtype)
+    qt_arg = qt | (SCALE_F16 if scale_f16 else 0)
     rows, cols = W.shape
     n = rows * cols
-    sz = state_sizes(qt, n, blocksize, double_quant)
     dev = W.device
     if out is not None:
-        if (out.qtype, out.rows, out.cols, out.blocksize, out.double_quant) != \
-                (qt, rows, cols, blocksize, bool(double_quant)):
+        if (out.qtype, out.rows, out.cols, out.blocksize, out.double_quant, out.scale_f16) != \
+                (qt, rows, cols, blocksize, bool(double_quant), bool(scale_f16)):
             raise Q4Error("out= state has a different shape or format")
         if out.absmax is None:
             raise Q4Error("out= state has released its absmax buffer, which quantize writes")
         out.src_dtype = W.dtype
-    st = out if out is not None else Q4State(qt, W.dtype, rows, cols, blocksize, bool(double_quant),
-                 packed=torch.empty(sz[0], dtype=torch.uint8, device=dev),
-                 absmax=torch.empty(sz[1] // 4, dtype=torch.float32, device=dev),
-                 zero=torch.empty(sz[2], dtype=torch.uint8, device=dev) if sz[2] else None,
-                 absmax_q=torch.empty(sz[3], dtype=torch.int8, device=dev) if sz[3] else None,
-                 absmax_scale=torch.empty(sz[4] // 4, dtype=torch.float32, device=dev) if sz[4] else None,
-                 absmax_mean=torch.empty(1, dtype=torch.float32, device=dev) if sz[5] else None)
+    st = out if out is not None else _new_state(qt, W.dtype, rows, cols, blocksize, double_quant, dev, scale_f16)
     wsz = ctypes.c_size_t(0)
-    _check(library().q4_quantize_workspace_size(qt, n, blocksize, int(double_quant), ctypes.byref(wsz)),
+    _check(library().q4_quantize_workspace_size(qt_arg, n, blocksize, int(double_quant), ctypes.byref(wsz)),
            "q4_quantize_workspace_size")
     ws = _workspace(dev, "quantize", wsz.value)
     cs = st.c_struct()
-    _check(library().q4_quantize(_ptr(W), _DT[W.dtype], rows, cols, blocksize, qt, int(double_quant),
+    _check(library().q4_quantize(_ptr(W), _DT[W.dtype], rows, cols, blocksize, qt_arg, int(double_quant),
                                  ctypes.byref(cs), _ptr(ws), 0 if ws is None else ws.numel(),
                                  _stream(stream)), "q4_quantize")
     return st
 
 
-def _new_state(qt, dtype, rows, cols, blocksize, double_quant, dev) -> Q4State:
-    sz = state_sizes(qt, rows * cols, blocksize, double_quant)
+def _new_state(qt, dtype, rows, cols, blocksize, double_quant, dev, scale_f16=False) -> Q4State:
+    sz = state_sizes(qt | (SCALE_F16 if scale_f16 else 0), rows * cols, blocksize, double_quant)
     return Q4State(qt, dtype, rows, cols, blocksize, bool(double_quant),
                    packed=torch.empty(sz[0], dtype=torch.uint8, device=dev),
-                   absmax=torch.empty(sz[1] // 4, dtype=torch.float32, device=dev),
+                   absmax=(torch.empty(sz[1] // 2, dtype=torch.float16, device=dev) if scale_f16 else
+                           torch.empty(sz[1] // 4, dtype=torch.float32, device=dev)),
                    zero=torch.empty(sz[2], dtype=torch.uint8, device=dev) if sz[2] else None,
                    absmax_q=torch.empty(sz[3], dtype=torch.int8, device=dev) if sz[3] else None,
                    absmax_scale=torch.empty(sz[4] // 4, dtype=torch.float32, device=dev) if sz[4] else None,
-                   absmax_mean=torch.empty(1, dtype=torch.float32, device=dev) if sz[5] else None)
+                   absmax_mean=torch.empty(1, dtype=torch.float32, device=dev) if sz[5] else None,
+                   scale_f16=bool(scale_f16))
 
 
 def quantize_grouped(Ws, blocksize: int = 64, qtype="nf4", double_quant: bool = False, stream=None,
-                     outs=None) -> list:
+                     outs=None, scale_f16: bool = False) -> list:
     """Quantize several 2-D weights of one dtype and one format in one launch
     (plus one second-level launch with double quantization); the states are
     bit for bit those of quantize() on each weight.  `outs` reuses earlier
     states of the same shapes and format (no allocation)."""
     _require_gpu(Ws[0])
     qt = QTYPES[qtype] if isinstance(qtype, str) else int(qtype)
+    qt_arg = qt | (SCALE_F16 if scale_f16 else 0)
     dtype = Ws[0].dtype
     for W in Ws:
         if W.dtype != dtype or W.dim() != 2 or W.dtype not in (torch.float16, torch.bfloat16):
@@ -335,24 +336,26 @@ def quantize_grouped(Ws, blocksize: int = 64, qtype="nf4", double_quant: bool = 
     Ws = [W.contiguous() for W in Ws]
     dev = Ws[0].device
     if outs is None:
-        outs = [_new_state(qt, dtype, W.shape[0], W.shape[1], blocksize, double_quant, dev) for W in Ws]
+        outs = [_new_state(qt, dtype, W.shape[0], W.shape[1], blocksize, double_quant, dev, scale_f16)
+                for W in Ws]
     else:
         for st, W in zip(outs, Ws):
-            if (st.qtype, st.rows, st.cols, st.blocksize, st.double_quant) != \
-                    (qt, W.shape[0], W.shape[1], blocksize, bool(double_quant)) or st.absmax is None:
+            if (st.qtype, st.rows, st.cols, st.blocksize, st.double_quant, st.scale_f16) != \
+                    (qt, W.shape[0], W.shape[1], blocksize, bool(double_quant), bool(scale_f16)) \
+                    or st.absmax is None:
                 raise Q4Error("outs= states have a different shape or format")
             st.src_dtype = dtype
     n = len(Ws)
     rows = (ctypes.c_int64 * n)(*[W.shape[0] for W in Ws])
     cols = (ctypes.c_int64 * n)(*[W.shape[1] for W in Ws])
     wsz = ctypes.c_size_t(0)
-    _check(library().q4_quantize_grouped_workspace_size(n, rows, cols, blocksize, qt, int(double_quant),
+    _check(library().q4_quantize_grouped_workspace_size(n, rows, cols, blocksize, qt_arg, int(double_quant),
                                                          ctypes.byref(wsz)), "q4_quantize_grouped_workspace_size")
     ws = _workspace(dev, "quantize", wsz.value)
     structs = [st.c_struct() for st in outs]
     arr = (ctypes.POINTER(_CState) * n)(*[ctypes.pointer(c) for c in structs])
     wp = (ctypes.c_void_p * n)(*[W.data_ptr() for W in Ws])
-    _check(library().q4_quantize_grouped(n, wp, _DT[dtype], rows, cols, blocksize, qt, int(double_quant), arr,
+    _check(library().q4_quantize_grouped(n, wp, _DT[dtype], rows, cols, blocksize, qt_arg, int(double_quant), arr,
                                          _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
            "q4_quantize_grouped")
     return outs

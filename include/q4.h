@@ -80,6 +80,15 @@ typedef enum {
 
 typedef enum { Q4_F16 = 0, Q4_BF16 = 1, Q4_F32 = 2 /* outputs only */ } q4_dtype;
 
+/* OR'ed into an INT4 qtype (Q4_INT4_SYM | Q4_SCALE_F16, Q4_INT4_ASYM |
+ * Q4_SCALE_F16) at q4_state_sizes / q4_quantize*: the group scale is stored
+ * as binary16 ([INT4] "Components": the per-group scale is "usually stored
+ * in FP16").  s is rounded to binary16 (round to nearest even) as soon as
+ * it is formed, and the zero-point and every code are computed against the
+ * rounded s; the state's qtype keeps the plain INT4 value and its
+ * scale_f16 field is 1.  Not defined for NF4 (Q4_ERR_ARG). */
+#define Q4_SCALE_F16 0x100
+
 #define Q4_DQ_GROUP 256 /* [BWQ]: the block scales are quantized in blocks of 256 */
 
 /*
@@ -92,6 +101,8 @@ typedef enum { Q4_F16 = 0, Q4_BF16 = 1, Q4_F32 = 2 /* outputs only */ } q4_dtype
  *                two's-complement nibble of q in [-8, 7].
  *   absmax       float [nb], nb = ceil(n / blocksize): the NF4 absmax c, or
  *                the INT4 scale s.  With double_quant it still holds c.
+ *                With scale_f16 it holds binary16 [nb] (the pointer type is
+ *                unchanged; the buffer is nb * 2 bytes).
  *   zero         uint8 [ceil(nb/2)] (INT4_ASYM only, else NULL): zero-point
  *                of block b in nibble b, low nibble first.
  *   absmax_q     int8 [nb] (double_quant only, else NULL): 8-bit code of c.
@@ -106,7 +117,7 @@ typedef struct {
   int32_t blocksize;    /* B: 32, 64, 128 or 256 */
   int32_t double_quant; /* 0 / 1 (NF4 only) */
   int32_t dq_group;     /* Q4_DQ_GROUP */
-  int32_t reserved;
+  int32_t scale_f16;    /* 0 / 1: binary16 INT4 scales (see Q4_SCALE_F16) */
   uint8_t *packed;
   float *absmax;
   uint8_t *zero;
@@ -139,7 +150,8 @@ Q4_API int q4_quantize_workspace_size(int32_t qtype, int64_t n, int32_t blocksiz
  *   W          device, 16-byte aligned, rows*cols 16-bit floats of w_dtype
  *              (Q4_F16 / Q4_BF16), row-major.
  *   blocksize  32, 64, 128 or 256 (64 is the [BWQ] default for NF4).
- *   qtype      Q4_NF4 / Q4_INT4_SYM / Q4_INT4_ASYM.
+ *   qtype      Q4_NF4 / Q4_INT4_SYM / Q4_INT4_ASYM, the INT4 ones
+ *              optionally | Q4_SCALE_F16.
  *   double_quant  0 or 1; 1 only with Q4_NF4.
  *   out        host struct; its six pointers must already point to device
  *              buffers of q4_state_sizes() bytes (packed/absmax 16-byte

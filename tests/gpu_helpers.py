@@ -47,8 +47,13 @@ def assert_matmul_close(y_gpu, y_ref, rel_fro=REL_FRO, max_abs=MAX_ABS):
 def assert_state_equal(st, ost):
     """GPU state (Q4State) equals the oracle state bit for bit."""
     assert np.array_equal(st.packed.cpu().numpy(), ost.packed), "packed codes differ"
-    assert np.array_equal(st.absmax.cpu().numpy().view(np.uint32), ost.absmax.view(np.uint32)), \
-        "absmax / scale differs"
+    if getattr(ost, "scale_f16", 0):
+        assert st.scale_f16 and st.absmax.dtype == torch.float16
+        assert np.array_equal(st.absmax.cpu().numpy().view(np.uint16), ost.scale_f16_bits()), \
+            "binary16 scale differs"
+    else:
+        assert np.array_equal(st.absmax.cpu().numpy().view(np.uint32), ost.absmax.view(np.uint32)), \
+            "absmax / scale differs"
     if ost.zero is not None:
         assert np.array_equal(st.zero.cpu().numpy(), ost.zero), "zero-points differ"
     if ost.absmax_q is not None:
@@ -59,5 +64,5 @@ def assert_state_equal(st, ost):
                               ost.absmax_mean.view(np.uint32)), "double-quant mean differs"
 
 
-def oracle_state(oracle, W: torch.Tensor, blocksize, qtype, dq):
-    return oracle.quantize(bits(W), is_bf16(W), blocksize, qtype, dq)
+def oracle_state(oracle, W: torch.Tensor, blocksize, qtype, dq, scale_f16=False):
+    return oracle.quantize(bits(W), is_bf16(W), blocksize, qtype, dq, scale_f16)

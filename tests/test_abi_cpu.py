@@ -263,3 +263,28 @@ def test_grouped_calls_reject_a_null_entry_before_any_use(lib):
             assert lib.q4_gemv_grouped(2, ptrs, arr, bad, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None) == -1
             assert lib.q4_gemm_grouped(2, bad, arr, ptrs, 512, 1, 1, None) == -1
             assert lib.q4_gemm_grouped(2, ptrs, arr, bad, 512, 1, 1, None) == -1
+
+
+def test_binary16_scale_sizes_and_checks(lib, oracle):
+    """Q4_SCALE_F16 (INT4 only): the scale buffer is 2 bytes per block, the
+    rest of the state unchanged, and the sizes match the oracle's storage
+    count; NF4 with the flag is Q4_ERR_ARG, and so is a state that claims
+    binary16 scales for NF4."""
+    from bit_blockwise_weight_absmax_b200 import q4
+    out = (ctypes.c_size_t * 6)()
+    n, bs = 100_000, 128
+    nb = -(-n // bs)
+    for qt in (1, 2):
+        assert lib.q4_state_sizes(qt | 0x100, n, bs, 0, out) == 0
+        assert out[1] == 2 * nb
+        total = sum(out)
+        bits = oracle.storage_bits_per_param(qt, bs, False, n, scale_f16=True)
+        assert abs(8 * total / n - bits) < 1e-12
+    assert lib.q4_state_sizes(0 | 0x100, n, bs, 0, out) == -1
+    assert lib.q4_state_sizes(1 | 0x100, n, bs, 1, out) == -1
+    st = _fake_state(0, 256, 512, 64, False)
+    st.scale_f16 = 1
+    P = ctypes.POINTER(q4._CState)
+    arr = (P * 1)(ctypes.pointer(st))
+    ptrs = (ctypes.c_void_p * 1)(0x70000)
+    assert lib.q4_gemm_grouped(1, ptrs, arr, ptrs, 512, 1, 1, None) == -1

@@ -410,3 +410,62 @@ def test_dequantize_grouped_equals_single_and_oracle(q4, oracle, qtype, bs, dq, 
         assert torch.equal(o.view(torch.int16), single.view(torch.int16))
         ost = oracle_state(oracle, W, bs, QT[qtype], dq)
         assert np.array_equal(bits(o), oracle.dequantize(ost, out_dtype == torch.bfloat16))
+
+
+# ------------------------------------------------------- binary16 scales --
+# robotsatlas.com, "INT4", "Components": the per-group scale "usually stored
+# in FP16".
+
+@pytest.mark.parametrize("qtype", ["int4_sym", "int4_asym"])
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_fp16_scales_quantize_dequantize(q4, oracle, qtype, bs, dtype):
+    """Binary16 group scales: the single and the grouped quantize give the
+    oracle's state bit for bit (codes taken against the rounded scale) on
+    ragged shapes with tiny and large groups; dequantize is bit-exact too."""
+    g = torch.Generator().manual_seed(90 + bs)
+    shapes = [(300, 1024), (17, 96 * 2), (5, 7 * 32)]
+    Ws = [torch.randn(N, K, generator=g) * 0.02 for N, K in shapes]
+    Ws[0][3] *= 1e-5  # scales that round to binary16 subnormals
+    Ws[0][5] *= 3e3
+    Ws = [W.to(dtype) for W in Ws]
+    grouped = q4.quantize_grouped([dev(W) for W in Ws], bs, qtype, False, scale_f16=True)
+    for W, gst in zip(Ws, grouped):
+        ost = oracle_state(oracle, W, bs, QT[qtype], False, scale_f16=True)
+        assert_state_equal(gst, ost)
+        st = q4.quantize(dev(W), bs, qtype, False, scale_f16=True)
+        assert_state_equal(st, ost)
+        for out_dt in (torch.float16, torch.bfloat16):
+            d = q4.dequantize(st, out_dt)
+            assert np.array_equal(bits(d), oracle.dequantize(ost, out_dt == torch.bfloat16))
+
+
+@pytest.mark.parametrize("qtype,M", [("int4_sym", 1), ("int4_sym", 16), ("int4_sym", 24),
+                                     ("int4_asym", 4), ("int4_asym", 32)])
+def test_fp16_scales_gemv(q4, oracle, qtype, M):
+    """Both decode kernels read binary16 scales: the GEMV of a binary16-scale
+    state against the oracle's product of its dequantized weights."""
+    g = torch.Generator().manual_seed(95 + M)
+    N, K = 1000, 4096
+    W = (torch.randn(N, K, generator=g) * 0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).half()
+    st = q4.quantize(dev(W), 128, qtype, False, scale_f16=True)
+    ost = oracle_state(oracle, W, 128, QT[qtype], False, scale_f16=True)
+    y = q4.gemv(dev(A), st)
+    ref = oracle.gemv_reference(bits(A), False, ost, N, K)
+    assert_matmul_close(y, ref)
+
+
+@pytest.mark.parametrize("qtype", ["int4_sym", "int4_asym"])
+def test_fp16_scales_gemm(q4, oracle, qtype):
+    """The GEMM reads binary16 scales; against the oracle at M = 300."""
+    g = torch.Generator().manual_seed(99)
+    M, N, K = 300, 272, 4608
+    W = (torch.randn(N, K, generator=g) * 0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).bfloat16()
+    st = q4.quantize(dev(W), 64, qtype, False, scale_f16=True)
+    ost = oracle_state(oracle, W, 64, QT[qtype], False, scale_f16=True)
+    y = q4.gemm(dev(A), st)
+    w16 = oracle.dequantize(ost, True).reshape(N, K)
+    ref = oracle.matmul(bits(A), True, w16, True, M, N, K)
+    assert_matmul_close(y, ref)
