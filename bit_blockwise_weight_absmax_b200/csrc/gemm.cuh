@@ -68,6 +68,13 @@ struct alignas(64) GemmMat {
   int32_t pad;
 };
 
+// Up to this many tiles a launch carries an explicit tile list per CTA,
+// balanced on the host by the k-blocks of each tile (longest first onto the
+// least loaded CTA); above it the tiles are dealt round robin, which is then
+// within a few percent of even.
+constexpr int kGemmListTiles = 2048;
+constexpr int kGemmListCtas = 256;  // grid bound of a listed launch
+
 struct GemmParams {
   GemmMat mat[16];
   int32_t count;
@@ -80,6 +87,9 @@ struct GemmParams {
   uint64_t wait_ns;      // bound of every mbarrier wait
   int *status;
   float levels[16];
+  int32_t listed;        // tiles come from tile_list (else round robin)
+  uint16_t cta_off[kGemmListCtas + 1];  // CTA c runs tile_list[cta_off[c] .. cta_off[c + 1])
+  uint16_t tile_list[kGemmListTiles];
 };
 
 // ---- PTX wrappers ------------------------------------------------------------
@@ -290,13 +300,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   volatile int *abort = &s_abort;
+  // this CTA's tiles: a host-balanced list, or every gridDim.x-th tile
+  const int64_t n_my = p.listed ? (int64_t)(p.cta_off[blockIdx.x + 1] - p.cta_off[blockIdx.x])
+                                : (p.total_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+  auto my_tile = [&](int64_t k) -> int64_t {
+    return p.listed ? (int64_t)p.tile_list[p.cta_off[blockIdx.x] + k] : (int64_t)blockIdx.x + k * gridDim.x;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x) {
-        const TileCoord tc = gemm_tile(p, t);
+      for (int64_t k = 0; k < n_my && !*abort; ++k) {
+        const TileCoord tc = gemm_tile(p, my_tile(k));
         const GemmMat &m = p.mat[tc.mi];
         const int nk = m.K / kGemmBK;
         for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -324,8 +340,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       uint32_t it = 0, tcount = 0;
       uint32_t last_bar = 0, last_par = 0;  // the barrier and phase of the last commit issued
       bool committed = false;
-      for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++tcount) {
-        const TileCoord tc = gemm_tile(p, t);
+      for (int64_t k = 0; k < n_my && !*abort; ++k, ++tcount) {
+        const TileCoord tc = gemm_tile(p, my_tile(k));
         const int nk = p.mat[tc.mi].K / kGemmBK;
         const int ab = tcount & 1;  // accumulator set of this tile
         if (!mbar_wait(accempty_bar(ab), ((tcount >> 1) & 1) ^ 1, p.status, abort, p.wait_ns)) break;
@@ -424,8 +440,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     TileCoord prev_tc{0, 0, 0};
     uint32_t prev_count = 0;
     uint32_t it = 0, tcount = 0;
-    for (int64_t t = blockIdx.x; t < p.total_tiles && !*abort; t += gridDim.x, ++tcount) {
-      const TileCoord tc = gemm_tile(p, t);
+    for (int64_t k = 0; k < n_my && !*abort; ++k, ++tcount) {
+      const TileCoord tc = gemm_tile(p, my_tile(k));
       const GemmMat &m = p.mat[tc.mi];
       const int nk = m.K / kGemmBK;
       const int lbs = p.log2_bs;

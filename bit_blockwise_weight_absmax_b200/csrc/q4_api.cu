@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "q4_internal.h"
 
@@ -719,6 +720,40 @@ int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void 
   return q4_gemv_grouped(1, a, w, y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
 }
 
+// The tiles of a small launch dealt to the CTAs longest first (k-blocks of
+// the tile), each onto the CTA with the least work so far; every CTA then
+// runs its tiles in ascending order.  Round robin otherwise.
+static void gemm_balance(GemmParams &p, int count, int64_t grid) {
+  p.listed = 0;
+  if (p.total_tiles > kGemmListTiles || grid > kGemmListCtas || p.total_tiles <= grid) return;
+  std::vector<std::pair<int, int>> order;  // (k-blocks, tile)
+  order.reserve((size_t)p.total_tiles);
+  for (int i = 0; i < count; ++i) {
+    const GemmMat &m = p.mat[i];
+    const int64_t n = (int64_t)m.tiles_m * m.tiles_n;
+    for (int64_t t = 0; t < n; ++t) order.emplace_back(m.K / kGemmBK, (int)(m.tile_begin + t));
+  }
+  std::stable_sort(order.begin(), order.end(),
+                   [](const std::pair<int, int> &a, const std::pair<int, int> &b) { return a.first > b.first; });
+  std::vector<std::vector<int>> per((size_t)grid);
+  std::vector<int64_t> load((size_t)grid, 0);
+  for (const auto &o : order) {
+    int64_t best = 0;
+    for (int64_t c = 1; c < grid; ++c)
+      if (load[(size_t)c] < load[(size_t)best]) best = c;
+    load[(size_t)best] += o.first;
+    per[(size_t)best].push_back(o.second);
+  }
+  int off = 0;
+  for (int64_t c = 0; c < grid; ++c) {
+    p.cta_off[c] = (uint16_t)off;
+    std::sort(per[(size_t)c].begin(), per[(size_t)c].end());
+    for (int t : per[(size_t)c]) p.tile_list[off++] = (uint16_t)t;
+  }
+  p.cta_off[grid] = (uint16_t)off;
+  p.listed = 1;
+}
+
 int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream) {
   if (count < 1 || count > kGvMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
@@ -728,7 +763,7 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
   for (int i = 0; i < count; ++i)
     if (!Wq[i] || !A[i] || !Y[i]) return Q4_ERR_ARG;
   const DeviceInfo di = device_info();
-  static thread_local GemmParams p;  // host staging of the kernel parameters (~5 KB)
+  static thread_local GemmParams p;  // host staging of the kernel parameters (~10 KB)
   memset(&p, 0, sizeof(p));
   int rc = Q4_OK;
   int64_t tiles = 0;
@@ -791,6 +826,7 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     }
     p.log2_bs = __builtin_ctz((unsigned)Wq[0]->blocksize);
     p.scale_f16 = Wq[0]->scale_f16;
+    gemm_balance(p, count, std::min<int64_t>(tiles, di.sms));
     p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
     rc = run_gemm(a_dtype, mode, p, di.sms, (cudaStream_t)stream);
