@@ -334,7 +334,9 @@ template <int R> struct GsShape {
 // groups per compute warp.
 template <int DA, int NT, int B, int R>
 __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(const __grid_constant__ GsParams p) {
-  pdl_launch_then_wait();
+  // set-up (barriers, matrix fields, table, tensor-map prefetch) overlaps
+  // the previous kernel; each warp waits for it before touching global memory
+  pdl_launch_dependents();
   constexpr int WARPS = GsShape<R>::kWarps;
   constexpr int PRODUCER = WARPS;
   constexpr bool EXACT = (DA == Q4_BF16);
@@ -378,7 +380,10 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   SA = min(SA, S);
   const uint32_t rb_adj = rb - (uint32_t)SA * STAGE;  // stage s >= SA at rb_adj + s * STAGE
   if (S < 4 || hi > end) {  // not reachable with this launch's shared-memory size; refuse loudly
-    if (threadIdx.x == 0) raise_status(p.status, Q4_STATUS_LAYOUT);
+    if (threadIdx.x == 0) {
+      pdl_wait();
+      raise_status(p.status, Q4_STATUS_LAYOUT);
+    }
     return;
   }
   auto stage_addr = [&](int s) { return (s < SA ? ra : rb_adj) + (uint32_t)s * STAGE; };
@@ -429,7 +434,12 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
 
   if (warp == PRODUCER) {
     // ------------------------------------------------------------ producer
+    if (lane < p.count) {
+      prefetch_tensormap(&p.mat[lane].tmW);
+      prefetch_tensormap(&p.mat[lane].tmA);
+    }
     if (lane == 0) {
+      pdl_wait();
       const uint32_t tx = (uint32_t)kGsWTile + 2u * 128u * (uint32_t)M;
       int s = 0, mi = 0, issued = 0;
       uint32_t ph = 0;
@@ -472,15 +482,8 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   }
 
   // -------------------------------------------------------------- compute warps
-  // the first unit's c~ inputs are loaded before the table is built
-  int mi = 0;
-  GsScaleIn sin[R];
-  GsUnit u;
-  if (g0 < g1) {
-    u = gs_describe<B>(info, p.count, mi, g0, g0, g1);
-#pragma unroll
-    for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
-  }
+  // the table (launch parameters only) first, then the first unit's c~
+  // inputs once the previous kernel has finished
   for (int i = tid; i < 256 * 32; i += WARPS * 32) {
     const int b = i >> 5, l = i & 31;
     const uint32_t a = lut + (uint32_t)b * 256u + (uint32_t)l * ES;
@@ -489,6 +492,15 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   }
   // the table is complete for every compute warp (the producer does not wait)
   asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32) : "memory");
+  pdl_wait();
+  int mi = 0;
+  GsScaleIn sin[R];
+  GsUnit u;
+  if (g0 < g1) {
+    u = gs_describe<B>(info, p.count, mi, g0, g0, g1);
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
+  }
 
   const uint32_t lb = lut + ES * (uint32_t)lane;
   uint32_t sb = 0;  // c~ buffer parity
@@ -727,6 +739,20 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   // ---- count this CTA's partial tiles; finish every 16-row group it completes
   fence_acq_rel_gpu();  // this thread's slot stores are visible before its count
   __syncwarp();
+  // lane 0 counts every partial row group of the warp at once (the atomics
+  // are in flight together), then each one is checked for completion
+  unsigned olds[2][R];
+#pragma unroll
+  for (int rl = 0; rl < 2; ++rl)
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) {
+      olds[rl][rt] = 0u;
+      const int pmi = rl ? pend_mi1 : pend_mi0;
+      if (pmi < 0 || lane != 0) continue;
+      const GsInfo &mt = info[pmi];
+      const int r_base = (rl ? pend_tile1 : pend_tile0) * kGsRows + warp * 16 * R + rt * 16;
+      if (r_base < mt.N) olds[rl][rt] = atomicAdd(mt.cnt + (r_base >> 4), (unsigned)(rl ? pend_len1 : pend_len0));
+    }
 #pragma unroll
   for (int rl = 0; rl < 2; ++rl) {
     const int pmi = rl ? pend_mi1 : pend_mi0;
@@ -740,9 +766,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
     for (int rt = 0; rt < R; ++rt) {
       const int r_base = tile * kGsRows + warp * 16 * R + rt * 16;
       if (r_base >= N) continue;
-      unsigned old = 0;
-      if (lane == 0) old = atomicAdd(mt.cnt + (r_base >> 4), len);
-      old = __shfl_sync(0xffffffffu, old, 0);
+      const unsigned old = __shfl_sync(0xffffffffu, olds[rl][rt], 0);
       if (old + len != (unsigned)Q) continue;
       // every contributor has counted: sum their slots in CTA order
       __syncwarp();

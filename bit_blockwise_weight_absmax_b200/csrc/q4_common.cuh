@@ -16,10 +16,18 @@ namespace q4 {
 // the previous kernel of the stream drains.  It first lets the next kernel
 // start launching, then waits until the previous one has completed and its
 // memory operations are visible, before touching global memory.
-__device__ __forceinline__ void pdl_launch_then_wait() {
+__device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_then_wait() {
+  pdl_launch_dependents();
+  pdl_wait();
+}
+// A kernel whose set-up reads neither global memory nor anything the
+// previous kernel writes (shared-memory tables, barrier init, tensor-map
+// prefetch) runs it between the two: it then overlaps the previous kernel's
+// last CTAs, and each thread calls pdl_wait() before its first global access.
 
 __device__ __forceinline__ void raise_status(int *status, int bit) {
   if (status) atomicOr(status, bit);
