@@ -151,7 +151,7 @@ __device__ __forceinline__ void dq_emit(const DqGMat &m, int64_t base, int lane,
 // lies, are in flight while the current one is expanded).
 template <int QT, int DOUT, int B, bool DQ>
 __global__ void __launch_bounds__(kDqThreads, 1) dequantize_kernel(const __grid_constant__ DequantGroupParams p) {
-  pdl_launch_then_wait();
+  pdl_launch_dependents();  // the table below is built while the previous kernel drains
   static_assert(B % 8 == 0, "a chunk never straddles two blocks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int lane = threadIdx.x & 31;
@@ -167,6 +167,7 @@ __global__ void __launch_bounds__(kDqThreads, 1) dequantize_kernel(const __grid_
                  : "memory");
   }
   __syncthreads();
+  pdl_wait();
   const uint32_t lb = lut + 8u * (uint32_t)lane;
   const int wpb = kDqThreads / 32;
   const int64_t stride = (int64_t)gridDim.x * wpb;

@@ -260,7 +260,7 @@ constexpr int kGemmPlain = 0, kGemmDq = 1, kGemmAsym = 2;
 template <int DA, int MODE>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool DQ = MODE == kGemmDq, ASYM = MODE == kGemmAsym;
-  pdl_launch_then_wait();
+  pdl_launch_dependents();  // set-up (barriers, TMEM, level table) overlaps the previous kernel
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *sA = smem;                                        // [stages][32 KB]
@@ -301,9 +301,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                  "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  if (warp == 0 && lane < p.count) {
+    prefetch_tensormap(&p.mat[lane].tmA);
+    prefetch_tensormap(&p.mat[lane].tmW);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = s_tmem;
   volatile int *abort = &s_abort;
   // this CTA's tiles: a host-balanced list, or every gridDim.x-th tile

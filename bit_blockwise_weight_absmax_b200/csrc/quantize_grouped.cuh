@@ -109,7 +109,7 @@ __device__ __forceinline__ double qg_matrix_sum(const double *src, int64_t n, do
 
 template <int DT, int QT, int B, bool DQ>
 __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const __grid_constant__ QuantGroupParams p) {
-  pdl_launch_then_wait();
+  pdl_launch_dependents();  // the set-up below overlaps the previous kernel
   static_assert(B % 32 == 0 && B <= 256, "half a slice covers an even number of whole blocks");
   constexpr int LPB = B / 16;                                  // lanes per block
   constexpr int64_t CHUNK = (int64_t)kChunkBlocks * B;         // weights per chunk
@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(kQgThreads, 1) quantize_grouped_kernel(const _
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  pdl_wait();
 
   if (warp == kQgWarps) {
     // ------------------------------------------------------------ producer
