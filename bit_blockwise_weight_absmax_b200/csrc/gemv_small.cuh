@@ -29,7 +29,9 @@
 //   * 16 compute warps own 16 rows each (the MMA rows; swap-AB) and read
 //     their bytes and the activation rows from the ring without conflicts;
 //     the two halves of a stage are independent chains (more work in flight
-//     per warp, half the barrier traffic of 64-k stages);
+//     per warp, half the barrier traffic of 64-k stages); a warp holds the
+//     activation fragments of one 64-k segment at a time, which keeps every
+//     batch size within the 96 registers a thread gets with 17 warps;
 //   * a byte maps to the pair of its two codebook values through a
 //     256-entry table in shared memory (one copy per lane) placed at a
 //     64 KB-aligned shared address, so a single PRMT forms the address
@@ -510,14 +512,11 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   int pend_mi1 = -1, pend_tile1 = 0, pend_len1 = 0;
   float acc[R][NT][4];
   int qstart = 0;
-  uint32_t av[NT][SEGS][SEG / 8];
+  uint32_t av[NT][SEG / 8];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int sg = 0; sg < SEGS; ++sg)
-#pragma unroll
-      for (int i = 0; i < SEG / 8; ++i) av[nt][sg][i] = 0u;
-  }
+    for (int i = 0; i < SEG / 8; ++i) av[nt][i] = 0u;
   int s = 0;
   uint32_t ph = 0;
 
@@ -616,31 +615,27 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
             }
           }
         }
-      // activation rows nt*8 + g (< M only; the rest stay zero): 128-byte swizzle
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int ar = nt * 8 + g;
-        if (ar < M) {
+      for (int sg = 0; sg < SEGS; ++sg) {
+        if (q * kGsStageK + sg * SEG >= K) break;
+        // this segment's activation rows nt*8 + g (< M only; the rest stay zero): 128-byte swizzle
 #pragma unroll
-          for (int sg = 0; sg < SEGS; ++sg) {
-            const uint32_t aa = st + (uint32_t)(sg / SPH) * ATILE + (uint32_t)ar * 128u;  // the segment's half
+        for (int nt = 0; nt < NT; ++nt) {
+          const int ar = nt * 8 + g;
+          if (ar < M) {
+            const uint32_t aa = st + (uint32_t)(sg / SPH) * ATILE + (uint32_t)ar * 128u;
             const int sgh = sg % SPH;
             if constexpr (SEG == 64) {
               const uint4 x0 = lds128v(aa + (((2 * tig) ^ (ar & 7)) << 4));
               const uint4 x1 = lds128v(aa + (((2 * tig + 1) ^ (ar & 7)) << 4));
-              av[nt][sg][0] = x0.x; av[nt][sg][1] = x0.y; av[nt][sg][2] = x0.z; av[nt][sg][3] = x0.w;
-              av[nt][sg][4] = x1.x; av[nt][sg][5] = x1.y; av[nt][sg][6] = x1.z; av[nt][sg][7] = x1.w;
+              av[nt][0] = x0.x; av[nt][1] = x0.y; av[nt][2] = x0.z; av[nt][3] = x0.w;
+              av[nt][4] = x1.x; av[nt][5] = x1.y; av[nt][6] = x1.z; av[nt][7] = x1.w;
             } else {
               const uint4 x0 = lds128v(aa + (((sgh * 4 + tig) ^ (ar & 7)) << 4));
-              av[nt][sg][0] = x0.x; av[nt][sg][1] = x0.y; av[nt][sg][2] = x0.z; av[nt][sg][3] = x0.w;
+              av[nt][0] = x0.x; av[nt][1] = x0.y; av[nt][2] = x0.z; av[nt][3] = x0.w;
             }
           }
         }
-      }
-
-#pragma unroll
-      for (int sg = 0; sg < SEGS; ++sg) {
-        if (q * kGsStageK + sg * SEG >= K) break;
         // block of this segment within the 16-block window
         const int bw = ((q * kGsStageK + sg * SEG) / B) & (kGsWinBlocks - 1);
         const uint32_t soff = EXACT ? (uint32_t)bw * 64u : (uint32_t)(bw >> 1) * 256u + (uint32_t)(bw & 1) * 64u;
@@ -665,7 +660,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
               a3 = Dt<DA>::pack2(__fmul_rn(sc.y, e3.x), __fmul_rn(sc.y, e3.y));
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt)
-                MmaS<DA>::run(acc[rt][nt], a0, a1, a2, a3, av[nt][sg][2 * qq], av[nt][sg][2 * qq + 1]);
+                MmaS<DA>::run(acc[rt][nt], a0, a1, a2, a3, av[nt][2 * qq], av[nt][2 * qq + 1]);
             } else {
               a0 = lut32(lut_addr(w0, b0 & 3, lb));
               a1 = lut32(lut_addr(w1, b0 & 3, lb));
@@ -673,8 +668,8 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
               a3 = lut32(lut_addr(w1, b1 & 3, lb));
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
-                if (qq == 0) MmaS<DA>::run0(part[nt], a0, a1, a2, a3, av[nt][sg][0], av[nt][sg][1]);
-                else MmaS<DA>::run(part[nt], a0, a1, a2, a3, av[nt][sg][2 * qq], av[nt][sg][2 * qq + 1]);
+                if (qq == 0) MmaS<DA>::run0(part[nt], a0, a1, a2, a3, av[nt][0], av[nt][1]);
+                else MmaS<DA>::run(part[nt], a0, a1, a2, a3, av[nt][2 * qq], av[nt][2 * qq + 1]);
               }
             }
           }

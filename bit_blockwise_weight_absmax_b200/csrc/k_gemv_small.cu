@@ -11,9 +11,12 @@ namespace {
 // kernel lays out its table, buffers and ring itself).
 template <int DA, int NT, int B>
 int go_small(const GsParams &p, int sms, cudaStream_t st) {
-  // 16-row groups per compute warp: M <= 8 fits 16 compute warps (+ the
-  // producer) in the registers; M <= 16 uses 8 warps of 32 rows
-  constexpr int R = NT == 1 ? 1 : 2;
+  // 16-row groups per compute warp: one, so 16 compute warps (+ the
+  // producer), wherever that fits the 96 registers 17 warps leave a thread
+  // (per-scheduler register file) without spilling: every binary16 case and
+  // bf16 up to M = 8 (at M = 16, 8 warps of 32 rows were 9% slower for
+  // binary16).  bf16 at 9 <= M <= 16 keeps 8 warps of 32 rows.
+  constexpr int R = (DA == Q4_BF16 && NT == 2) ? 2 : 1;
   constexpr auto kern = gemv_small_kernel<DA, NT, B, R>;
   if (set_smem_attr_once<kern>(kGsSmemBytes, true) != Q4_OK) return Q4_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(p.total_stages, (int64_t)std::min(sms, kGsMaxCtas));
