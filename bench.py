@@ -307,7 +307,7 @@ def run_gpu(args, rank, world, local_rank):
     # one grouped launch per layer (quantize: plus its second-level launch)
     launches = {"quantize": L * 2, "dequantize": L, "gemm": L}
     for M in DECODE_M:
-        launches[f"gemv_m{M}"] = L * (1 if M <= 16 else 2)
+        launches[f"gemv_m{M}"] = L
     launches_per_step = sum(launches.values())
     if args.profile:
         # a short eager run of one phase for a profiler capture (no timing)

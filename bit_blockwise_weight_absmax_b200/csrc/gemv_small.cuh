@@ -1,6 +1,6 @@
 // gemv_small.cuh -- fused 4-bit dequant-GEMV for decode batches (sm_100a),
-// Y[M,N] = A[M,K] . W^[N,K]^T for 1 <= M <= 16 activation rows per launch
-// (q4_gemv runs 16 < M <= 32 as two launches).  NF4 states use the 16-level
+// Y[M,N] = A[M,K] . W^[N,K]^T for 1 <= M <= 32 activation rows in one pass
+// (one, two or four n8 column tiles).  NF4 states use the 16-level
 // codebook and the block absmax c~; INT4 symmetric states the integers -8..7
 // and the group scale.
 //

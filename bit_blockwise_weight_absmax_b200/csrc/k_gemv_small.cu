@@ -13,10 +13,11 @@ template <int DA, int NT, int B>
 int go_small(const GsParams &p, int sms, cudaStream_t st) {
   // 16-row groups per compute warp: one, so 16 compute warps (+ the
   // producer), wherever that fits the 96 registers 17 warps leave a thread
-  // (per-scheduler register file) without spilling: every binary16 case and
-  // bf16 up to M = 8 (at M = 16, 8 warps of 32 rows were 9% slower for
-  // binary16).  bf16 at 9 <= M <= 16 keeps 8 warps of 32 rows.
-  constexpr int R = (DA == Q4_BF16 && NT == 2) ? 2 : 1;
+  // (per-scheduler register file) without spilling: binary16 up to M = 16
+  // and bf16 up to M = 8 (at M = 16, 8 warps of 32 rows were 9% slower for
+  // binary16).  bf16 at 9 <= M <= 16 and every M > 16 (four column tiles)
+  // use 8 warps of 32 rows.
+  constexpr int R = (NT == 4 || (DA == Q4_BF16 && NT == 2)) ? 2 : 1;
   constexpr auto kern = gemv_small_kernel<DA, NT, B, R>;
   if (set_smem_attr_once<kern>(kGsSmemBytes, true) != Q4_OK) return Q4_ERR_CUDA;
   const int grid = (int)std::min<int64_t>(p.total_stages, (int64_t)std::min(sms, kGsMaxCtas));
@@ -36,7 +37,8 @@ int small_bs(int bs, const GsParams &p, int sms, cudaStream_t st) {
 template <int DA>
 int small_m(int M, int bs, const GsParams &p, int sms, cudaStream_t st) {
   if (M <= 8) return small_bs<DA, 1>(bs, p, sms, st);
-  return small_bs<DA, 2>(bs, p, sms, st);
+  if (M <= 16) return small_bs<DA, 2>(bs, p, sms, st);
+  return small_bs<DA, 4>(bs, p, sms, st);
 }
 }  // namespace
 

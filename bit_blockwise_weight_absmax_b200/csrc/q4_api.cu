@@ -142,28 +142,27 @@ int check_state(const q4_state *s) {
 }
 
 // ---- GEMV planning ----------------------------------------------------------
-// NF4 and INT4 symmetric states run the decode kernel of gemv_small.cuh: it
-// takes M <= 16 rows of activations; 16 < M <= 32 runs it twice (rows 0..15,
-// then the rest).  Tiles of 256 rows cut into 128-k stages, the stages of
-// all matrices split evenly over at most kGsMaxCtas CTAs.  Workspace: a
+// NF4 and INT4 symmetric states run the decode kernel of gemv_small.cuh in
+// one pass for every M <= 32 (one, two or four column tiles of 8 activation
+// rows).  Tiles of 256 rows cut into 128-k stages, the stages of all
+// matrices split evenly over at most kGsMaxCtas CTAs.  Workspace: a
 // 256-byte head, the per-CTA partial-row slots, then per matrix one counter
-// per 16 rows; both passes reuse it.
+// per 16 rows.
 // INT4 asymmetric states run the one-pass kernel of gemv.cuh for every M:
 // units are (tile of 256 rows, 256-k chunk) pairs cut evenly over at most
 // min(SMs, kGvMaxCtas) CTAs; the same workspace layout with slots of 8, 16 or
 // 32 columns.  Either kernel leaves the whole workspace zeroed.
 constexpr size_t kGemvWsHead = 256;
-constexpr int kGemvPassRows = 16;
 size_t gemv_counters_for(const q4_state *s) { return align256((size_t)ceil_div(s->rows, 16) * 4); }
 size_t gemv_ws_for(const q4_state *s, int64_t *n_tiles, int64_t *n_stages) {
   *n_tiles = ceil_div(s->rows, kGsRows);
   *n_stages = ceil_div(s->cols, kGsStageK);  // stages per tile
   return gemv_counters_for(s);
 }
-// Slots of the decode kernel: [grid][2][256 rows][8 or 16] fp32.
+// Slots of the decode kernel: [grid][2][256 rows][8, 16 or 32] fp32.
 size_t gemv_small_slots(int64_t total_stages, int64_t M) {
   const int64_t grid = std::min<int64_t>(total_stages, kGsMaxCtas);
-  return align256((size_t)grid * 2 * kGsRows * (M <= 8 ? 8 : 16) * 4);
+  return align256((size_t)grid * 2 * kGsRows * (M <= 8 ? 8 : (M <= 16 ? 16 : 32)) * 4);
 }
 // The one-pass kernel (INT4 asymmetric): activation tiles and slots.
 inline int gemv_nt(int64_t M) { return M <= 8 ? 1 : (M <= 16 ? 2 : 4); }
@@ -677,7 +676,7 @@ int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
     }
   }
   total += Wq[0]->qtype == Q4_INT4_ASYM ? gemv_slots_for(units, M)
-                                        : gemv_small_slots(units, std::min<int64_t>(M, kGemvPassRows));
+                                        : gemv_small_slots(units, M);
   *bytes = total;
   return Q4_OK;
 }
@@ -695,21 +694,7 @@ int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *
     if (Wq[i]->qtype != Wq[0]->qtype || Wq[i]->scale_f16 != Wq[0]->scale_f16) return Q4_ERR_ARG;
   if (Wq[0]->qtype == Q4_INT4_ASYM)
     return gemv_grouped_impl(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
-  if (M <= kGemvPassRows)
-    return gemv_small_grouped(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
-  // two passes of the decode kernel: activation rows 0..15, then 16..M-1
-  int rc = gemv_small_grouped(count, A, Wq, Y, kGemvPassRows, a_dtype, y_dtype, workspace, workspace_bytes,
-                              stream);
-  if (rc != Q4_OK) return rc;
-  const void *A2[kGsMaxGroup];
-  void *Y2[kGsMaxGroup];
-  const size_t ysize = y_dtype == Q4_F32 ? 4 : 2;
-  for (int i = 0; i < count; ++i) {
-    A2[i] = static_cast<const char *>(A[i]) + (size_t)kGemvPassRows * (size_t)Wq[i]->cols * 2;
-    Y2[i] = static_cast<char *>(Y[i]) + (size_t)kGemvPassRows * (size_t)Wq[i]->rows * ysize;
-  }
-  return gemv_small_grouped(count, A2, Wq, Y2, M - kGemvPassRows, a_dtype, y_dtype, workspace, workspace_bytes,
-                            stream);
+  return gemv_small_grouped(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
 }
 
 int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,

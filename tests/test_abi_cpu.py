@@ -155,10 +155,9 @@ def _gemv(lib, states, M):
 
 
 def test_gemv_workspace_sizes_per_format(lib):
-    """NF4 / INT4 symmetric: 16 < M <= 32 runs the decode kernel twice on one
-    workspace, so every such M needs the 16-row size (slots of 16 columns)
-    and M <= 8 less (8 columns).  INT4 asymmetric runs one pass for every M:
-    its slots hold 8, 16 or 32 columns.  M outside 1..32 is refused."""
+    """Both decode kernels run one pass for every M <= 32: their slots hold
+    8, 16 or 32 columns (M <= 8, <= 16, <= 32).  M outside 1..32 is
+    refused."""
     from bit_blockwise_weight_absmax_b200 import q4
 
     def sizes(qt, bs, dq):
@@ -174,7 +173,7 @@ def test_gemv_workspace_sizes_per_format(lib):
         assert lib.q4_gemv_workspace_size(2, arr, 0, ctypes.byref(out)) == -2
         return size
     nf4 = sizes(0, 64, True)
-    assert nf4(1) == nf4(8) < nf4(9) == nf4(16) == nf4(17) == nf4(32)
+    assert nf4(1) == nf4(8) < nf4(9) == nf4(16) < nf4(17) == nf4(32)
     asym = sizes(2, 128, False)
     assert asym(1) == asym(8) < asym(9) == asym(16) < asym(17) == asym(32)
 

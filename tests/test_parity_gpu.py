@@ -306,7 +306,7 @@ def test_gemv_grouped_7b_layer(q4, oracle):
 def test_gemv_repeat_calls_are_bit_identical(q4, oracle):
     """The split-K partial sums are added in a fixed order and the workspace
     is left zeroed: identical calls give identical bits, at every batch size
-    and output type (17..32 rows run two passes on one workspace)."""
+    and output type (17..32 rows use four column tiles)."""
     g = torch.Generator().manual_seed(6)
     W = dev(torch.randn(4096, 11008, generator=g).mul(0.02).bfloat16())
     st = q4.quantize(W, 64, "nf4", True)
