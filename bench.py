@@ -49,7 +49,7 @@ NCU_TRAFFIC = {
     "gemm": ("bit_blockwise_weight_absmax_b200/csrc/gemm.cuh",
              "c4a3b94c1237b0f11845950e5df0f07ce0300188897b1847880f8e69cd2406d3", 147_771_392 + 30_718_976),
     "gemv": ("bit_blockwise_weight_absmax_b200/csrc/gemv_small.cuh",
-             "b62b4d6130cb8eaca57e0fc21062f07a2fcc1e74e08369c46921f827d7578652", 108_837_376 + 4_373_504),
+             "856d17a0f493cbdab108afa2c2985ce7e59ef010933746be3b4ab05d02e495a6", 108_892_672 + 4_189_952),
 }
 
 
