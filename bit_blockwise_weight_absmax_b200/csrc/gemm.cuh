@@ -226,15 +226,13 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 }
 
 // 32 lanes x 32 consecutive fp32 columns of TMEM -> 32 registers per thread.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// 16 fp32 accumulator columns of this warp's 32 TMEM lanes (one lane per
+// thread); 16 at a time keeps the epilogue within the kernel's registers.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -415,28 +413,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const int h = piece / (kGemmBN / 128), part = piece % (kGemmBN / 128);
           const int mrow = tc.tm * kGemmBM + h * 128 + q * 32 + lane;
           const int col0 = cc * (kGemmBN / 4) + part * 32;
-          uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((ab * kGemmAccs + h) * kGemmBN + col0), r);
-          const int n0 = tc.tn * kGemmBN + col0;
-          if (mrow < m.M && n0 < m.N) {
-            if (p.y_dtype == Q4_F32) {
-              float *y = reinterpret_cast<float *>(m.Y) + (int64_t)mrow * m.N + n0;
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {  // 16 columns per tcgen05.ld
+            const int c16 = col0 + 16 * hh;
+            uint32_t r[16];
+            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((ab * kGemmAccs + h) * kGemmBN + c16), r);
+            const int n0 = tc.tn * kGemmBN + c16;
+            if (mrow < m.M && n0 < m.N) {
+              if (p.y_dtype == Q4_F32) {
+                float *y = reinterpret_cast<float *>(m.Y) + (int64_t)mrow * m.N + n0;
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                if (n0 + 4 * v < m.N)
-                  *reinterpret_cast<uint4 *>(y + 4 * v) = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-            } else {
-              uint16_t *y = reinterpret_cast<uint16_t *>(m.Y) + (int64_t)mrow * m.N + n0;
+                for (int v = 0; v < 4; ++v)
+                  if (n0 + 4 * v < m.N)
+                    *reinterpret_cast<uint4 *>(y + 4 * v) = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+              } else {
+                uint16_t *y = reinterpret_cast<uint16_t *>(m.Y) + (int64_t)mrow * m.N + n0;
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                if (n0 + 8 * v < m.N) {
-                  uint32_t o[4];
+                for (int v = 0; v < 2; ++v) {
+                  if (n0 + 8 * v < m.N) {
+                    uint32_t o[4];
 #pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const float f0 = __uint_as_float(r[8 * v + 2 * e]), f1 = __uint_as_float(r[8 * v + 2 * e + 1]);
-                    o[e] = (p.y_dtype == Q4_BF16) ? Dt<Q4_BF16>::pack2(f0, f1) : Dt<Q4_F16>::pack2(f0, f1);
+                    for (int e = 0; e < 4; ++e) {
+                      const float f0 = __uint_as_float(r[8 * v + 2 * e]), f1 = __uint_as_float(r[8 * v + 2 * e + 1]);
+                      o[e] = (p.y_dtype == Q4_BF16) ? Dt<Q4_BF16>::pack2(f0, f1) : Dt<Q4_F16>::pack2(f0, f1);
+                    }
+                    *reinterpret_cast<uint4 *>(y + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
                   }
-                  *reinterpret_cast<uint4 *>(y + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
               }
             }
