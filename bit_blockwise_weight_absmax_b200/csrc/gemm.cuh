@@ -548,7 +548,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         }
         const int blk = ((kk + kGemmCodes * qk) >> lbs) & 15;  // this thread's block in the window
         const float sc = scrow[blk];
-        const float zf = ASYM ? (float)zrow[blk] : 0.0f;
+        const uint64_t sc2 = f2_pack(sc, sc);
+        const float nz = ASYM ? -(float)zrow[blk] : 0.0f;
+        const uint64_t nz2 = f2_pack(nz, nz);
         // lane 0 waits for the copy (acquire); the shuffle keeps the other
         // lanes' reads of the stage after it
         {
@@ -581,10 +583,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             // level table: entry e of this lane at lvb + e * 128
-            float l0 = lds_f32((__byte_perm(lo, 0u, 0x4440u | j) << 7) + lvb);
-            float l1 = lds_f32((__byte_perm(hi, 0u, 0x4440u | j) << 7) + lvb);
-            if constexpr (ASYM) l0 = __fsub_rn(l0, zf), l1 = __fsub_rn(l1, zf);  // q - z, exact
-            o[j] = Dt<DA>::pack2(__fmul_rn(sc, l0), __fmul_rn(sc, l1));
+            const float l0 = lds_f32((__byte_perm(lo, 0u, 0x4440u | j) << 7) + lvb);
+            const float l1 = lds_f32((__byte_perm(hi, 0u, 0x4440u | j) << 7) + lvb);
+            uint64_t l2 = f2_pack(l0, l1);
+            if constexpr (ASYM) l2 = f2_add(l2, nz2);  // q - z, exact
+            float p0, p1;  // one rounding each, as the scalar multiply
+            f2_unpack(f2_mul(sc2, l2), p0, p1);
+            o[j] = Dt<DA>::pack2(p0, p1);
           }
           const int c = (kGemmCodes / 8) * qk + c2;
           *reinterpret_cast<uint4 *>(brow + ((c ^ (d & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
