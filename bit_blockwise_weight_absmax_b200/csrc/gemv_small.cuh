@@ -2,7 +2,9 @@
 // Y[M,N] = A[M,K] . W^[N,K]^T for 1 <= M <= 32 activation rows in one pass
 // (one, two or four n8 column tiles).  NF4 states use the 16-level
 // codebook and the block absmax c~; INT4 symmetric states the integers -8..7
-// and the group scale.
+// and the group scale; INT4 asymmetric states the integers 0..15, the group
+// scale s and zero-point z (robotsatlas.com, "INT4", "How it works":
+// w^ = (q - z) s).
 //
 // What it computes: n4n.ai, "What is 4-bit quantization and why does it
 // matter?", "Why it matters for deployment" (decode at batch < 32 reads every
@@ -10,8 +12,6 @@
 // "Loading a model in 4-bit", "Where the accuracy goes" (weights dequantized
 // to the compute dtype, then a 16-bit matmul); the dequantization is fused
 // into the streaming of the packed weights.
-//
-// INT4 asymmetric states run the one-pass kernel of gemv.cuh instead.
 //
 // Design (B200, decode sizes).  At M <= 16 a tcgen05 MMA (128 x 16 x 16
 // takes ~44 cycles) would cap the kernel near the HBM rate, while the
@@ -37,7 +37,9 @@
 //     64 KB-aligned shared address, so a single PRMT forms the address
 //     (byte 1 = the packed byte, the other bytes = table base + lane);
 //   * the MMA runs on the unscaled fp16 levels and each block's fp32 partial
-//     is scaled once by its absmax c~; the k order inside a segment of
+//     is scaled once by its absmax c~ (INT4 asymmetric: s (P - z S), with
+//     P the partial over the codes q and S the activations' sum over the
+//     segment, from one more MMA of an all-ones tile); the k order inside a segment of
 //     min(B, 64) is permuted identically on both operands so that a lane
 //     reads consecutive bytes;
 //   * each warp computes the c~ of its rows for the next 16 blocks one unit
@@ -49,7 +51,8 @@
 //     completes a group sums the slots of all contributors, in CTA order,
 //     into Y and zeroes them (deterministic; nothing waits mid-stream).
 // bf16 activations multiply the exact w^ = bf16(c~ * level) (the definition
-// dequantizes to the compute dtype first), with a binary32 pair table.
+// dequantizes to the compute dtype first; INT4 asymmetric bf16(s (q - z))),
+// with a binary32 pair table.
 #pragma once
 #include <cuda.h>
 
@@ -68,7 +71,8 @@ constexpr int kGsWinBlocks = 16;                  // blocks per scale window
 constexpr int kGsScaleBuf = kGsWinBlocks * 16 * 4;        // c~ of one 16-row group's unit
 constexpr int kGsScaleBytes = (kGsRows / 16) * 2 * kGsScaleBuf;  // two per row group
 constexpr int kGsBarBytes = 2 * kGsMaxStages * 8 + 16;  // barriers + abort flag
-constexpr int kGsInfoBytes = 16 * 64;             // per-matrix fields, copied to shared memory
+constexpr int kGsInfoBytes = 16 * 80;             // per-matrix fields, copied to shared memory
+constexpr int kGsZeroBytes = (kGsRows / 16) * 2 * kGsWinBlocks * 16;  // zero-points of a window, per row group and parity
 constexpr int kGsSmemBytes = 227 * 1024;          // dynamic shared memory of a CTA
 
 struct alignas(64) GsMat {
@@ -78,6 +82,7 @@ struct alignas(64) GsMat {
   const int8_t *absmax_q;
   const float *absmax_scale;
   const float *absmax_mean;
+  const uint8_t *zero;  // INT4 asymmetric zero-points, two per byte
   void *Y;
   unsigned *cnt;    // per 16-row group: stages counted so far (zero between calls)
   uint32_t stage_begin;  // first global stage index of this matrix
@@ -94,10 +99,11 @@ struct alignas(16) GsInfo {
   const int8_t *absmax_q;
   const float *absmax_scale;
   const float *absmax_mean;
+  const uint8_t *zero;
   void *Y;
   unsigned *cnt;
 };
-static_assert(sizeof(GsInfo) == 64, "GsInfo layout");
+static_assert(sizeof(GsInfo) == 80, "GsInfo layout");
 
 struct GsParams {
   GsMat mat[kGsMaxGroup];
@@ -191,6 +197,14 @@ __device__ __forceinline__ float2 lut64f(uint32_t addr) {
   asm("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ uint32_t lds16v(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts8(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -269,9 +283,10 @@ struct GsScaleIn {
   float s2a, s2b, mu;
   int bsplit, nvalid;
   float f[8];        // fp32 absmax (no double quant)
+  uint32_t zw;       // INT4 asymmetric: zero-points of the 8 blocks, block j in bits 4j..4j+3
 };
 
-template <int B>
+template <int B, bool AZ>
 __device__ __forceinline__ void gs_scale_load(const GsInfo *info, bool dq, bool sf16, const GsUnit &u, int r0, int lane,
                                               GsScaleIn &in) {
   constexpr int W = kGsWinBlocks * B / kGsStageK;
@@ -283,10 +298,22 @@ __device__ __forceinline__ void gs_scale_load(const GsInfo *info, bool dq, bool 
   in.c0 = in.c1 = 0;
   in.s2a = in.s2b = in.mu = 0.0f;
   in.bsplit = 8;
+  in.zw = 0u;
 #pragma unroll
   for (int j = 0; j < 8; ++j) in.f[j] = 0.0f;
   if (in.nvalid == 0) return;
   const int64_t bi0 = (int64_t)row * nbk + b0;
+  if constexpr (AZ) {
+    const uint8_t *zp = mt.zero + (bi0 >> 1);
+    if (in.nvalid == 8 && (bi0 & 1) == 0 && ((uintptr_t)zp & 3) == 0) {
+      in.zw = __ldg(reinterpret_cast<const unsigned *>(zp));  // blocks bi0 .. bi0 + 7, low nibble first
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < in.nvalid)
+          in.zw |= (uint32_t)((__ldg(mt.zero + ((bi0 + j) >> 1)) >> (((bi0 + j) & 1) * 4)) & 15) << (4 * j);
+    }
+  }
   if (dq) {
     in.mu = __ldg(mt.absmax_mean);
     const int64_t g0 = bi0 >> 8;
@@ -333,8 +360,9 @@ template <int R> struct GsShape {
 };
 
 // DA: activation dtype; NT: n8 tiles (M <= 8 NT); B: blocksize; R: 16-row
-// groups per compute warp.
-template <int DA, int NT, int B, int R>
+// groups per compute warp; AZ: INT4 asymmetric (codes 0..15 with a
+// zero-point per block).
+template <int DA, int NT, int B, int R, bool AZ>
 __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(const __grid_constant__ GsParams p) {
   // set-up (barriers, matrix fields, table, tensor-map prefetch) overlaps
   // the previous kernel; each warp waits for it before touching global memory
@@ -353,7 +381,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   constexpr int STAGE = 2 * ATILE + kGsWTile;
   constexpr uint32_t ES = EXACT ? 8u : 4u;     // table entry bytes per lane
   // fp16 tables use 128 of every 256 bytes: the c~ buffers live in the gaps
-  constexpr int MISC = (EXACT ? kGsScaleBytes : 0) + kGsBarBytes + kGsInfoBytes;
+  constexpr int MISC = (EXACT ? kGsScaleBytes : 0) + kGsBarBytes + kGsInfoBytes + (AZ ? kGsZeroBytes : 0);
   static_assert(STAGE % 1024 == 0, "stage alignment");
   static_assert(EXACT || kGsScaleBytes == 256 * 128, "c~ buffers fill the table gaps");
 
@@ -395,6 +423,9 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   auto sempty = [&](int s) { return bar0 + 8u * (kGsMaxStages + s); };
   volatile int *abort = reinterpret_cast<volatile int *>(smem_raw + (bar0 + 16u * kGsMaxStages - base));
   GsInfo *info = reinterpret_cast<GsInfo *>(smem_raw + (bar0 + kGsBarBytes - base));
+  // zero-points of a window (INT4 asymmetric), per row group and parity:
+  // [block][row & 7][row >> 3] bytes, so rows g and g + 8 of a block are adjacent
+  const uint32_t zbase = bar0 + kGsBarBytes + kGsInfoBytes;
   // c~ buffer of 16-row group grp (0..15), parity sb, byte offset o < 1024:
   // contiguous (bf16) or in the 128-byte gaps of the table (fp16)
   auto scale_addr = [&](int grp, uint32_t sb, uint32_t o) -> uint32_t {
@@ -421,6 +452,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
     d.absmax_q = m.absmax_q;
     d.absmax_scale = m.absmax_scale;
     d.absmax_mean = m.absmax_mean;
+    d.zero = m.zero;
     d.Y = m.Y;
     d.cnt = m.cnt;
   }
@@ -501,7 +533,7 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   if (g0 < g1) {
     u = gs_describe<B>(info, p.count, mi, g0, g0, g1);
 #pragma unroll
-    for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
+    for (int rt = 0; rt < R; ++rt) gs_scale_load<B, AZ>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
   }
 
   const uint32_t lb = lut + ES * (uint32_t)lane;
@@ -527,12 +559,16 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
   auto joff = [](int j) -> uint32_t {
     return EXACT ? (uint32_t)j * 64u : (uint32_t)(j >> 1) * 256u + (uint32_t)(j & 1) * 64u;
   };
-  uint32_t cst[R], srd0[R];
+  uint32_t cst[R], srd0[R], zst[R], zrd0[R];
 #pragma unroll
   for (int rt = 0; rt < R; ++rt) {
     const int r = lane & 15, blk0 = (lane >> 4) * 8;
     cst[rt] = scale_addr(warp * R + rt, 0u, (uint32_t)((blk0 * 8 + (r & 7)) * 2 + (r >> 3)) * 4u);
     srd0[rt] = scale_addr(warp * R + rt, 0u, (uint32_t)g * 8u);
+    // zero-points: this lane writes block blk0 + j of row r at + 16 j, reads
+    // the (row g, row g + 8) byte pair of block bw at + 16 bw
+    zst[rt] = zbase + (uint32_t)(warp * R + rt) * 512u + (uint32_t)((blk0 * 8 + (r & 7)) * 2 + (r >> 3));
+    zrd0[rt] = zbase + (uint32_t)(warp * R + rt) * 512u + (uint32_t)g * 2u;
   }
 
   bool ok = true;
@@ -559,18 +595,27 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
           for (int j = 0; j < 8; ++j)
             sts32(cst[rt] + sb * kSbStride + joff(j), __float_as_uint(gs_scale_value(sin[rt], dq, j)));
       }
+      if constexpr (AZ) {
+#pragma unroll
+        for (int rt = 0; rt < R; ++rt)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sts8(zst[rt] + sb * 256u + 16u * j, (sin[rt].zw >> (4 * j)) & 15u);
+      }
     }
     __syncwarp();
-    uint32_t srd[R];  // this lane's (row g, row g+8) pair of block 0, per row group
+    uint32_t srd[R], zrd[R];  // this lane's (row g, row g+8) pair of block 0, per row group
 #pragma unroll
-    for (int rt = 0; rt < R; ++rt) srd[rt] = srd0[rt] + sb * kSbStride;
+    for (int rt = 0; rt < R; ++rt) {
+      srd[rt] = srd0[rt] + sb * kSbStride;
+      zrd[rt] = zrd0[rt] + sb * 256u;
+    }
     sb ^= 1u;
     const GsUnit cu = u;
     const uint32_t gn = gi + (uint32_t)(cu.q1 - cu.q0);
     if (gn < g1) {  // next unit: issue its c~ loads now, use them a unit later
       u = gs_next<B>(info, p.count, cu, gn, g0, g1);
 #pragma unroll
-      for (int rt = 0; rt < R; ++rt) gs_scale_load<B>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
+      for (int rt = 0; rt < R; ++rt) gs_scale_load<B, AZ>(info, dq, sf16, u, (warp * R + rt) * 16, lane, sin[rt]);
     }
     const GsInfo &mt = info[cu.mi];
     const int K = mt.K, N = mt.N;
@@ -639,9 +684,28 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
         // block of this segment within the 16-block window
         const int bw = ((q * kGsStageK + sg * SEG) / B) & (kGsWinBlocks - 1);
         const uint32_t soff = EXACT ? (uint32_t)bw * 64u : (uint32_t)(bw >> 1) * 256u + (uint32_t)(bw & 1) * 64u;
+        // INT4 asymmetric, binary16: the activations' sum over the segment,
+        // S, in the accumulator layout (an all-ones A tile)
+        float csum[NT][4];
+        if constexpr (AZ && !EXACT) {
+          constexpr uint32_t kOne = 0x3C003C00u;  // binary16 1.0, twice
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int qq = 0; qq < STEPS; ++qq) {
+              if (qq == 0) MmaS<DA>::run0(csum[nt], kOne, kOne, kOne, kOne, av[nt][0], av[nt][1]);
+              else MmaS<DA>::run(csum[nt], kOne, kOne, kOne, kOne, av[nt][2 * qq], av[nt][2 * qq + 1]);
+            }
+        }
 #pragma unroll
         for (int rt = 0; rt < R; ++rt) {
           const float2 sc = lds64fv(srd[rt] + soff);
+          float z0 = 0.0f, z1 = 0.0f;  // zero-points of rows g and g + 8 (INT4 asymmetric)
+          if constexpr (AZ) {
+            const uint32_t zz = lds16v(zrd[rt] + 16u * (uint32_t)bw);
+            z0 = (float)(zz & 0xFFu);
+            z1 = (float)(zz >> 8);
+          }
           float part[NT][4];
 #pragma unroll
           for (int qq = 0; qq < STEPS; ++qq) {
@@ -654,10 +718,17 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
               const float2 e1 = lut64f(lut_addr(w1, b0 & 3, lb));
               const float2 e2 = lut64f(lut_addr(w0, b1 & 3, lb));
               const float2 e3 = lut64f(lut_addr(w1, b1 & 3, lb));
-              a0 = Dt<DA>::pack2(__fmul_rn(sc.x, e0.x), __fmul_rn(sc.x, e0.y));
-              a1 = Dt<DA>::pack2(__fmul_rn(sc.y, e1.x), __fmul_rn(sc.y, e1.y));
-              a2 = Dt<DA>::pack2(__fmul_rn(sc.x, e2.x), __fmul_rn(sc.x, e2.y));
-              a3 = Dt<DA>::pack2(__fmul_rn(sc.y, e3.x), __fmul_rn(sc.y, e3.y));
+              if constexpr (AZ) {  // (q - z) s, q - z exact
+                a0 = Dt<DA>::pack2(__fmul_rn(sc.x, __fsub_rn(e0.x, z0)), __fmul_rn(sc.x, __fsub_rn(e0.y, z0)));
+                a1 = Dt<DA>::pack2(__fmul_rn(sc.y, __fsub_rn(e1.x, z1)), __fmul_rn(sc.y, __fsub_rn(e1.y, z1)));
+                a2 = Dt<DA>::pack2(__fmul_rn(sc.x, __fsub_rn(e2.x, z0)), __fmul_rn(sc.x, __fsub_rn(e2.y, z0)));
+                a3 = Dt<DA>::pack2(__fmul_rn(sc.y, __fsub_rn(e3.x, z1)), __fmul_rn(sc.y, __fsub_rn(e3.y, z1)));
+              } else {
+                a0 = Dt<DA>::pack2(__fmul_rn(sc.x, e0.x), __fmul_rn(sc.x, e0.y));
+                a1 = Dt<DA>::pack2(__fmul_rn(sc.y, e1.x), __fmul_rn(sc.y, e1.y));
+                a2 = Dt<DA>::pack2(__fmul_rn(sc.x, e2.x), __fmul_rn(sc.x, e2.y));
+                a3 = Dt<DA>::pack2(__fmul_rn(sc.y, e3.x), __fmul_rn(sc.y, e3.y));
+              }
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt)
                 MmaS<DA>::run(acc[rt][nt], a0, a1, a2, a3, av[nt][2 * qq], av[nt][2 * qq + 1]);
@@ -680,6 +751,16 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
               acc[rt][nt][1] = fmaf(sc.x, part[nt][1], acc[rt][nt][1]);
               acc[rt][nt][2] = fmaf(sc.y, part[nt][2], acc[rt][nt][2]);
               acc[rt][nt][3] = fmaf(sc.y, part[nt][3], acc[rt][nt][3]);
+            }
+            if constexpr (AZ) {  // - z s S
+              const float n0 = -z0 * sc.x, n1 = -z1 * sc.y;
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                acc[rt][nt][0] = fmaf(n0, csum[nt][0], acc[rt][nt][0]);
+                acc[rt][nt][1] = fmaf(n0, csum[nt][1], acc[rt][nt][1]);
+                acc[rt][nt][2] = fmaf(n1, csum[nt][2], acc[rt][nt][2]);
+                acc[rt][nt][3] = fmaf(n1, csum[nt][3], acc[rt][nt][3]);
+              }
             }
           }
         }

@@ -142,16 +142,12 @@ int check_state(const q4_state *s) {
 }
 
 // ---- GEMV planning ----------------------------------------------------------
-// NF4 and INT4 symmetric states run the decode kernel of gemv_small.cuh in
-// one pass for every M <= 32 (one, two or four column tiles of 8 activation
-// rows).  Tiles of 256 rows cut into 128-k stages, the stages of all
-// matrices split evenly over at most kGsMaxCtas CTAs.  Workspace: a
-// 256-byte head, the per-CTA partial-row slots, then per matrix one counter
-// per 16 rows.
-// INT4 asymmetric states run the one-pass kernel of gemv.cuh for every M:
-// units are (tile of 256 rows, 256-k chunk) pairs cut evenly over at most
-// min(SMs, kGvMaxCtas) CTAs; the same workspace layout with slots of 8, 16 or
-// 32 columns.  Either kernel leaves the whole workspace zeroed.
+// Every format runs the decode kernel of gemv_small.cuh in one pass for
+// every M <= 32 (one, two or four column tiles of 8 activation rows).
+// Tiles of 256 rows cut into 128-k stages, the stages of all matrices split
+// evenly over at most kGsMaxCtas CTAs.  Workspace: a 256-byte head, the
+// per-CTA partial-row slots, then per matrix one counter per 16 rows; the
+// kernel leaves all of it zeroed.
 constexpr size_t kGemvWsHead = 256;
 size_t gemv_counters_for(const q4_state *s) { return align256((size_t)ceil_div(s->rows, 16) * 4); }
 size_t gemv_ws_for(const q4_state *s, int64_t *n_tiles, int64_t *n_stages) {
@@ -163,17 +159,6 @@ size_t gemv_ws_for(const q4_state *s, int64_t *n_tiles, int64_t *n_stages) {
 size_t gemv_small_slots(int64_t total_stages, int64_t M) {
   const int64_t grid = std::min<int64_t>(total_stages, kGsMaxCtas);
   return align256((size_t)grid * 2 * kGsRows * (M <= 8 ? 8 : (M <= 16 ? 16 : 32)) * 4);
-}
-// The one-pass kernel (INT4 asymmetric): activation tiles and slots.
-inline int gemv_nt(int64_t M) { return M <= 8 ? 1 : (M <= 16 ? 2 : 4); }
-size_t gemv_slots_for(int64_t total_units, int64_t M) {
-  const int nt = gemv_nt(M);
-  const int64_t grid = std::min<int64_t>(total_units, kGvMaxCtas);
-  return align256((size_t)grid * 2 * gv_tile_rows(nt) * 8 * nt * 4);
-}
-int64_t gemv_units_for(const q4_state *s, int64_t M) {
-  const int tr = gv_tile_rows(gemv_nt(M));
-  return ceil_div(s->rows, tr) * ceil_div(s->cols, kGvChunk);
 }
 
 // ---- TMA descriptors ----------------------------------------------------------------
@@ -237,11 +222,8 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
     const q4_state *s = Wq[i];
     int rc = check_state(s);
     if (rc != Q4_OK) return rc;
-    // NF4, or INT4 symmetric (its codebook: the integers -8..7); one
-    // format per grouped call
-    if ((s->qtype != Q4_NF4 && s->qtype != Q4_INT4_SYM) || s->qtype != qt || s->blocksize != bs ||
-        s->double_quant != dq)
-      return Q4_ERR_ARG;
+    // one format per grouped call
+    if (s->qtype != qt || s->blocksize != bs || s->double_quant != dq) return Q4_ERR_ARG;
     if (s->cols % bs || s->rows > INT32_MAX || s->cols > INT32_MAX) return Q4_ERR_SHAPE;
     if (!A[i] || !Y[i]) return Q4_ERR_ARG;
     if (!aligned16(A[i])) return Q4_ERR_ALIGN;
@@ -260,6 +242,7 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
     m.absmax_q = s->absmax_q;
     m.absmax_scale = s->absmax_scale;
     m.absmax_mean = s->absmax_mean;
+    m.zero = s->zero;
     m.Y = Y[i];
     m.N = (int32_t)s->rows;
     m.K = (int32_t)s->cols;
@@ -280,94 +263,16 @@ int gemv_small_grouped(int32_t count, const void *const *A, const q4_state *cons
   p.scale_f16 = Wq[0]->scale_f16;
   if (qt == Q4_NF4) {
     memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
-  } else {
+  } else if (qt == Q4_INT4_SYM) {
     // INT4 symmetric: code j is the two's-complement nibble of q, w^ = q * s
     for (int j = 0; j < 16; ++j) p.levels[j] = (float)((j ^ 8) - 8);
+  } else {
+    // INT4 asymmetric: code j is q itself, w^ = (q - z) * s
+    for (int j = 0; j < 16; ++j) p.levels[j] = (float)j;
   }
-  return run_gemv_small(a_dtype, bs, (int)M, p, di.sms, (cudaStream_t)stream);
+  return run_gemv_small(a_dtype, bs, (int)M, qt == Q4_INT4_ASYM, p, di.sms, (cudaStream_t)stream);
 }
 
-// The one-pass decode GEMV (gemv.cuh) for INT4 asymmetric states: one launch
-// for the whole group and 1 <= M <= 32.
-int gemv_grouped_impl(int32_t count, const void *const *A, const q4_state *const *Wq, void *const *Y,
-                      int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace, size_t workspace_bytes,
-                      void *stream) {
-  static thread_local GvParams p;  // host staging of the kernel parameters (~1.7 KB)
-  memset(&p, 0, sizeof(p));
-  p.count = count;
-  p.M = (int)M;
-  p.y_dtype = y_dtype;
-  const int bs = Wq[0]->blocksize;
-  const int dq = Wq[0]->double_quant;
-  const int qt = Wq[0]->qtype;
-  const int nt = gemv_nt(M);
-  const int tr = gv_tile_rows(nt);
-  int64_t total = 0;
-  for (int i = 0; i < count; ++i) {
-    const q4_state *s = Wq[i];
-    int rc = check_state(s);
-    if (rc != Q4_OK) return rc;
-    // one format per grouped call
-    if (s->qtype != qt || s->blocksize != bs || s->double_quant != dq) return Q4_ERR_ARG;
-    if (s->cols % bs || s->rows > INT32_MAX || s->cols > INT32_MAX) return Q4_ERR_SHAPE;
-    if (!aligned16(A[i])) return Q4_ERR_ALIGN;
-    total += gemv_units_for(s, M);
-  }
-  if (total * kGvMaxCtas >= ((int64_t)1 << 32)) return Q4_ERR_SHAPE;  // 32-bit unit indices
-  if (!workspace || workspace_bytes < kGemvWsHead) return Q4_ERR_WORKSPACE;
-  size_t ws_off = kGemvWsHead + gemv_slots_for(total, M);
-  if (ws_off > workspace_bytes) return Q4_ERR_WORKSPACE;
-  const DeviceInfo di = device_info();
-  if (di.ok != Q4_OK) return di.ok;
-  p.slots = reinterpret_cast<float *>((char *)workspace + kGemvWsHead);
-  uint32_t units = 0;
-  for (int i = 0; i < count; ++i) {
-    const q4_state *s = Wq[i];
-    GvInfo &m = p.mat[i].f;
-    // the packed weights [N, K/2] bytes, one 256-k chunk of a tile per box,
-    // 128-byte swizzled (conflict-free ldmatrix)
-    if (!make_map(&p.mat[i].tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1,
-                  kGvChunk / 2, tr, CU_TENSOR_MAP_SWIZZLE_128B))
-      return Q4_ERR_CUDA;
-    m.packed = s->packed;
-    m.A = reinterpret_cast<const uint16_t *>(A[i]);
-    m.Y = Y[i];
-    m.absmax = s->absmax;
-    m.absmax_q = s->absmax_q;
-    m.absmax_scale = s->absmax_scale;
-    m.absmax_mean = s->absmax_mean;
-    m.zero = s->zero;
-    m.N = (int32_t)s->rows;
-    m.K = (int32_t)s->cols;
-    m.n_tiles = (int32_t)ceil_div(s->rows, tr);
-    m.n_chunks = (int32_t)ceil_div(s->cols, kGvChunk);
-    m.unit_begin = units;
-    units += (uint32_t)(m.n_tiles * m.n_chunks);
-    const size_t need = gemv_counters_for(s);
-    if (ws_off + need > workspace_bytes) return Q4_ERR_WORKSPACE;
-    m.cnt = reinterpret_cast<unsigned *>((char *)workspace + ws_off);
-    ws_off += need;
-  }
-  p.total_units = units;
-  p.status = di.status;
-  p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-  p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
-  p.scale_f16 = Wq[0]->scale_f16;
-  int mode = kGvPlain;
-  if (qt == Q4_NF4) {
-    memcpy(p.levels, kNF4Levels, sizeof(kNF4Levels));
-    if (dq) mode = kGvDq;
-  } else if (qt == Q4_INT4_SYM) {
-    // code j is the two's-complement nibble of q, w^ = q * s
-    for (int j = 0; j < 16; ++j) p.levels[j] = (float)((j ^ 8) - 8);
-  } else {
-    // code j is q in 0..15, w^ = (q - z) * s
-    for (int j = 0; j < 16; ++j) p.levels[j] = (float)j;
-    mode = kGvAsym;
-  }
-  const int grid = (int)std::min<int64_t>(units, std::min(di.sms, kGvMaxCtas));
-  return run_gemv(a_dtype, mode, nt, bs, p, grid, (cudaStream_t)stream);
-}
 
 }  // namespace
 
@@ -657,7 +562,7 @@ int q4_dequantize_grouped(int32_t count, const q4_state *const *Wq, void *const 
 }
 
 int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {
-  if (!bytes || !Wq || count < 1 || count > kGvMaxGroup) return Q4_ERR_ARG;
+  if (!bytes || !Wq || count < 1 || count > kGsMaxGroup) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
   for (int i = 0; i < count; ++i) {
     if (!Wq[i]) return Q4_ERR_ARG;
@@ -667,16 +572,11 @@ int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
   int64_t units = 0;
   for (int i = 0; i < count; ++i) {
     total += gemv_counters_for(Wq[i]);
-    if (Wq[0]->qtype == Q4_INT4_ASYM) {
-      units += gemv_units_for(Wq[i], M);
-    } else {
-      int64_t t, q;
-      gemv_ws_for(Wq[i], &t, &q);
-      units += t * q;
-    }
+    int64_t t, q;
+    gemv_ws_for(Wq[i], &t, &q);
+    units += t * q;
   }
-  total += Wq[0]->qtype == Q4_INT4_ASYM ? gemv_slots_for(units, M)
-                                        : gemv_small_slots(units, M);
+  total += gemv_small_slots(units, M);
   *bytes = total;
   return Q4_OK;
 }
@@ -684,7 +584,7 @@ int q4_gemv_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
 int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace,
                     size_t workspace_bytes, void *stream) {
-  if (count < 1 || count > kGvMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (count < 1 || count > kGsMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (M < 1 || M > 32) return Q4_ERR_SHAPE;
   // every entry is checked before any of them is dereferenced
@@ -692,8 +592,6 @@ int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *const *
     if (!Wq[i] || !A[i] || !Y[i]) return Q4_ERR_ARG;
   for (int i = 0; i < count; ++i)  // one format per grouped call
     if (Wq[i]->qtype != Wq[0]->qtype || Wq[i]->scale_f16 != Wq[0]->scale_f16) return Q4_ERR_ARG;
-  if (Wq[0]->qtype == Q4_INT4_ASYM)
-    return gemv_grouped_impl(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
   return gemv_small_grouped(count, A, Wq, Y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
 }
 
@@ -741,7 +639,7 @@ static void gemm_balance(GemmParams &p, int count, int64_t grid) {
 
 int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream) {
-  if (count < 1 || count > kGvMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (count < 1 || count > kGsMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
   if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
   if (y_dtype != Q4_F32 && y_dtype != a_dtype) return Q4_ERR_ARG;
   if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;

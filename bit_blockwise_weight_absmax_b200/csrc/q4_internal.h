@@ -10,7 +10,6 @@
 #include "q4_common.cuh"
 #include "quantize.cuh"
 #include "dequantize.cuh"
-#include "gemv.cuh"
 #include "gemv_small.cuh"
 #include "gemm.cuh"
 #include "quantize_grouped.cuh"
@@ -65,9 +64,7 @@ int run_quantize_grouped(int dt, int qt, int bs, bool dq, const QuantGroupParams
 int run_double_quant_grouped(const DqGroupParams &p, cudaStream_t st);
 int run_dequantize(int qt, int dout, int bs, bool dq, const DequantGroupParams &p, int sms, cudaStream_t st);
 int run_gemm(int da, int mode, const GemmParams &p, int sms, cudaStream_t st);
-int run_gemv_small(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st);
-int run_gemv(int da, int mode, int nt, int bs, const GvParams &p, int grid, cudaStream_t st);
-int gv_tile_rows(int nt);
-template <int DA, int MODE>
-int run_gemv_dm(int nt, int bs, const GvParams &p, int grid, cudaStream_t st);
+int run_gemv_small(int da, int bs, int M, bool asym, const GsParams &p, int sms, cudaStream_t st);
+template <bool AZ>
+int run_gemv_small_t(int da, int bs, int M, const GsParams &p, int sms, cudaStream_t st);
 }  // namespace q4
