@@ -1,5 +1,5 @@
 """Failure detection without a GPU fault: every pipeline wait in the decode
-GEMVs and the grouped quantize is bounded by the launch's wait limit.  With
+GEMV, the GEMM and the grouped quantize is bounded by the launch's wait limit.  With
 the copy stall test hook on, the copy warp issues no copies (a flag that
 nothing sets), so every compute warp's wait for a stage must run out after
 the (short) wait limit: the call must set Q4_STATUS_TIMEOUT and return, and
@@ -16,8 +16,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("qtype,bs,dq,N,K", [("nf4", 64, True, 4096, 8192), ("int4_asym", 128, False, 4096, 8192)])
 def test_gemv_wait_limit_times_out_and_recovers(oracle, qtype, bs, dq, N, K):
-    """Both decode kernels (NF4 and INT4 symmetric run one, INT4 asymmetric
-    the other)."""
+    """The decode kernel's two instance sets: NF4 (with INT4 symmetric) and
+    INT4 asymmetric (zero-point window)."""
     from bit_blockwise_weight_absmax_b200 import build
     build.build()
     from bit_blockwise_weight_absmax_b200 import q4
