@@ -170,7 +170,20 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- CPU oracle ---
-def oracle_sample(rows_per_matrix=16, quantize_layer=True, seed=0):
+def cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), else the platform's."""
+    import platform
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def oracle_sample(rows_per_matrix=16, quantize_layer=True, seed=0, threads=None):
     """Time the oracle on a bounded sample of the same workload and scale it
     to one whole layer.  Quantize: NF4 + DQ of the full layer (all seven
     matrices) when `quantize_layer`, else of the 4096x4096 q matrix.  GEMV:
@@ -185,7 +198,7 @@ def oracle_sample(rows_per_matrix=16, quantize_layer=True, seed=0):
 
     import oracle
     from bit_blockwise_weight_absmax_b200 import workloads as wl
-    threads = oracle.set_threads(os.cpu_count() or 1)
+    threads = oracle.set_threads(threads or os.cpu_count() or 1)
     t0 = time.perf_counter()
     q_bytes, tq = 0, 0.0
     for i, (_, N, K) in enumerate(wl.LAYER_7B if quantize_layer else wl.LAYER_7B[:1]):
@@ -374,7 +387,11 @@ def run_gpu(args, rank, world, local_rank):
     ph_ms = {p: vec[2 + i] for i, p in enumerate(phases)}
 
     value = whole_job_rate(sum(gemv_B.values()), world, gemv_ms) / 1e12
+    # effective TB/s counts weights + state + A + Y; weight_tb_s the packed
+    # weights and their state alone
     per_m = {f"M={M}": {"tb_s": gemv_B[M] / (ph_ms[f"gemv_m{M}"] / 1e3) / 1e12,
+                        "weight_tb_s": gemv_B[M] * layer_state_bytes(shapes) / gemv_bytes(shapes, M)
+                                       / (ph_ms[f"gemv_m{M}"] / 1e3) / 1e12,
                         "us_per_layer": ph_ms[f"gemv_m{M}"] * 1e3 / (L * args.steps),
                         "bytes_per_layer": gemv_bytes(shapes, M)} for M in DECODE_M}
     hbm = peaks["hbm_gbs"]
@@ -548,7 +565,12 @@ def run_gpu(args, rank, world, local_rank):
     if rank == 0 and not args.no_cpu_baseline:
         tb, qg, thr, desc, secs, _ = oracle_sample(rows_per_matrix=args.cpu_rows)
         cpu = {"value": tb, "unit": UNIT, "cores": thr, "kind": "oracle", "sample": desc,
-               "quantize_gbs": qg, "seconds": round(secs, 1)}
+               "quantize_gbs": qg, "seconds": round(secs, 1), "cpu_model": cpu_model()}
+        # the same oracle on one thread, on a smaller sample (the q matrix's
+        # quantize, 16 output rows per matrix for the GEMV reference)
+        tb1, qg1, thr1, desc1, secs1, _ = oracle_sample(rows_per_matrix=16, quantize_layer=False, threads=1)
+        cpu["single_thread"] = {"value": tb1, "unit": UNIT, "cores": thr1, "quantize_gbs": qg1, "sample": desc1,
+                                "seconds": round(secs1, 1)}
 
     if rank == 0:
         line = {
