@@ -64,27 +64,27 @@ def test_gemm_dtypes(q4, oracle, a_dtype, dq):
 
 def test_gemm_prefill_7b_layer_m512(q4, oracle):
     """Prefill config: the 7B layer shapes, NF4 double-quant weights, bf16
-    activations at M = 512, one grouped launch; sampled output columns."""
+    activations at M = 512, one grouped launch; every output of the layer
+    against the oracle's binary64 product (about 200 GFLOP on the host)."""
     from bit_blockwise_weight_absmax_b200 import workloads as wl
     Ws = wl.layer_weights(wl.LAYER_7B, 0.02, seed=300)
     sts = [q4.quantize(W.cuda(), 64, "nf4", True) for W in Ws]
     osts = [oracle_state(oracle, W, 64, 0, True) for W in Ws]
-    rng = np.random.default_rng(1)
     M = 512
     As = [wl.activation(M, K, torch.bfloat16, seed=400 + i) for i, (_, N, K) in enumerate(wl.LAYER_7B)]
     ys = q4.gemm_grouped([a.cuda() for a in As], sts)
     torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
     for (name, N, K), a, y, ost in zip(wl.LAYER_7B, As, ys, osts):
-        rows = np.sort(rng.choice(N, 128, replace=False))
-        w16 = oracle.dequantize(ost, True).reshape(N, K)[rows]
-        ref = oracle.matmul(bits(a), True, w16, True, M, len(rows), K)
-        assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+        w16 = oracle.dequantize(ost, True)
+        ref = oracle.matmul(bits(a), True, w16, True, M, N, K)
+        assert_matmul_close(y, ref)
 
 
 @pytest.mark.parametrize("M", [2048, 8192])
 def test_gemm_prefill_7b_layer_large_m(q4, oracle, M):
     """Prefill config at M = 2048 and 8192 tokens: one grouped launch over the
-    7B layer; checked on a deterministic sample of 64 token rows x 128 output
+    7B layer; checked on a deterministic sample of 64 token rows x 256 output
     columns per matrix (the oracle's binary64 product of those)."""
     from bit_blockwise_weight_absmax_b200 import workloads as wl
     Ws = wl.layer_weights(wl.LAYER_7B, 0.02, seed=310)
@@ -96,7 +96,7 @@ def test_gemm_prefill_7b_layer_large_m(q4, oracle, M):
     torch.cuda.synchronize()
     assert q4.last_device_status() == 0
     for (name, N, K), a, y, ost in zip(wl.LAYER_7B, As, ys, osts):
-        rows = np.sort(rng.choice(N, 128, replace=False))
+        rows = np.sort(rng.choice(N, 256, replace=False))
         toks = np.sort(rng.choice(M, 64, replace=False))
         w16 = oracle.dequantize(ost, True).reshape(N, K)[rows]
         a16 = bits(a).reshape(M, K)[toks]
