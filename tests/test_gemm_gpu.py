@@ -40,6 +40,27 @@ def test_gemm_one_tile(q4, oracle):
     assert_matmul_close(y, ref)
 
 
+def test_gemm_exact_small_integers(q4, oracle):
+    """A in {-1, 0, 1}, every block's maximum 1 (so w^ is the bf16 level),
+    K = 64, fp32 output: each partial sum of the tensor cores is exactly
+    representable in binary32 (the terms' magnitudes span under 2^17 ulps),
+    so Y equals the oracle's binary64 product exactly."""
+    g = torch.Generator().manual_seed(9)
+    M, N, K = 40, 64, 64
+    L = torch.tensor(oracle.nf4_levels())
+    codes = torch.randint(0, 16, (N, K), generator=g)
+    W = L[codes]
+    W[:, 0] = 1.0  # the block absmax
+    W = W.bfloat16()
+    A = torch.randint(-1, 2, (M, K), generator=g).bfloat16()
+    st = q4.quantize(W.cuda(), 64, "nf4", False)
+    ost = oracle_state(oracle, W, 64, 0, False)
+    y = q4.gemm(A.cuda(), st, torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.matmul(bits(A), True, oracle.dequantize(ost, True), True, M, N, K)
+    assert np.array_equal(y.cpu().double().numpy(), ref)
+
+
 def test_gemm_fp32_out_tight(q4, oracle):
     """fp32 output: the only difference from the binary64 reference is the
     fp32 accumulation order, far below the tolerance."""
