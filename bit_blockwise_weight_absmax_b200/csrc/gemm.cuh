@@ -68,12 +68,22 @@ struct alignas(64) GemmMat {
   int32_t pad;
 };
 
-// Up to this many tiles a launch carries an explicit tile list per CTA,
-// balanced on the host by the k-blocks of each tile (longest first onto the
-// least loaded CTA); above it the tiles are dealt round robin, which is then
-// within a few percent of even.
+// Up to this many work items a launch carries an explicit item list per
+// CTA, balanced on the host by the k-blocks of each item (longest first onto
+// the least loaded CTA); above it whole tiles are dealt round robin, which
+// is then within a few percent of even.  An item is a whole tile or one
+// half of a tile's k range (split-K): both halves write their fp32
+// partials to the workspace and the second to finish adds the other's and
+// writes Y.  Item encoding: bits 0-15 tile, 16-17 half (0 whole, 1 first,
+// 2 second), 18-31 split slot.
 constexpr int kGemmListTiles = 2048;
 constexpr int kGemmListCtas = 256;  // grid bound of a listed launch
+constexpr int kGemmSplitWarpFloats = 2 * 2 * 32 * 16;  // one epilogue warp's partial: pieces x halves x lanes x 16
+constexpr size_t kGemmSplitSlotBytes = 2 * 16 * kGemmSplitWarpFloats * sizeof(float);  // two halves x 16 warps
+// The arrival counters sit at the start of the workspace in a region of a
+// fixed size (every slot a listed launch can have), so that whatever slot
+// count the previous call used, they are the zeroed words it left.
+constexpr size_t kGemmSplitCntBytes = (size_t)(kGemmListTiles / 2) * 16 * sizeof(unsigned);
 
 struct GemmParams {
   GemmMat mat[16];
@@ -87,9 +97,12 @@ struct GemmParams {
   uint64_t wait_ns;      // bound of every mbarrier wait
   int *status;
   float levels[16];
-  int32_t listed;        // tiles come from tile_list (else round robin)
+  int32_t listed;        // items come from tile_list (else whole tiles round robin)
+  int32_t grid;          // CTAs of the launch
+  unsigned *split_cnt;   // split-K: [slot][epilogue warp] arrivals (zero between calls), at the workspace start
+  float *partials;       // split-K: [slot][half][epilogue warp][kGemmSplitWarpFloats] fp32, after the counters
   uint16_t cta_off[kGemmListCtas + 1];  // CTA c runs tile_list[cta_off[c] .. cta_off[c + 1])
-  uint16_t tile_list[kGemmListTiles];
+  uint32_t tile_list[kGemmListTiles];
 };
 
 // ---- PTX wrappers ------------------------------------------------------------
@@ -239,23 +252,123 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 struct TileCoord {
   int mi, tm, tn;
+  int kb0, kb1;  // the k-blocks of this item
+  int slot;      // split-K slot (-1: a whole tile)
+  int half;      // split-K half (0, 1)
 };
-__device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t t) {
+// Work item v: an encoded list item when the launch is listed, else a
+// whole tile index.
+__device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t v) {
+  const int64_t t = p.listed ? (int64_t)(v & 0xFFFF) : v;
+  const int hc = p.listed ? (int)((v >> 16) & 3) : 0;
   int mi = 0;
   while (mi + 1 < p.count && t >= p.mat[mi + 1].tile_begin) ++mi;
   const int64_t local = t - p.mat[mi].tile_begin;
   const int tm_count = p.mat[mi].tiles_m;
+  const int nk = p.mat[mi].K / kGemmBK;
   // m-tiles fastest: consecutive CTAs share one weight tile (read once from HBM)
-  return TileCoord{mi, (int)(local % tm_count), (int)(local / tm_count)};
+  TileCoord tc{mi, (int)(local % tm_count), (int)(local / tm_count), 0, nk, -1, 0};
+  if (hc != 0) {
+    tc.half = hc - 1;
+    tc.slot = (int)(v >> 18);
+    tc.kb0 = tc.half == 0 ? 0 : nk / 2;
+    tc.kb1 = tc.half == 0 ? nk / 2 : nk;
+  }
+  return tc;
+}
+
+// Epilogue helpers.  A dequant warp's share of a tile: TMEM lanes q * 32 ..
+// + 31 (its quadrant) and accumulator columns cc * 32 .. + 31 of both
+// accumulators, in four chunks of 16 columns (ch = 2 accumulator + half).
+__device__ __forceinline__ uint32_t gemm_chunk(uint32_t tmem, int ab, int ch, int q, int cc, int &h, int &c16) {
+  const int piece = ch >> 1, hh = ch & 1;
+  h = piece / (kGemmBN / 128);
+  const int part = piece % (kGemmBN / 128);
+  c16 = cc * (kGemmBN / 4) + part * 32 + 16 * hh;
+  return tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((ab * kGemmAccs + h) * kGemmBN + c16);
+}
+constexpr int kGemmChunks = kGemmAccs * kGemmBN / 128 * 2;  // 16-column chunks per warp
+static_assert(kGemmChunks * 32 * 16 == kGemmSplitWarpFloats, "split-K partial layout");
+// Y[mrow, n0 .. n0 + 15] of one lane (its row) from 16 fp32 accumulators.
+__device__ __forceinline__ void gemm_store_y(const GemmMat &m, int y_dtype, int mrow, int n0, const uint32_t (&r)[16]) {
+  if (mrow >= m.M || n0 >= m.N) return;
+  if (y_dtype == Q4_F32) {
+    float *y = reinterpret_cast<float *>(m.Y) + (int64_t)mrow * m.N + n0;
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      if (n0 + 4 * v < m.N)
+        *reinterpret_cast<uint4 *>(y + 4 * v) = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+  } else {
+    uint16_t *y = reinterpret_cast<uint16_t *>(m.Y) + (int64_t)mrow * m.N + n0;
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      if (n0 + 8 * v < m.N) {
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float f0 = __uint_as_float(r[8 * v + 2 * e]), f1 = __uint_as_float(r[8 * v + 2 * e + 1]);
+          o[e] = (y_dtype == Q4_BF16) ? Dt<Q4_BF16>::pack2(f0, f1) : Dt<Q4_F16>::pack2(f0, f1);
+        }
+        *reinterpret_cast<uint4 *>(y + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+}
+// Split-K epilogue of one warp's share of a cut tile.  The half's fp32 partial is published, then counted; the warp that
+// completes the count adds the other half's partial (a + b: the same bits
+// whichever half finishes second), writes Y and zeroes the counter.
+static __device__ __forceinline__ void gemm_split_epilogue(const GemmParams *pp, uint32_t tmem, int ab, int mi, int tm,
+                                                        int tn, int slot, int half, int q, int cc, int lane, int wp) {
+  const GemmParams &p = *pp;
+  const GemmMat &m = p.mat[mi];
+  float *mine = p.partials + ((int64_t)(slot * 2 + half) * 16 + wp) * kGemmSplitWarpFloats;
+#pragma unroll 1
+  for (int ch = 0; ch < kGemmChunks; ++ch) {
+    int h, c16;
+    uint32_t r[16];
+    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, h, c16), r);
+    float4 *dst = reinterpret_cast<float4 *>(mine + (ch * 32 + lane) * 16);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      __stcg(dst + v, make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                  __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
+  }
+  __threadfence();  // this lane's partial is visible before its count
+  __syncwarp();
+  unsigned old = 0;
+  if (lane == 0) old = atomicAdd(p.split_cnt + slot * 16 + wp, 1u);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  if (old != 1) return;  // the other half will finish the tile
+  __threadfence();
+  const float *other = p.partials + ((int64_t)(slot * 2 + (1 - half)) * 16 + wp) * kGemmSplitWarpFloats;
+#pragma unroll 1
+  for (int ch = 0; ch < kGemmChunks; ++ch) {
+    int h, c16;
+    uint32_t r[16];
+    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, h, c16), r);
+    const float4 *src = reinterpret_cast<const float4 *>(other + (ch * 32 + lane) * 16);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const float4 o = __ldcg(src + v);
+      r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + o.x);
+      r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + o.y);
+      r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + o.z);
+      r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + o.w);
+    }
+    gemm_store_y(m, p.y_dtype, tm * kGemmBM + h * 128 + q * 32 + lane, tn * kGemmBN + c16, r);
+  }
+  if (lane == 0) p.split_cnt[slot * 16 + wp] = 0u;  // the workspace is left zeroed
 }
 
 // Block-scale modes of the GEMM: absmax as stored (NF4, INT4 symmetric),
 // double-quantized (NF4), or scale plus zero-point (INT4 asymmetric).
 constexpr int kGemmPlain = 0, kGemmDq = 1, kGemmAsym = 2;
 
-// DA: activation dtype; MODE: block-scale mode.  The blocksize is a launch
-// parameter: it only decides which block scale a thread's 16 codes take.
-template <int DA, int MODE>
+// DA: activation dtype; MODE: block-scale mode; SPLIT: the launch has cut
+// tiles (the instance without them carries no split-K code, so its
+// registers do not spill).  The blocksize is a launch parameter: it only
+// decides which block scale a thread's 16 codes take.
+template <int DA, int MODE, bool SPLIT>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool DQ = MODE == kGemmDq, ASYM = MODE == kGemmAsym;
   pdl_launch_dependents();  // set-up (barriers, TMEM, level table) overlaps the previous kernel
@@ -323,8 +436,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       for (int64_t k = 0; k < n_my && !*abort; ++k) {
         const TileCoord tc = gemm_tile(p, my_tile(k));
         const GemmMat &m = p.mat[tc.mi];
-        const int nk = m.K / kGemmBK;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
           const int s = it % kGemmStages;
           const uint32_t use = it / kGemmStages;
           if (!mbar_wait(empty_bar(s), (use & 1) ^ 1, p.status, abort, p.wait_ns)) break;
@@ -351,12 +463,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       bool committed = false;
       for (int64_t k = 0; k < n_my && !*abort; ++k, ++tcount) {
         const TileCoord tc = gemm_tile(p, my_tile(k));
-        const int nk = p.mat[tc.mi].K / kGemmBK;
         const int ab = tcount & 1;  // accumulator set of this tile
         if (!mbar_wait(accempty_bar(ab), ((tcount >> 1) & 1) ^ 1, p.status, abort, p.wait_ns)) break;
         tc_fence_after();
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
           const int s = it % kGemmStages;
           const uint32_t use = it / kGemmStages;
           if (!mbar_wait(full_bar(s), use & 1, p.status, abort, p.wait_ns) ||
@@ -373,7 +484,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
 #pragma unroll
             for (int h = 0; h < kGemmAccs; ++h) {
               const uint64_t da = umma_desc_sw128(a0 + h * (128 * kGemmBK * 2) + 32 * k16);
-              umma_f16(tmem + (uint32_t)((ab * kGemmAccs + h) * kGemmBN), da, db, idesc, (kb | k16) != 0);
+              umma_f16(tmem + (uint32_t)((ab * kGemmAccs + h) * kGemmBN), da, db, idesc, kb != tc.kb0 || k16 != 0);
             }
           }
           umma_commit(empty_bar(s));
@@ -401,62 +512,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const int q = warp & 3;            // TMEM lane quadrant of this warp
     const int cc = (warp - 2) >> 2;    // quarter of the accumulator columns handled in the epilogue
     const uint32_t lvb = smem_u32(s_lv) + 4u * lane;
-    // epilogue of a finished tile: its accumulator set -> Y
-    // (the MMAs of the next tile go to the other accumulator set meanwhile)
-    auto epilogue = [&](const TileCoord &tc, uint32_t tcount) -> bool {
-      const GemmMat &m = p.mat[tc.mi];
-        const int ab = tcount & 1;
-        if (!mbar_wait_warp(accfull_bar(ab), (tcount >> 1) & 1, p.status, abort, p.wait_ns)) return false;
-        tc_fence_after();
+    // epilogue of a finished item: its accumulator set -> Y
+    // (the MMAs of the next item go to the other accumulator set meanwhile)
+    const int wp = warp - 2;  // this warp's share of a tile's accumulators: 0..15
+    auto epilogue = [&](int64_t item, uint32_t tcount) -> bool {
+      const TileCoord tc = gemm_tile(p, item);  // decoded again: one word stays live across the loop
+      const int ab = tcount & 1;
+      if (!mbar_wait_warp(accfull_bar(ab), (tcount >> 1) & 1, p.status, abort, p.wait_ns)) return false;
+      tc_fence_after();
+      if (SPLIT && tc.slot >= 0) {
+        if constexpr (SPLIT) gemm_split_epilogue(&p, tmem, ab, tc.mi, tc.tm, tc.tn, tc.slot, tc.half, q, cc, lane, wp);
+      } else {
+        const GemmMat &m = p.mat[tc.mi];
 #pragma unroll 1
-        for (int piece = 0; piece < kGemmAccs * kGemmBN / 128; ++piece) {
-          const int h = piece / (kGemmBN / 128), part = piece % (kGemmBN / 128);
-          const int mrow = tc.tm * kGemmBM + h * 128 + q * 32 + lane;
-          const int col0 = cc * (kGemmBN / 4) + part * 32;
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {  // 16 columns per tcgen05.ld
-            const int c16 = col0 + 16 * hh;
-            uint32_t r[16];
-            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((ab * kGemmAccs + h) * kGemmBN + c16), r);
-            const int n0 = tc.tn * kGemmBN + c16;
-            if (mrow < m.M && n0 < m.N) {
-              if (p.y_dtype == Q4_F32) {
-                float *y = reinterpret_cast<float *>(m.Y) + (int64_t)mrow * m.N + n0;
-#pragma unroll
-                for (int v = 0; v < 4; ++v)
-                  if (n0 + 4 * v < m.N)
-                    *reinterpret_cast<uint4 *>(y + 4 * v) = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-              } else {
-                uint16_t *y = reinterpret_cast<uint16_t *>(m.Y) + (int64_t)mrow * m.N + n0;
-#pragma unroll
-                for (int v = 0; v < 2; ++v) {
-                  if (n0 + 8 * v < m.N) {
-                    uint32_t o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                      const float f0 = __uint_as_float(r[8 * v + 2 * e]), f1 = __uint_as_float(r[8 * v + 2 * e + 1]);
-                      o[e] = (p.y_dtype == Q4_BF16) ? Dt<Q4_BF16>::pack2(f0, f1) : Dt<Q4_F16>::pack2(f0, f1);
-                    }
-                    *reinterpret_cast<uint4 *>(y + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
-                  }
-                }
-              }
-            }
-          }
+        for (int ch = 0; ch < kGemmChunks; ++ch) {
+          int h, c16;
+          uint32_t r[16];
+          tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, h, c16), r);
+          gemm_store_y(m, p.y_dtype, tc.tm * kGemmBM + h * 128 + q * 32 + lane, tc.tn * kGemmBN + c16, r);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(accempty_bar(ab));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty_bar(ab));
       return true;
     };
     bool have_prev = false;
-    TileCoord prev_tc{0, 0, 0};
+    int64_t prev_item = 0;
     uint32_t prev_count = 0;
     uint32_t it = 0, tcount = 0;
     for (int64_t k = 0; k < n_my && !*abort; ++k, ++tcount) {
-      const TileCoord tc = gemm_tile(p, my_tile(k));
+      const int64_t item = my_tile(k);
+      const TileCoord tc = gemm_tile(p, item);
       const GemmMat &m = p.mat[tc.mi];
-      const int nk = m.K / kGemmBK;
       const int lbs = p.log2_bs;
       const int nblk = m.K >> lbs;  // blocks per weight row
       const int row = tc.tn * kGemmBN + d;
@@ -523,22 +611,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         *reinterpret_cast<float4 *>(scrow + 4 * qk) = make_float4(v[0], v[1], v[2], v[3]);
         if constexpr (ASYM) *reinterpret_cast<uint32_t *>(zrow + 4 * qk) = o.cw;
       };
+      // the window of 16 blocks holding the item's first k-block
+      const int w0 = ((tc.kb0 * kGemmBK) >> lbs) & ~15;
       In4 nin;
       {
         In4 cin;
-        load4(4 * qk, cin);
-        load4(16 + 4 * qk, nin);  // zeros past the row's end
+        load4(w0 + 4 * qk, cin);
+        load4(w0 + 16 + 4 * qk, nin);  // zeros past the row's end
         __syncwarp();  // the row's previous c~ have been read
         store4(cin);
         __syncwarp();
       }
-      int wnext = 16;  // first block of the window held in nin
+      int wnext = w0 + 16;  // first block of the window held in nin
       bool ok = true;
-      for (int kb = 0; kb < nk; ++kb, ++it) {
+      for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
         const int s = it % kGemmStages;
         const uint32_t use = it / kGemmStages;
         const int kk = kb * kGemmBK;
-        if (kb > 0 && (kk & ((16 << lbs) - 1)) == 0) {
+        if (kb > tc.kb0 && (kk & ((16 << lbs) - 1)) == 0) {
           // a new window of 16 blocks starts at this k-block
           __syncwarp();  // the row's c~ of the previous window have been read
           store4(nin);
@@ -599,8 +689,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         if (lane == 0) mbar_arrive(bfull_bar(s));
         // the previous tile's epilogue once this tile's first stages are
         // queued: its stores overlap the MMAs of those stages
-        if (have_prev && kb == min(kGemmStages, nk) - 1) {
-          if (!epilogue(prev_tc, prev_count)) {
+        if (have_prev && kb - tc.kb0 == min(kGemmStages, tc.kb1 - tc.kb0) - 1) {
+          if (!epilogue(prev_item, prev_count)) {
             ok = false;
             break;
           }
@@ -609,10 +699,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       }
       if (!ok) break;
       have_prev = true;
-      prev_tc = tc;
+      prev_item = item;
       prev_count = tcount;
     }
-    if (have_prev && !*abort) epilogue(prev_tc, prev_count);
+    if (have_prev && !*abort) epilogue(prev_item, prev_count);
   }
 
   tc_fence_before();

@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <queue>
 #include <vector>
 
 #include "q4_internal.h"
@@ -603,58 +604,131 @@ int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void 
   return q4_gemv_grouped(1, a, w, y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
 }
 
-// The tiles of a small launch dealt to the CTAs longest first (k-blocks of
-// the tile), each onto the CTA with the least work so far; every CTA then
-// runs its tiles in ascending order.  Round robin otherwise.
-static void gemm_balance(GemmParams &p, int count, int64_t grid) {
-  p.listed = 0;
-  if (p.total_tiles > kGemmListTiles || grid > kGemmListCtas || p.total_tiles <= grid) return;
-  std::vector<std::pair<int, int>> order;  // (k-blocks, tile)
-  order.reserve((size_t)p.total_tiles);
+// ---- GEMM planning -----------------------------------------------------------
+// A launch of at most kGemmListTiles work items deals them to the CTAs
+// longest first (k-blocks), each onto the CTA with the least work so far;
+// every CTA then runs its items in ascending order.  With a workspace the
+// planner may also cut tiles into two halves of their k range (split-K):
+// it deals three candidates -- whole tiles, the longest tiles cut, every
+// tile of at least two k-blocks cut -- and keeps the one whose busiest CTA
+// has the least work (ties: fewer cuts), a cut only when it takes at least
+// a tenth off the whole tiles' busiest CTA (the cut instance also carries
+// the split-K code, which costs its registers).  A half counts its k-blocks plus
+// kGemmSplitCost for its fix-up (an fp32 partial written, counted and, by
+// the second half, read back; measured at M = 512 on one B200 as about 16
+// k-blocks' time).  Larger launches deal whole tiles round robin, which is
+// then within a few percent of even.
+constexpr int kGemmSplitCost = 16;
+struct GemmPlan {
+  int64_t grid = 0;    // CTAs
+  int64_t slots = 0;   // split tiles
+  int64_t max_load = 0;
+  int listed = 0;
+  int cut = 0;         // 0 none, 1 the longest tiles, 2 every tile
+};
+size_t gemm_split_bytes(int64_t slots) {
+  return slots ? kGemmSplitCntBytes + (size_t)slots * kGemmSplitSlotBytes : 0;
+}
+// The items of cut mode `cut` as (work, encoded item); slots counts the cut tiles.
+static void gemm_items(const GemmParams &p, int count, int cut, std::vector<std::pair<int, uint32_t>> &items,
+                       int64_t &slots) {
+  int max_nk = 0;
+  for (int i = 0; i < count; ++i) max_nk = std::max(max_nk, p.mat[i].K / kGemmBK);
+  items.clear();
+  slots = 0;
   for (int i = 0; i < count; ++i) {
     const GemmMat &m = p.mat[i];
+    const int nk = m.K / kGemmBK;
+    const bool split = nk >= 2 && (cut == 2 || (cut == 1 && nk == max_nk));
     const int64_t n = (int64_t)m.tiles_m * m.tiles_n;
-    for (int64_t t = 0; t < n; ++t) order.emplace_back(m.K / kGemmBK, (int)(m.tile_begin + t));
+    for (int64_t t = 0; t < n; ++t) {
+      const uint32_t tile = (uint32_t)(m.tile_begin + t);
+      if (split) {
+        items.emplace_back(nk / 2 + kGemmSplitCost, tile | (1u << 16) | ((uint32_t)slots << 18));
+        items.emplace_back(nk - nk / 2 + kGemmSplitCost, tile | (2u << 16) | ((uint32_t)slots << 18));
+        ++slots;
+      } else {
+        items.emplace_back(nk, tile);
+      }
+    }
   }
-  std::stable_sort(order.begin(), order.end(),
-                   [](const std::pair<int, int> &a, const std::pair<int, int> &b) { return a.first > b.first; });
-  std::vector<std::vector<int>> per((size_t)grid);
+}
+// Longest first onto the least loaded of `grid` CTAs; the busiest CTA's
+// k-blocks.  With `out`, its lists are written there.
+static int64_t gemm_lpt(std::vector<std::pair<int, uint32_t>> items, int64_t grid, GemmParams *out) {
+  std::stable_sort(items.begin(), items.end(),
+                   [](const std::pair<int, uint32_t> &a, const std::pair<int, uint32_t> &b) { return a.first > b.first; });
+  std::vector<std::vector<uint32_t>> per((size_t)grid);
   std::vector<int64_t> load((size_t)grid, 0);
-  for (const auto &o : order) {
-    int64_t best = 0;
-    for (int64_t c = 1; c < grid; ++c)
-      if (load[(size_t)c] < load[(size_t)best]) best = c;
+  // the least loaded CTA (the lowest index among equals) from a min-heap
+  std::priority_queue<std::pair<int64_t, int64_t>, std::vector<std::pair<int64_t, int64_t>>,
+                      std::greater<std::pair<int64_t, int64_t>>> heap;
+  for (int64_t c = 0; c < grid; ++c) heap.emplace(0, c);
+  for (const auto &o : items) {
+    const int64_t best = heap.top().second;
+    heap.pop();
     load[(size_t)best] += o.first;
     per[(size_t)best].push_back(o.second);
+    heap.emplace(load[(size_t)best], best);
   }
-  int off = 0;
-  for (int64_t c = 0; c < grid; ++c) {
-    p.cta_off[c] = (uint16_t)off;
-    std::sort(per[(size_t)c].begin(), per[(size_t)c].end());
-    for (int t : per[(size_t)c]) p.tile_list[off++] = (uint16_t)t;
+  if (out) {
+    int off = 0;
+    for (int64_t c = 0; c < grid; ++c) {
+      out->cta_off[c] = (uint16_t)off;
+      std::sort(per[(size_t)c].begin(), per[(size_t)c].end(),
+                [](uint32_t a, uint32_t b) { return (a & 0xFFFFu) != (b & 0xFFFFu) ? (a & 0xFFFFu) < (b & 0xFFFFu) : a < b; });
+      for (uint32_t v : per[(size_t)c]) out->tile_list[off++] = v;
+    }
+    out->cta_off[grid] = (uint16_t)off;
   }
-  p.cta_off[grid] = (uint16_t)off;
-  p.listed = 1;
+  return *std::max_element(load.begin(), load.end());
+}
+// The plan of a launch over p's matrices (tiles set); `max_split_bytes`
+// bounds the workspace a cut may use (0: no cuts).  With `out`, the chosen
+// lists are written there.
+static GemmPlan gemm_plan(const GemmParams &p, int count, int sms, size_t max_split_bytes, GemmParams *out) {
+  GemmPlan best;
+  const int64_t tiles = p.total_tiles;
+  best.grid = std::min<int64_t>(tiles, sms);
+  if (tiles > kGemmListTiles) return best;  // round robin over whole tiles
+  std::vector<std::pair<int, uint32_t>> items;
+  bool have = false;
+  int64_t whole_load = 0;  // the busiest CTA of whole tiles (cut 0 comes first)
+  for (int cut = 0; cut <= 2; ++cut) {
+    int64_t slots = 0;
+    gemm_items(p, count, cut, items, slots);
+    if (cut > 0 && (slots == 0 || gemm_split_bytes(slots) > max_split_bytes)) continue;
+    if ((int64_t)items.size() > kGemmListTiles || slots > kGemmListTiles / 2) continue;
+    const int64_t grid = std::min<int64_t>({(int64_t)items.size(), (int64_t)sms, (int64_t)kGemmListCtas});
+    const int64_t mx = gemm_lpt(items, grid, nullptr);
+    if (cut > 0 && 10 * mx > 9 * whole_load) continue;
+    if (!have || mx < best.max_load || (mx == best.max_load && slots < best.slots)) {
+      best.grid = grid;
+      best.slots = slots;
+      best.max_load = mx;
+      best.cut = cut;
+      // a list is needed for cut tiles, or to balance more tiles than CTAs
+      best.listed = (slots > 0 || (int64_t)items.size() > grid) ? 1 : 0;
+      have = true;
+    }
+    if (cut == 0) whole_load = mx;
+  }
+  if (out && best.listed) {
+    int64_t slots = 0;
+    gemm_items(p, count, best.cut, items, slots);
+    gemm_lpt(items, best.grid, out);
+  }
+  return best;
 }
 
-int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
-                    void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream) {
-  if (count < 1 || count > kGsMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
-  if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
-  if (y_dtype != Q4_F32 && y_dtype != a_dtype) return Q4_ERR_ARG;
-  if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;
-  for (int i = 0; i < count; ++i)
-    if (!Wq[i] || !A[i] || !Y[i]) return Q4_ERR_ARG;
-  const DeviceInfo di = device_info();
-  static thread_local GemmParams p;  // host staging of the kernel parameters (~10 KB)
-  memset(&p, 0, sizeof(p));
-  int rc = Q4_OK;
+// Shapes and formats of a GEMM call (host only); fills the per-matrix tile
+// counts of `p`.
+static int gemm_check(int32_t count, const q4_state *const *Wq, int64_t M, GemmParams &p) {
   int64_t tiles = 0;
-  int dq = -1;
-  // every matrix's format and shape first (host only), then the device
   for (int i = 0; i < count; ++i) {
     const q4_state *s = Wq[i];
-    rc = check_state(s);
+    if (!s) return Q4_ERR_ARG;
+    const int rc = check_state(s);
     if (rc != Q4_OK) return rc;
     // one format per grouped call
     if (s->qtype != Wq[0]->qtype || s->blocksize != Wq[0]->blocksize ||
@@ -663,10 +737,54 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     // whole 64-k blocks of whole quantization blocks
     if (s->cols % 64 || s->cols % s->blocksize || s->rows % 16 || s->rows > INT32_MAX || s->cols > INT32_MAX)
       return Q4_ERR_SHAPE;
-    if (!aligned16(A[i]) || !aligned16(Y[i])) return Q4_ERR_ALIGN;
+    GemmMat &m = p.mat[i];
+    m.M = (int32_t)M;
+    m.N = (int32_t)s->rows;
+    m.K = (int32_t)s->cols;
+    m.tiles_m = (int32_t)ceil_div(M, kGemmBM);
+    m.tiles_n = (int32_t)ceil_div(s->rows, kGemmBN);
+    m.tile_begin = tiles;
+    tiles += (int64_t)m.tiles_m * m.tiles_n;
   }
+  p.count = count;
+  p.total_tiles = tiles;
+  return Q4_OK;
+}
+
+int q4_gemm_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {
+  if (!bytes || !Wq || count < 1 || count > kGsMaxGroup) return Q4_ERR_ARG;
+  if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;
+  static thread_local GemmParams p;
+  memset(&p, 0, sizeof(p));
+  const int rc = gemm_check(count, Wq, M, p);
+  if (rc != Q4_OK) return rc;
+  const DeviceInfo di = device_info();
   if (di.ok != Q4_OK) return di.ok;
-  dq = Wq[0]->double_quant;
+  const GemmPlan plan = gemm_plan(p, count, di.sms, (size_t)-1, nullptr);
+  *bytes = gemm_split_bytes(plan.slots);
+  return Q4_OK;
+}
+
+int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
+                    void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+  if (count < 1 || count > kGsMaxGroup || !A || !Wq || !Y) return Q4_ERR_ARG;
+  if (!valid_in_dtype(a_dtype) || !valid_out_dtype(y_dtype)) return Q4_ERR_ARG;
+  if (y_dtype != Q4_F32 && y_dtype != a_dtype) return Q4_ERR_ARG;
+  if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;
+  for (int i = 0; i < count; ++i)
+    if (!Wq[i] || !A[i] || !Y[i]) return Q4_ERR_ARG;
+  static thread_local GemmParams p;  // host staging of the kernel parameters (~14 KB)
+  memset(&p, 0, sizeof(p));
+  // every matrix's format and shape first (host only), then the device
+  int rc = gemm_check(count, Wq, M, p);
+  if (rc != Q4_OK) return rc;
+  for (int i = 0; i < count; ++i)
+    if (!aligned16(A[i]) || !aligned16(Y[i])) return Q4_ERR_ALIGN;
+  if (workspace && !aligned16(workspace)) return Q4_ERR_ALIGN;
+  const DeviceInfo di = device_info();
+  if (di.ok != Q4_OK) return di.ok;
+  const int dq = Wq[0]->double_quant;
   for (int i = 0; i < count && rc == Q4_OK; ++i) {
     const q4_state *s = Wq[i];
     GemmMat &m = p.mat[i];
@@ -683,19 +801,10 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     m.absmax = s->absmax;
     m.zero = s->zero;
     m.Y = Y[i];
-    m.M = (int32_t)M;
-    m.N = (int32_t)s->rows;
-    m.K = (int32_t)s->cols;
-    m.tiles_m = (int32_t)ceil_div(M, kGemmBM);
-    m.tiles_n = (int32_t)ceil_div(s->rows, kGemmBN);
-    m.tile_begin = tiles;
-    tiles += (int64_t)m.tiles_m * m.tiles_n;
   }
   if (rc == Q4_OK) {
-    p.count = count;
     p.y_dtype = y_dtype;
     p.dq = dq;
-    p.total_tiles = tiles;
     p.status = di.status;
     const int qt = Wq[0]->qtype;
     int mode = dq ? kGemmDq : kGemmPlain;
@@ -709,20 +818,26 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     }
     p.log2_bs = __builtin_ctz((unsigned)Wq[0]->blocksize);
     p.scale_f16 = Wq[0]->scale_f16;
-    gemm_balance(p, count, std::min<int64_t>(tiles, di.sms));
+    const GemmPlan plan = gemm_plan(p, count, di.sms, workspace ? workspace_bytes : 0, &p);
+    p.listed = plan.listed;
+    p.grid = (int32_t)plan.grid;
+    if (plan.slots) {
+      p.split_cnt = reinterpret_cast<unsigned *>(workspace);
+      p.partials = reinterpret_cast<float *>((char *)workspace + kGemmSplitCntBytes);
+    }
     p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     p.stall_copies = g_copy_stall.load(std::memory_order_relaxed);
-    rc = run_gemm(a_dtype, mode, p, di.sms, (cudaStream_t)stream);
+    rc = run_gemm(a_dtype, mode, plan.slots > 0, p, (cudaStream_t)stream);
   }
   return rc;
 }
 
 int q4_gemm(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
-            int32_t y_dtype, void *stream) {
+            int32_t y_dtype, void *workspace, size_t workspace_bytes, void *stream) {
   const void *a[1] = {A};
   const q4_state *w[1] = {Wq};
   void *y[1] = {Y};
-  return q4_gemm_grouped(1, a, w, y, M, a_dtype, y_dtype, stream);
+  return q4_gemm_grouped(1, a, w, y, M, a_dtype, y_dtype, workspace, workspace_bytes, stream);
 }
 
 int q4_set_wait_limit_ns(uint64_t ns) {

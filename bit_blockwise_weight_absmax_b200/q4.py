@@ -73,9 +73,10 @@ def library():
             "q4_gemv": ([P, i32, i64, SP, P, i32, P, sz, P], i32),
             "q4_gemv_grouped": ([i32, ctypes.POINTER(P), ctypes.POINTER(SP), ctypes.POINTER(P), i64,
                                  i32, i32, P, sz, P], i32),
-            "q4_gemm": ([P, i32, i64, SP, P, i32, P], i32),
+            "q4_gemm_workspace_size": ([i32, ctypes.POINTER(SP), i64, ctypes.POINTER(ctypes.c_size_t)], i32),
+            "q4_gemm": ([P, i32, i64, SP, P, i32, P, ctypes.c_size_t, P], i32),
             "q4_gemm_grouped": ([i32, ctypes.POINTER(P), ctypes.POINTER(SP), ctypes.POINTER(P), i64,
-                                 i32, i32, P], i32),
+                                 i32, i32, P, ctypes.c_size_t, P], i32),
             "q4_device_status": ([ctypes.POINTER(i32)], i32),
             "q4_clear_device_status": ([], i32),
             "q4_set_wait_limit_ns": ([ctypes.c_uint64], i32),
@@ -443,8 +444,14 @@ def gemm_grouped(As, states, out_dtype: torch.dtype | None = None, outs=None, st
             raise Q4Error("activations must be contiguous [M, K] of one dtype")
     a_ptrs = (ctypes.c_void_p * len(As))(*[a.data_ptr() for a in As])
     y_ptrs = (ctypes.c_void_p * len(As))(*[y.data_ptr() for y in outs])
+    # the workspace that lets the launch cut tiles in k where that evens out
+    # the CTAs' work (cached per device; zero-filled, left zeroed)
+    wsz = ctypes.c_size_t(0)
+    _check(library().q4_gemm_workspace_size(len(As), arr, M, ctypes.byref(wsz)), "q4_gemm_workspace_size")
+    ws = _workspace(As[0].device, "gemm", wsz.value)
     _check(library().q4_gemm_grouped(len(As), a_ptrs, arr, y_ptrs, M, _DT[a_dtype], _DT[out_dtype],
-                                     _stream(stream)), "q4_gemm_grouped")
+                                     _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+           "q4_gemm_grouped")
     return outs
 
 

@@ -275,6 +275,16 @@ Q4_API int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *
 
 /* ---- W4A16 GEMM (prefill, large M) ------------------------------------ */
 
+/* Workspace for q4_gemm / q4_gemm_grouped: room for fp32 partial tiles and
+ * arrival counters when the launch cuts tiles in halves of their k range
+ * to even out the CTAs' work (a launch of few tiles, or of matrices with
+ * very different K).  0 when no cut pays off.  The size depends on the
+ * shapes, M and the current device's SM count.  Its first 64 KB hold the
+ * arrival counters (at that fixed place whatever the call), the partial
+ * tiles follow.  Zero-filled before first use; every call leaves the
+ * counters zeroed (after Q4_STATUS_TIMEOUT, zero-fill it again). */
+Q4_API int q4_gemm_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes);
+
 /*
  * q4_gemm -- the same product for any M >= 1, computed by dequantizing
  * weight tiles into shared memory (bit-exact w^ in a_dtype) and feeding
@@ -287,15 +297,21 @@ Q4_API int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *
  *       INT4 symmetric and cvt(s * (q - z)) for INT4 asymmetric: bit for
  *       bit what q4_dequantize gives.
  *   Y   device, y_dtype (a_dtype or Q4_F32), [M, N] row-major.
+ *   workspace  device, 16-byte aligned, q4_gemm_workspace_size() bytes,
+ *       zero-filled; or NULL / fewer bytes: then no tile is cut (the same
+ *       result, only the balance of the CTAs differs).  A cut tile's two
+ *       partial sums are added once, a + b, so the bits do not depend on
+ *       which half finishes first.
  * Same tolerance as q4_gemv.  A grouped call takes one format (qtype,
  * blocksize, double_quant) for all its matrices (Q4_ERR_ARG otherwise).
  */
 Q4_API int q4_gemm(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
-            int32_t y_dtype, void *stream);
+            int32_t y_dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /* q4_gemm over `count` (1..16) matrices in one persistent launch. */
 Q4_API int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
-                    void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *stream);
+                    void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace,
+                    size_t workspace_bytes, void *stream);
 
 /* ---- status and introspection ----------------------------------------- */
 

@@ -233,7 +233,7 @@ def test_gemm_host_checks_before_the_device(lib):
         n = len(states)
         arr = (P * n)(*[ctypes.pointer(st) for st in states])
         ptrs = (ctypes.c_void_p * n)(*([0x70000] * n))
-        return lib.q4_gemm_grouped(n, ptrs, arr, ptrs, M, 1, 1, None)
+        return lib.q4_gemm_grouped(n, ptrs, arr, ptrs, M, 1, 1, None, 0, None)
     for qt, dq in ((0, False), (0, True), (1, False), (2, False)):
         for bs in (32, 64, 128, 256):
             assert gemm([_fake_state(qt, 256, 1024, bs, dq)]) == -4  # Q4_ERR_NO_DEVICE
@@ -242,6 +242,25 @@ def test_gemm_host_checks_before_the_device(lib):
     assert gemm([_fake_state(1, 256, 96, 32, False)]) == -2      # K % 64
     assert gemm([_fake_state(1, 256, 384, 256, False)]) == -2    # K % B
     assert gemm([_fake_state(2, 250, 1024, 128, False)]) == -2   # N % 16
+
+
+def test_gemm_workspace_size_host_checks(lib):
+    """The GEMM workspace size takes the same shape and format checks as
+    the GEMM (mixed formats Q4_ERR_ARG, K % 64 a shape error) before it
+    asks for the device (its plan depends on the SM count)."""
+    from bit_blockwise_weight_absmax_b200 import q4
+    P = ctypes.POINTER(q4._CState)
+
+    def size(states, M=512):
+        arr = (P * len(states))(*[ctypes.pointer(st) for st in states])
+        out = ctypes.c_size_t(7)
+        return lib.q4_gemm_workspace_size(len(states), arr, M, ctypes.byref(out))
+    assert size([_fake_state(0, 256, 1024, 64, True)]) == -4  # Q4_ERR_NO_DEVICE
+    assert size([_fake_state(0, 256, 1024, 64, True), _fake_state(1, 256, 1024, 64, False)]) == -1
+    assert size([_fake_state(1, 256, 96, 32, False)]) == -2
+    assert size([_fake_state(0, 256, 1024, 64, True)], M=0) == -2
+    arr = (P * 1)(ctypes.pointer(_fake_state(0, 256, 1024, 64, True)))
+    assert lib.q4_gemm_workspace_size(1, arr, 512, None) == -1
 
 
 def test_grouped_calls_reject_a_null_entry_before_any_use(lib):
@@ -255,13 +274,13 @@ def test_grouped_calls_reject_a_null_entry_before_any_use(lib):
         arr = (P * 2)(ctypes.pointer(good), P())
         ptrs = (ctypes.c_void_p * 2)(0x70000, 0x70000)
         assert lib.q4_gemv_grouped(2, ptrs, arr, ptrs, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None) == -1
-        assert lib.q4_gemm_grouped(2, ptrs, arr, ptrs, 512, 1, 1, None) == -1
+        assert lib.q4_gemm_grouped(2, ptrs, arr, ptrs, 512, 1, 1, None, 0, None) == -1
         arr = (P * 2)(ctypes.pointer(good), ctypes.pointer(good))
         for bad in ((ctypes.c_void_p * 2)(0x70000, None),):
             assert lib.q4_gemv_grouped(2, bad, arr, ptrs, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None) == -1
             assert lib.q4_gemv_grouped(2, ptrs, arr, bad, M, 0, 0, ctypes.c_void_p(0x80000), 1 << 30, None) == -1
-            assert lib.q4_gemm_grouped(2, bad, arr, ptrs, 512, 1, 1, None) == -1
-            assert lib.q4_gemm_grouped(2, ptrs, arr, bad, 512, 1, 1, None) == -1
+            assert lib.q4_gemm_grouped(2, bad, arr, ptrs, 512, 1, 1, None, 0, None) == -1
+            assert lib.q4_gemm_grouped(2, ptrs, arr, bad, 512, 1, 1, None, 0, None) == -1
 
 
 def test_binary16_scale_sizes_and_checks(lib, oracle):
@@ -286,4 +305,4 @@ def test_binary16_scale_sizes_and_checks(lib, oracle):
     P = ctypes.POINTER(q4._CState)
     arr = (P * 1)(ctypes.pointer(st))
     ptrs = (ctypes.c_void_p * 1)(0x70000)
-    assert lib.q4_gemm_grouped(1, ptrs, arr, ptrs, 512, 1, 1, None) == -1
+    assert lib.q4_gemm_grouped(1, ptrs, arr, ptrs, 512, 1, 1, None, 0, None) == -1

@@ -40,6 +40,42 @@ def test_gemm_one_tile(q4, oracle):
     assert_matmul_close(y, ref)
 
 
+def test_gemm_split_k_few_tiles(q4, oracle):
+    """One matrix of few tiles (M = 512, N = 2048, K = 4608: 32 tiles for
+    many more SMs): the launch cuts tiles into k halves whose partials meet
+    in the workspace.  Against the oracle, bit-identical on repeat, the
+    workspace left zeroed, and within tolerance of the uncut launch."""
+    import ctypes
+    g = torch.Generator().manual_seed(12)
+    M, N, K = 512, 2048, 4608
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).bfloat16()
+    st = q4.quantize(W.cuda(), 64, "nf4", True)
+    ost = oracle_state(oracle, W, 64, 0, True)
+    arr = (ctypes.POINTER(q4._CState) * 1)(ctypes.pointer(st.c_struct()))
+    wsz = ctypes.c_size_t(0)
+    assert q4.library().q4_gemm_workspace_size(1, arr, M, ctypes.byref(wsz)) == 0
+    assert wsz.value > 0  # the plan cuts tiles
+    a = A.cuda()
+    ys = [q4.gemm(a, st) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+    rows = np.arange(0, N, 7)
+    w16 = oracle.dequantize(ost, True).reshape(N, K)[rows]
+    ref = oracle.matmul(bits(A), True, w16, True, M, len(rows), K)
+    assert_matmul_close(ys[0][:, torch.from_numpy(rows).cuda()], ref)
+    # the arrival counters (the workspace's first 64 KB) are left zeroed
+    ws = q4._workspace(a.device, "gemm", wsz.value)
+    assert int(ws[:65536].count_nonzero()) == 0
+    # the uncut launch (no workspace) gives the same product within tolerance
+    y1 = torch.empty_like(ys[0])
+    assert q4.library().q4_gemm(a.data_ptr(), 1, M, ctypes.pointer(st.c_struct()), y1.data_ptr(), 1,
+                                None, 0, None) == 0
+    torch.cuda.synchronize()
+    assert_matmul_close(y1[:, torch.from_numpy(rows).cuda()], ref)
+
+
 def test_gemm_exact_small_integers(q4, oracle):
     """A in {-1, 0, 1}, every block's maximum 1 (so w^ is the bf16 level),
     K = 64, fp32 output: each partial sum of the tensor cores is exactly
