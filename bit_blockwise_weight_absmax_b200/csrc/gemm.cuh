@@ -15,16 +15,23 @@
 //   warp 0      TMA producer: the A tile [256 x 64] (128B-swizzled, K-major)
 //               and the raw packed tile [128 rows x 32 bytes] per k-block,
 //               into a ring of 4 stages.
-//   warp 1      TMEM allocator and MMA issuer: per k-block 2 x 4
-//               tcgen05.mma kind::f16 (M=128, N=128, K=16) into two fp32
-//               accumulators of 128 columns; the two accumulator sets of a
-//               tile alternate between tiles (512 TMEM columns), so the
-//               epilogue of one tile overlaps the MMAs of the next.
+//   warp 1      TMEM allocator and MMA issuer: per k-block 4
+//               tcgen05.mma kind::f16 (M=128 weight rows, N=256 tokens,
+//               K=16) into one fp32 accumulator of 256 columns (a TMEM lane
+//               per weight row, a column per token); two accumulators
+//               alternate between tiles (512 TMEM columns), so the epilogue
+//               of one tile overlaps the MMAs of the next.  With the weight
+//               tile on the M side each MMA reads 12 KB of shared memory
+//               for 128 tensor cycles (two N=128 MMAs over the token halves
+//               read 16 KB), and shared-memory bandwidth is what the MMAs,
+//               the copies and the dequant stores share.
 //   warps 2..17 dequant: four threads per weight row, 16 codes each, scaled
 //               by the row's block scale into bf16/fp16 and written in the
 //               128B-swizzled K-major layout the UMMA descriptor reads; the
 //               block scales come 16 blocks per load.  Then the epilogue:
-//               tcgen05.ld of the accumulators, convert, store.
+//               tcgen05.ld of the accumulators (a lane per weight row, 16
+//               tokens at a time), convert, store one token row's 32
+//               consecutive outputs per warp instruction.
 // Every mbarrier wait is bounded in time; a timeout sets Q4_STATUS_TIMEOUT,
 // stops the pipeline, waits for issued copies and for the issued MMAs, and
 // frees TMEM.
@@ -46,10 +53,10 @@ constexpr int kGemmBTile = kGemmBN * kGemmBK * 2;   // 16 KB
 constexpr int kGemmRawTile = kGemmBN * kGemmBK / 2; // 4 KB
 constexpr int kGemmStageBytes = kGemmATile + kGemmBTile + kGemmRawTile;
 constexpr int kGemmScBytes = kGemmBN * 16 * 4;     // c~ of 16 blocks per weight row
-constexpr int kGemmAccs = kGemmBM / 128;            // M=128 accumulators per tile
 constexpr int kGemmTpr = kGemmDqWarps * 32 / kGemmBN;  // dequant threads per weight row
 constexpr int kGemmCodes = kGemmBK / kGemmTpr;      // codes per thread and stage
-static_assert(kGemmBM % 128 == 0 && 2 * kGemmAccs * kGemmBN <= 512, "two accumulator sets in TMEM");
+static_assert(kGemmBN == 128 && kGemmBM % 16 == 0 && kGemmBM <= 256, "UMMA M = 128 (weight rows), N = tokens");
+static_assert(2 * kGemmBM <= 512, "two accumulators in TMEM");
 static_assert(kGemmCodes == 16 || kGemmCodes == 32, "8 or 16 packed bytes per thread");
 constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmScBytes + 1024 /*align*/ + 256 /*barriers*/;
 
@@ -278,40 +285,32 @@ __device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t v) {
 }
 
 // Epilogue helpers.  A dequant warp's share of a tile: TMEM lanes q * 32 ..
-// + 31 (its quadrant) and accumulator columns cc * 32 .. + 31 of both
-// accumulators, in four chunks of 16 columns (ch = 2 accumulator + half).
-__device__ __forceinline__ uint32_t gemm_chunk(uint32_t tmem, int ab, int ch, int q, int cc, int &h, int &c16) {
-  const int piece = ch >> 1, hh = ch & 1;
-  h = piece / (kGemmBN / 128);
-  const int part = piece % (kGemmBN / 128);
-  c16 = cc * (kGemmBN / 4) + part * 32 + 16 * hh;
-  return tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)((ab * kGemmAccs + h) * kGemmBN + c16);
+// + 31 (its quadrant: weight rows q * 32 .. + 31 of the tile) and the
+// accumulator's token columns cc * 64 .. + 63, in four chunks of 16.
+__device__ __forceinline__ uint32_t gemm_chunk(uint32_t tmem, int ab, int ch, int q, int cc, int &t16) {
+  t16 = cc * (kGemmBM / 4) + 16 * ch;
+  return tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kGemmBM + t16);
 }
-constexpr int kGemmChunks = kGemmAccs * kGemmBN / 128 * 2;  // 16-column chunks per warp
+constexpr int kGemmChunks = kGemmBM / 4 / 16;  // 16-column chunks per warp
 static_assert(kGemmChunks * 32 * 16 == kGemmSplitWarpFloats, "split-K partial layout");
-// Y[mrow, n0 .. n0 + 15] of one lane (its row) from 16 fp32 accumulators.
-__device__ __forceinline__ void gemm_store_y(const GemmMat &m, int y_dtype, int mrow, int n0, const uint32_t (&r)[16]) {
-  if (mrow >= m.M || n0 >= m.N) return;
+// Y[t0 .. t0 + 15, n] of one lane (its weight row n) from 16 fp32
+// accumulators; the warp's 32 lanes are 32 consecutive n, so each store
+// instruction writes one contiguous run of a Y row.
+__device__ __forceinline__ void gemm_store_y(const GemmMat &m, int y_dtype, int n, int t0, const uint32_t (&r)[16]) {
+  if (n >= m.N || t0 >= m.M) return;
+  const int nt = min(16, m.M - t0);
   if (y_dtype == Q4_F32) {
-    float *y = reinterpret_cast<float *>(m.Y) + (int64_t)mrow * m.N + n0;
+    float *y = reinterpret_cast<float *>(m.Y) + (int64_t)t0 * m.N + n;
 #pragma unroll
-    for (int v = 0; v < 4; ++v)
-      if (n0 + 4 * v < m.N)
-        *reinterpret_cast<uint4 *>(y + 4 * v) = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+    for (int j = 0; j < 16; ++j)
+      if (j < nt) y[(int64_t)j * m.N] = __uint_as_float(r[j]);
   } else {
-    uint16_t *y = reinterpret_cast<uint16_t *>(m.Y) + (int64_t)mrow * m.N + n0;
+    uint16_t *y = reinterpret_cast<uint16_t *>(m.Y) + (int64_t)t0 * m.N + n;
 #pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      if (n0 + 8 * v < m.N) {
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float f0 = __uint_as_float(r[8 * v + 2 * e]), f1 = __uint_as_float(r[8 * v + 2 * e + 1]);
-          o[e] = (y_dtype == Q4_BF16) ? Dt<Q4_BF16>::pack2(f0, f1) : Dt<Q4_F16>::pack2(f0, f1);
-        }
-        *reinterpret_cast<uint4 *>(y + 8 * v) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
+    for (int j = 0; j < 16; ++j)
+      if (j < nt)
+        y[(int64_t)j * m.N] = (y_dtype == Q4_BF16) ? Dt<Q4_BF16>::from_f(__uint_as_float(r[j]))
+                                                   : Dt<Q4_F16>::from_f(__uint_as_float(r[j]));
   }
 }
 // Split-K epilogue of one warp's share of a cut tile.  The half's fp32 partial is published, then counted; the warp that
@@ -324,9 +323,9 @@ static __device__ __forceinline__ void gemm_split_epilogue(const GemmParams *pp,
   float *mine = p.partials + ((int64_t)(slot * 2 + half) * 16 + wp) * kGemmSplitWarpFloats;
 #pragma unroll 1
   for (int ch = 0; ch < kGemmChunks; ++ch) {
-    int h, c16;
+    int t16;
     uint32_t r[16];
-    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, h, c16), r);
+    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, t16), r);
     float4 *dst = reinterpret_cast<float4 *>(mine + (ch * 32 + lane) * 16);
 #pragma unroll
     for (int v = 0; v < 4; ++v)
@@ -343,9 +342,9 @@ static __device__ __forceinline__ void gemm_split_epilogue(const GemmParams *pp,
   const float *other = p.partials + ((int64_t)(slot * 2 + (1 - half)) * 16 + wp) * kGemmSplitWarpFloats;
 #pragma unroll 1
   for (int ch = 0; ch < kGemmChunks; ++ch) {
-    int h, c16;
+    int t16;
     uint32_t r[16];
-    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, h, c16), r);
+    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, t16), r);
     const float4 *src = reinterpret_cast<const float4 *>(other + (ch * 32 + lane) * 16);
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
@@ -355,7 +354,7 @@ static __device__ __forceinline__ void gemm_split_epilogue(const GemmParams *pp,
       r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + o.z);
       r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + o.w);
     }
-    gemm_store_y(m, p.y_dtype, tm * kGemmBM + h * 128 + q * 32 + lane, tn * kGemmBN + c16, r);
+    gemm_store_y(m, p.y_dtype, tn * kGemmBN + q * 32 + lane, tm * kGemmBM + t16, r);
   }
   if (lane == 0) p.split_cnt[slot * 16 + wp] = 0u;  // the workspace is left zeroed
 }
@@ -456,8 +455,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_f16(DA == Q4_BF16 ? 1 : 0, 128, kGemmBN);
-      static_assert(kGemmBN % 16 == 0 && kGemmBN <= 256, "UMMA N for M = 128");
+      // M = 128 weight rows (the dequantized tile), N = kGemmBM tokens
+      const uint32_t idesc = umma_idesc_f16(DA == Q4_BF16 ? 1 : 0, kGemmBN, kGemmBM);
       uint32_t it = 0, tcount = 0;
       uint32_t last_bar = 0, last_par = 0;  // the barrier and phase of the last commit issued
       bool committed = false;
@@ -479,14 +478,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           const uint32_t a0 = smem_u32(sA + s * kGemmATile);
           const uint32_t b0 = smem_u32(sB + s * kGemmBTile);
 #pragma unroll
-          for (int k16 = 0; k16 < kGemmBK / 16; ++k16) {
-            const uint64_t db = umma_desc_sw128(b0 + 32 * k16);
-#pragma unroll
-            for (int h = 0; h < kGemmAccs; ++h) {
-              const uint64_t da = umma_desc_sw128(a0 + h * (128 * kGemmBK * 2) + 32 * k16);
-              umma_f16(tmem + (uint32_t)((ab * kGemmAccs + h) * kGemmBN), da, db, idesc, kb != tc.kb0 || k16 != 0);
-            }
-          }
+          for (int k16 = 0; k16 < kGemmBK / 16; ++k16)
+            umma_f16(tmem + (uint32_t)(ab * kGemmBM), umma_desc_sw128(b0 + 32 * k16), umma_desc_sw128(a0 + 32 * k16),
+                     idesc, kb != tc.kb0 || k16 != 0);
           umma_commit(empty_bar(s));
           last_bar = empty_bar(s), last_par = use & 1, committed = true;
         }
@@ -526,10 +520,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         const GemmMat &m = p.mat[tc.mi];
 #pragma unroll 1
         for (int ch = 0; ch < kGemmChunks; ++ch) {
-          int h, c16;
+          int t16;
           uint32_t r[16];
-          tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, h, c16), r);
-          gemm_store_y(m, p.y_dtype, tc.tm * kGemmBM + h * 128 + q * 32 + lane, tc.tn * kGemmBN + c16, r);
+          tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, t16), r);
+          gemm_store_y(m, p.y_dtype, tc.tn * kGemmBN + q * 32 + lane, tc.tm * kGemmBM + t16, r);
         }
       }
       tc_fence_before();
