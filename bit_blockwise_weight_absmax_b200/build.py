@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libq4.so")
 BUILD = os.path.join(HERE, "_build")
-UNITS = ["q4_api.cu", "k_quantize.cu", "k_dequantize.cu", "k_gemv_small.cu", "k_gemv_small_asym.cu", "k_gemm.cu", "k_gemm_split.cu",
+UNITS = ["q4_api.cu", "k_quantize.cu", "k_dequantize.cu", "k_gemv_small.cu", "k_gemv_small_asym.cu", "k_gemm.cu", "k_gemm_low.cu", "k_gemm_split.cu", "k_gemm_split_low.cu",
          "q4_noalloc.cu"]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -42,23 +42,42 @@
 
 namespace q4 {
 
-constexpr int kGemmBM = 256;
-constexpr int kGemmBN = 128;
+constexpr int kGemmBM = 512;      // tokens per tile (at most; a launch may use tiles of kGemmHalfM)
+constexpr int kGemmHalfM = 256;   // tokens per MMA (UMMA N) and per activation slot
+constexpr int kGemmBN = 128;      // weight rows per tile (UMMA M)
 constexpr int kGemmBK = 64;
-constexpr int kGemmStages = 4;
+constexpr int kGemmStages = 4;    // ring of dequant stages (raw codes in, 16-bit weight tile out)
+constexpr int kGemmASlots = 4;    // ring of activation half tiles (two per k-block)
 constexpr int kGemmDqWarps = 16;                          // dequant + epilogue warps (2..17)
 constexpr int kGemmThreads = (2 + kGemmDqWarps) * 32;
-constexpr int kGemmATile = kGemmBM * kGemmBK * 2;   // 32 KB
-constexpr int kGemmBTile = kGemmBN * kGemmBK * 2;   // 16 KB
-constexpr int kGemmRawTile = kGemmBN * kGemmBK / 2; // 4 KB
-constexpr int kGemmStageBytes = kGemmATile + kGemmBTile + kGemmRawTile;
-constexpr int kGemmScBytes = kGemmBN * 16 * 4;     // c~ of 16 blocks per weight row
+constexpr int kGemmATile = kGemmHalfM * kGemmBK * 2;  // 32 KB: one activation half tile
+constexpr int kGemmBTile = kGemmBN * kGemmBK * 2;     // 16 KB
+constexpr int kGemmRawTile = kGemmBN * kGemmBK / 2;   // 4 KB
+constexpr int kGemmScBytes = kGemmBN * 16 * 4;       // c~ of 16 blocks per weight row
 constexpr int kGemmTpr = kGemmDqWarps * 32 / kGemmBN;  // dequant threads per weight row
 constexpr int kGemmCodes = kGemmBK / kGemmTpr;      // codes per thread and stage
-static_assert(kGemmBN == 128 && kGemmBM % 16 == 0 && kGemmBM <= 256, "UMMA M = 128 (weight rows), N = tokens");
-static_assert(2 * kGemmBM <= 512, "two accumulators in TMEM");
+// Per tile height (TALL: kGemmBM tokens, else kGemmHalfM):
+//  - accumulators in TMEM's 512 columns: one, or two that alternate so that
+//    an epilogue overlaps the next tile's MMAs;
+//  - the epilogue of a tile runs after this many dequant stages of the
+//    next: with two accumulators a ring's worth (its stores overlap the
+//    MMAs of those stages); with one two stages, about when the MMAs of its
+//    tile end, so that they find the next stages ready;
+//  - raw codes are issued this many k-blocks ahead of the activations: the
+//    activation ring holds two k-blocks of tall tiles and four of low ones,
+//    the raw ring four, so the lead evens the two rings' look-ahead.
+template <bool TALL> struct GemmShape {
+  static constexpr int kTileM = TALL ? kGemmBM : kGemmHalfM;
+  static constexpr int kSets = TALL ? 1 : 2;
+  static constexpr int kEpiAfter = TALL ? 2 : kGemmStages;
+  static constexpr int kRawLead = TALL ? 2 : 0;
+  static_assert(kSets * kTileM <= 512 && kRawLead < kGemmStages, "TMEM columns, raw ring");
+};
+static_assert(kGemmBN == 128 && kGemmHalfM % 16 == 0 && kGemmHalfM <= 256, "UMMA M = 128 (weight rows), N = tokens");
+static_assert(kGemmBM == 2 * kGemmHalfM && kGemmBM <= 512, "one accumulator of kGemmBM (or two of kGemmHalfM) TMEM columns");
 static_assert(kGemmCodes == 16 || kGemmCodes == 32, "8 or 16 packed bytes per thread");
-constexpr int kGemmSmem = kGemmStages * kGemmStageBytes + kGemmScBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kGemmSmem = kGemmASlots * kGemmATile + kGemmStages * (kGemmBTile + kGemmRawTile) + kGemmScBytes +
+                          1024 /*align*/ + 256 /*barriers*/;
 
 struct alignas(64) GemmMat {
   CUtensorMap tmA;  // A [M, K] 16-bit, box {64, 256}, 128B swizzle
@@ -85,7 +104,7 @@ struct alignas(64) GemmMat {
 // 2 second), 18-31 split slot.
 constexpr int kGemmListTiles = 2048;
 constexpr int kGemmListCtas = 256;  // grid bound of a listed launch
-constexpr int kGemmSplitWarpFloats = 2 * 2 * 32 * 16;  // one epilogue warp's partial: pieces x halves x lanes x 16
+constexpr int kGemmSplitWarpFloats = kGemmBM / 4 * 32;  // one epilogue warp's partial: its columns x lanes
 constexpr size_t kGemmSplitSlotBytes = 2 * 16 * kGemmSplitWarpFloats * sizeof(float);  // two halves x 16 warps
 // The arrival counters sit at the start of the workspace in a region of a
 // fixed size (every slot a listed launch can have), so that whatever slot
@@ -105,6 +124,7 @@ struct GemmParams {
   int *status;
   float levels[16];
   int32_t listed;        // items come from tile_list (else whole tiles round robin)
+  int32_t tile_m;        // tokens per tile: kGemmBM (one accumulator) or kGemmHalfM (two, alternating); picks the instance
   int32_t grid;          // CTAs of the launch
   unsigned *split_cnt;   // split-K: [slot][epilogue warp] arrivals (zero between calls), at the workspace start
   float *partials;       // split-K: [slot][half][epilogue warp][kGemmSplitWarpFloats] fp32, after the counters
@@ -284,15 +304,22 @@ __device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t v) {
   return tc;
 }
 
-// Epilogue helpers.  A dequant warp's share of a tile: TMEM lanes q * 32 ..
-// + 31 (its quadrant: weight rows q * 32 .. + 31 of the tile) and the
-// accumulator's token columns cc * 64 .. + 63, in four chunks of 16.
+// Epilogue helpers.  A dequant warp's share of a tile of TM tokens: TMEM
+// lanes q * 32 .. + 31 (its quadrant: weight rows q * 32 .. + 31 of the
+// tile) and the accumulator's token columns cc * TM / 4 .. + TM / 4 - 1, in
+// TM / 64 chunks of 16.
+template <int TM>
 __device__ __forceinline__ uint32_t gemm_chunk(uint32_t tmem, int ab, int ch, int q, int cc, int &t16) {
-  t16 = cc * (kGemmBM / 4) + 16 * ch;
-  return tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kGemmBM + t16);
+  t16 = cc * (TM / 4) + 16 * ch;
+  return tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * TM + t16);
 }
-constexpr int kGemmChunks = kGemmBM / 4 / 16;  // 16-column chunks per warp
-static_assert(kGemmChunks * 32 * 16 == kGemmSplitWarpFloats, "split-K partial layout");
+static_assert(kGemmBM / 64 * 32 * 16 == kGemmSplitWarpFloats, "split-K partial layout");
+// Token halves of tile tm that hold any of the M tokens (the second half of
+// the last tall tile may lie wholly past M: it is neither loaded nor
+// multiplied).
+template <bool TALL> __device__ __forceinline__ int gemm_halves(const GemmMat &m, int tm) {
+  return TALL && tm * kGemmBM + kGemmHalfM < m.M ? 2 : 1;
+}
 // Y[t0 .. t0 + 15, n] of one lane (its weight row n) from 16 fp32
 // accumulators; the warp's 32 lanes are 32 consecutive n, so each store
 // instruction writes one contiguous run of a Y row.
@@ -316,16 +343,21 @@ __device__ __forceinline__ void gemm_store_y(const GemmMat &m, int y_dtype, int 
 // Split-K epilogue of one warp's share of a cut tile.  The half's fp32 partial is published, then counted; the warp that
 // completes the count adds the other half's partial (a + b: the same bits
 // whichever half finishes second), writes Y and zeroes the counter.
+template <bool TALL>
 static __device__ __forceinline__ void gemm_split_epilogue(const GemmParams *pp, uint32_t tmem, int ab, int mi, int tm,
                                                         int tn, int slot, int half, int q, int cc, int lane, int wp) {
   const GemmParams &p = *pp;
   const GemmMat &m = p.mat[mi];
   float *mine = p.partials + ((int64_t)(slot * 2 + half) * 16 + wp) * kGemmSplitWarpFloats;
+  constexpr int TM = GemmShape<TALL>::kTileM, nch = TM / 64;
+  const int ncols = gemm_halves<TALL>(m, tm) * kGemmHalfM;  // accumulator columns the tile filled
 #pragma unroll 1
-  for (int ch = 0; ch < kGemmChunks; ++ch) {
+  for (int ch = 0; ch < nch; ++ch) {
     int t16;
     uint32_t r[16];
-    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, t16), r);
+    const uint32_t ta = gemm_chunk<TM>(tmem, ab, ch, q, cc, t16);
+    if (t16 >= ncols) break;
+    tmem_ld16(ta, r);
     float4 *dst = reinterpret_cast<float4 *>(mine + (ch * 32 + lane) * 16);
 #pragma unroll
     for (int v = 0; v < 4; ++v)
@@ -341,10 +373,12 @@ static __device__ __forceinline__ void gemm_split_epilogue(const GemmParams *pp,
   __threadfence();
   const float *other = p.partials + ((int64_t)(slot * 2 + (1 - half)) * 16 + wp) * kGemmSplitWarpFloats;
 #pragma unroll 1
-  for (int ch = 0; ch < kGemmChunks; ++ch) {
+  for (int ch = 0; ch < nch; ++ch) {
     int t16;
     uint32_t r[16];
-    tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, t16), r);
+    const uint32_t ta = gemm_chunk<TM>(tmem, ab, ch, q, cc, t16);
+    if (t16 >= ncols) break;
+    tmem_ld16(ta, r);
     const float4 *src = reinterpret_cast<const float4 *>(other + (ch * 32 + lane) * 16);
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
@@ -354,7 +388,7 @@ static __device__ __forceinline__ void gemm_split_epilogue(const GemmParams *pp,
       r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + o.z);
       r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + o.w);
     }
-    gemm_store_y(m, p.y_dtype, tn * kGemmBN + q * 32 + lane, tm * kGemmBM + t16, r);
+    gemm_store_y(m, p.y_dtype, tn * kGemmBN + q * 32 + lane, tm * TM + t16, r);
   }
   if (lane == 0) p.split_cnt[slot * 16 + wp] = 0u;  // the workspace is left zeroed
 }
@@ -367,18 +401,19 @@ constexpr int kGemmPlain = 0, kGemmDq = 1, kGemmAsym = 2;
 // tiles (the instance without them carries no split-K code, so its
 // registers do not spill).  The blocksize is a launch parameter: it only
 // decides which block scale a thread's 16 codes take.
-template <int DA, int MODE, bool SPLIT>
+template <int DA, int MODE, bool SPLIT, bool TALL>
 __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr bool DQ = MODE == kGemmDq, ASYM = MODE == kGemmAsym;
+  using Sh = GemmShape<TALL>;
   pdl_launch_dependents();  // set-up (barriers, TMEM, level table) overlaps the previous kernel
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *sA = smem;                                        // [stages][32 KB]
-  uint8_t *sB = smem + kGemmStages * kGemmATile;             // [stages][16 KB]
+  uint8_t *sA = smem;                                        // [activation slots][32 KB]
+  uint8_t *sB = smem + kGemmASlots * kGemmATile;             // [stages][16 KB]
   uint8_t *sR = sB + kGemmStages * kGemmBTile;               // [stages][4 KB]
   float *sSc = reinterpret_cast<float *>(sR + kGemmStages * kGemmRawTile);  // [128 rows][16]
   uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(sSc) + kGemmScBytes);
-  // bars: full[S], bfull[S], empty[S], accfull[2], accempty[2]
+  // bars: full[S], bfull[S], empty[S], accfull[2], accempty[2], afull[AS], aempty[AS]
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ float s_lv[16 * 32];
@@ -391,6 +426,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   auto empty_bar = [&](int s) { return bar0 + 8u * (2 * kGemmStages + s); };
   auto accfull_bar = [&](int b) { return bar0 + 8u * (3 * kGemmStages + b); };
   auto accempty_bar = [&](int b) { return bar0 + 8u * (3 * kGemmStages + 2 + b); };
+  auto afull_bar = [&](int a) { return bar0 + 8u * (3 * kGemmStages + 4 + a); };
+  auto aempty_bar = [&](int a) { return bar0 + 8u * (3 * kGemmStages + 4 + kGemmASlots + a); };
+  static_assert(8 * (3 * kGemmStages + 4 + 2 * kGemmASlots) <= 256, "barrier area");
 
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
@@ -401,6 +439,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     for (int b = 0; b < 2; ++b) {
       mbar_init(accfull_bar(b), 1);
       mbar_init(accempty_bar(b), kGemmDqWarps);
+    }
+    for (int a = 0; a < kGemmASlots; ++a) {
+      mbar_init(afull_bar(a), 1);
+      mbar_init(aempty_bar(a), 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     s_abort = 0;
@@ -431,62 +473,130 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t it = 0;
-      for (int64_t k = 0; k < n_my && !*abort; ++k) {
-        const TileCoord tc = gemm_tile(p, my_tile(k));
-        const GemmMat &m = p.mat[tc.mi];
-        for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
-          const int s = it % kGemmStages;
-          const uint32_t use = it / kGemmStages;
-          if (!mbar_wait(empty_bar(s), (use & 1) ^ 1, p.status, abort, p.wait_ns)) break;
-          if (p.stall_copies) continue;  // test hook: the stage is never filled
-          mbar_arrive_expect_tx(full_bar(s), kGemmATile + kGemmRawTile);
-          tma_load_2d(smem_u32(sA + s * kGemmATile), &m.tmA, full_bar(s), kb * kGemmBK, tc.tm * kGemmBM);
-          tma_load_2d(smem_u32(sR + s * kGemmRawTile), &m.tmW, full_bar(s), kb * (kGemmBK / 2), tc.tn * kGemmBN);
+      // Two cursors over this CTA's (item, k-block) sequence: the raw codes
+      // run kGemmRawLead k-blocks ahead of the activation halves, so that a
+      // stage's codes land and are dequantized while the MMAs still work on
+      // earlier k-blocks (the activation ring holds two k-blocks).
+      struct Cur {
+        int64_t k;  // item index; n_my when the sequence is exhausted
+        int kb;
+        TileCoord tc;
+      };
+      auto cur_init = [&](Cur &c) {
+        c.k = 0;
+        c.kb = 0;
+        if (n_my > 0) {
+          c.tc = gemm_tile(p, my_tile(0));
+          c.kb = c.tc.kb0;
         }
+      };
+      auto cur_next = [&](Cur &c) {
+        if (++c.kb == c.tc.kb1 && ++c.k < n_my) {
+          c.tc = gemm_tile(p, my_tile(c.k));
+          c.kb = c.tc.kb0;
+        }
+      };
+      Cur cr, ca;
+      cur_init(cr);
+      cur_init(ca);
+      uint32_t it = 0, ia = 0;  // dequant stages and activation half tiles issued
+      auto issue_raw = [&]() -> bool {
+        const int s = it % kGemmStages;
+        if (!mbar_wait(empty_bar(s), ((it / kGemmStages) & 1) ^ 1, p.status, abort, p.wait_ns)) return false;
+        if (!p.stall_copies) {  // test hook: no stage is ever filled
+          mbar_arrive_expect_tx(full_bar(s), kGemmRawTile);
+          tma_load_2d(smem_u32(sR + s * kGemmRawTile), &p.mat[cr.tc.mi].tmW, full_bar(s), cr.kb * (kGemmBK / 2),
+                      cr.tc.tn * kGemmBN);
+        }
+        ++it;
+        cur_next(cr);
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; j < Sh::kRawLead && cr.k < n_my && ok; ++j) ok = issue_raw();
+      while (ok && ca.k < n_my && !*abort) {
+        if (cr.k < n_my && !(ok = issue_raw())) break;
+        const GemmMat &m = p.mat[ca.tc.mi];
+        const int nh = gemm_halves<TALL>(m, ca.tc.tm);
+        for (int h = 0; h < nh; ++h) {
+          const int a = ia % kGemmASlots;
+          if (!mbar_wait(aempty_bar(a), ((ia / kGemmASlots) & 1) ^ 1, p.status, abort, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          if (!p.stall_copies) {
+            mbar_arrive_expect_tx(afull_bar(a), kGemmATile);
+            tma_load_2d(smem_u32(sA + a * kGemmATile), &m.tmA, afull_bar(a), ca.kb * kGemmBK,
+                        ca.tc.tm * Sh::kTileM + h * kGemmHalfM);
+          }
+          ++ia;
+        }
+        cur_next(ca);
       }
-      // every issued copy completes before the CTA may exit
+      // every issued copy completes before the CTA may exit (only the last
+      // use of each ring slot can still be in flight)
       for (uint32_t j = (it > kGemmStages ? it - kGemmStages : 0); j < it && !p.stall_copies; ++j) {
         int dummy = 0;
         volatile int no_abort = 0;
         mbar_wait(full_bar(j % kGemmStages), (j / kGemmStages) & 1, &dummy, &no_abort);
       }
+      for (uint32_t j = (ia > kGemmASlots ? ia - kGemmASlots : 0); j < ia && !p.stall_copies; ++j) {
+        int dummy = 0;
+        volatile int no_abort = 0;
+        mbar_wait(afull_bar(j % kGemmASlots), (j / kGemmASlots) & 1, &dummy, &no_abort);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // M = 128 weight rows (the dequantized tile), N = kGemmBM tokens
-      const uint32_t idesc = umma_idesc_f16(DA == Q4_BF16 ? 1 : 0, kGemmBN, kGemmBM);
-      uint32_t it = 0, tcount = 0;
+      // M = 128 weight rows (the dequantized tile), N = kGemmHalfM tokens;
+      // both token halves of a k-block multiply the same weight stage
+      const uint32_t idesc = umma_idesc_f16(DA == Q4_BF16 ? 1 : 0, kGemmBN, kGemmHalfM);
+      uint32_t it = 0, ia = 0, tcount = 0;
       uint32_t last_bar = 0, last_par = 0;  // the barrier and phase of the last commit issued
-      bool committed = false;
-      for (int64_t k = 0; k < n_my && !*abort; ++k, ++tcount) {
+      bool committed = false, ok = true;
+      for (int64_t k = 0; k < n_my && ok && !*abort; ++k, ++tcount) {
         const TileCoord tc = gemm_tile(p, my_tile(k));
-        const int ab = tcount & 1;  // accumulator set of this tile
-        if (!mbar_wait(accempty_bar(ab), ((tcount >> 1) & 1) ^ 1, p.status, abort, p.wait_ns)) break;
+        const int nh = gemm_halves<TALL>(p.mat[tc.mi], tc.tm);
+        const int ab = tcount % Sh::kSets;  // accumulator of this tile
+        const uint32_t aph = (tcount / Sh::kSets) & 1;
+        if (!mbar_wait(accempty_bar(ab), aph ^ 1, p.status, abort, p.wait_ns)) break;
         tc_fence_after();
-        bool ok = true;
-        for (int kb = tc.kb0; kb < tc.kb1; ++kb, ++it) {
+        for (int kb = tc.kb0; kb < tc.kb1 && ok; ++kb) {
           const int s = it % kGemmStages;
           const uint32_t use = it / kGemmStages;
-          if (!mbar_wait(full_bar(s), use & 1, p.status, abort, p.wait_ns) ||
-              !mbar_wait(bfull_bar(s), use & 1, p.status, abort, p.wait_ns)) {
+          if (!mbar_wait(bfull_bar(s), use & 1, p.status, abort, p.wait_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + s * kGemmATile);
           const uint32_t b0 = smem_u32(sB + s * kGemmBTile);
+          for (int h = 0; h < nh; ++h) {
+            const int a = ia % kGemmASlots;
+            const uint32_t ause = ia / kGemmASlots;
+            if (!mbar_wait(afull_bar(a), ause & 1, p.status, abort, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA + a * kGemmATile);
+            const uint32_t d = tmem + (uint32_t)(ab * Sh::kTileM + h * kGemmHalfM);
 #pragma unroll
-          for (int k16 = 0; k16 < kGemmBK / 16; ++k16)
-            umma_f16(tmem + (uint32_t)(ab * kGemmBM), umma_desc_sw128(b0 + 32 * k16), umma_desc_sw128(a0 + 32 * k16),
-                     idesc, kb != tc.kb0 || k16 != 0);
+            for (int k16 = 0; k16 < kGemmBK / 16; ++k16)
+              umma_f16(d, umma_desc_sw128(b0 + 32 * k16), umma_desc_sw128(a0 + 32 * k16), idesc,
+                       kb != tc.kb0 || k16 != 0);
+            umma_commit(aempty_bar(a));
+            last_bar = aempty_bar(a), last_par = ause & 1, committed = true;
+            ++ia;
+          }
+          if (!ok) break;
           umma_commit(empty_bar(s));
           last_bar = empty_bar(s), last_par = use & 1, committed = true;
+          ++it;
         }
         if (!ok) break;
         umma_commit(accfull_bar(ab));
-        last_bar = accfull_bar(ab), last_par = (tcount >> 1) & 1, committed = true;
+        last_bar = accfull_bar(ab), last_par = aph, committed = true;
       }
       // Every MMA issued completes before the CTA may free its TMEM, also
       // after a timeout: a commit's arrival covers all earlier MMAs of this
@@ -511,19 +621,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     const int wp = warp - 2;  // this warp's share of a tile's accumulators: 0..15
     auto epilogue = [&](int64_t item, uint32_t tcount) -> bool {
       const TileCoord tc = gemm_tile(p, item);  // decoded again: one word stays live across the loop
-      const int ab = tcount & 1;
-      if (!mbar_wait_warp(accfull_bar(ab), (tcount >> 1) & 1, p.status, abort, p.wait_ns)) return false;
+      const int ab = tcount % Sh::kSets;
+      if (!mbar_wait_warp(accfull_bar(ab), (tcount / Sh::kSets) & 1, p.status, abort, p.wait_ns)) return false;
       tc_fence_after();
       if (SPLIT && tc.slot >= 0) {
-        if constexpr (SPLIT) gemm_split_epilogue(&p, tmem, ab, tc.mi, tc.tm, tc.tn, tc.slot, tc.half, q, cc, lane, wp);
+        if constexpr (SPLIT) gemm_split_epilogue<TALL>(&p, tmem, ab, tc.mi, tc.tm, tc.tn, tc.slot, tc.half, q, cc, lane, wp);
       } else {
         const GemmMat &m = p.mat[tc.mi];
+        constexpr int TM = Sh::kTileM, nch = TM / 64;
+        const int ncols = gemm_halves<TALL>(m, tc.tm) * kGemmHalfM;
 #pragma unroll 1
-        for (int ch = 0; ch < kGemmChunks; ++ch) {
+        for (int ch = 0; ch < nch; ++ch) {
           int t16;
           uint32_t r[16];
-          tmem_ld16(gemm_chunk(tmem, ab, ch, q, cc, t16), r);
-          gemm_store_y(m, p.y_dtype, tc.tn * kGemmBN + q * 32 + lane, tc.tm * kGemmBM + t16, r);
+          const uint32_t ta = gemm_chunk<TM>(tmem, ab, ch, q, cc, t16);
+          if (t16 >= ncols) break;
+          tmem_ld16(ta, r);
+          gemm_store_y(m, p.y_dtype, tc.tn * kGemmBN + q * 32 + lane, tc.tm * TM + t16, r);
         }
       }
       tc_fence_before();
@@ -682,8 +796,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
         __syncwarp();
         if (lane == 0) mbar_arrive(bfull_bar(s));
         // the previous tile's epilogue once this tile's first stages are
-        // queued: its stores overlap the MMAs of those stages
-        if (have_prev && kb - tc.kb0 == min(kGemmStages, tc.kb1 - tc.kb0) - 1) {
+        // queued (GemmShape::kEpiAfter)
+        if (have_prev && kb - tc.kb0 == min(Sh::kEpiAfter, tc.kb1 - tc.kb0) - 1) {
           if (!epilogue(prev_item, prev_count)) {
             ok = false;
             break;

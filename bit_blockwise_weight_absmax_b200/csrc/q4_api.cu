@@ -618,7 +618,17 @@ int q4_gemv(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void 
 // the second half, read back; measured at M = 512 on one B200 as about 16
 // k-blocks' time).  Larger launches deal whole tiles round robin, which is
 // then within a few percent of even.
+//
+// Tiles are kGemmBM tokens high (one accumulator; each dequantized weight
+// stage feeds two MMAs) or kGemmHalfM (two accumulators that alternate, so
+// an epilogue overlaps the next tile's MMAs; twice the dequant work per
+// flop).  The planner weighs a k-block of a token half at kGemmCostHalf in
+// the first and kGemmCostWhole in the second (measured on the 7B layer at
+// M = 512 and 2048: 820 -> 955 and 878 -> 1102 TFLOP/s) and takes the
+// height whose busiest CTA finishes first: the tall tiles unless they
+// leave most SMs idle (few tiles) or M fits one half anyway.
 constexpr int kGemmSplitCost = 16;
+constexpr int kGemmCostHalf = 17, kGemmCostWhole = 20;
 struct GemmPlan {
   int64_t grid = 0;    // CTAs
   int64_t slots = 0;   // split tiles
@@ -629,7 +639,9 @@ struct GemmPlan {
 size_t gemm_split_bytes(int64_t slots) {
   return slots ? kGemmSplitCntBytes + (size_t)slots * kGemmSplitSlotBytes : 0;
 }
-// The items of cut mode `cut` as (work, encoded item); slots counts the cut tiles.
+// The items of cut mode `cut` as (work, encoded item); slots counts the cut
+// tiles.  Work is k-blocks (plus the fix-up of a cut) times the tile's
+// token halves times the cost of a half at this tile height.
 static void gemm_items(const GemmParams &p, int count, int cut, std::vector<std::pair<int, uint32_t>> &items,
                        int64_t &slots) {
   int max_nk = 0;
@@ -643,12 +655,15 @@ static void gemm_items(const GemmParams &p, int count, int cut, std::vector<std:
     const int64_t n = (int64_t)m.tiles_m * m.tiles_n;
     for (int64_t t = 0; t < n; ++t) {
       const uint32_t tile = (uint32_t)(m.tile_begin + t);
+      const int64_t tm = t % m.tiles_m;  // m-tiles fastest, as the kernel decodes them
+      const int unit = p.tile_m == kGemmBM ? kGemmCostHalf * (tm * kGemmBM + kGemmHalfM < m.M ? 2 : 1)
+                                           : kGemmCostWhole;
       if (split) {
-        items.emplace_back(nk / 2 + kGemmSplitCost, tile | (1u << 16) | ((uint32_t)slots << 18));
-        items.emplace_back(nk - nk / 2 + kGemmSplitCost, tile | (2u << 16) | ((uint32_t)slots << 18));
+        items.emplace_back((nk / 2 + kGemmSplitCost) * unit, tile | (1u << 16) | ((uint32_t)slots << 18));
+        items.emplace_back((nk - nk / 2 + kGemmSplitCost) * unit, tile | (2u << 16) | ((uint32_t)slots << 18));
         ++slots;
       } else {
-        items.emplace_back(nk, tile);
+        items.emplace_back(nk * unit, tile);
       }
     }
   }
@@ -685,7 +700,7 @@ static int64_t gemm_lpt(std::vector<std::pair<int, uint32_t>> items, int64_t gri
 }
 // The plan of a launch over p's matrices (tiles set); `max_split_bytes`
 // bounds the workspace a cut may use (0: no cuts).  With `out`, the chosen
-// lists are written there.
+// lists are written there.  max_load is 0 for round robin (not estimated).
 static GemmPlan gemm_plan(const GemmParams &p, int count, int sms, size_t max_split_bytes, GemmParams *out) {
   GemmPlan best;
   const int64_t tiles = p.total_tiles;
@@ -721,10 +736,22 @@ static GemmPlan gemm_plan(const GemmParams &p, int count, int sms, size_t max_sp
   return best;
 }
 
-// Shapes and formats of a GEMM call (host only); fills the per-matrix tile
-// counts of `p`.
-static int gemm_check(int32_t count, const q4_state *const *Wq, int64_t M, GemmParams &p) {
+// Token tiles of height tile_m for every matrix of p (M, N set).
+static void gemm_tiles(GemmParams &p, int tile_m) {
   int64_t tiles = 0;
+  p.tile_m = tile_m;
+  for (int i = 0; i < p.count; ++i) {
+    GemmMat &m = p.mat[i];
+    m.tiles_m = (int32_t)ceil_div(m.M, tile_m);
+    m.tile_begin = tiles;
+    tiles += (int64_t)m.tiles_m * m.tiles_n;
+  }
+  p.total_tiles = tiles;
+}
+
+// Shapes and formats of a GEMM call (host only); fills the per-matrix tile
+// counts of `p` (tall tiles).
+static int gemm_check(int32_t count, const q4_state *const *Wq, int64_t M, GemmParams &p) {
   for (int i = 0; i < count; ++i) {
     const q4_state *s = Wq[i];
     if (!s) return Q4_ERR_ARG;
@@ -741,14 +768,89 @@ static int gemm_check(int32_t count, const q4_state *const *Wq, int64_t M, GemmP
     m.M = (int32_t)M;
     m.N = (int32_t)s->rows;
     m.K = (int32_t)s->cols;
-    m.tiles_m = (int32_t)ceil_div(M, kGemmBM);
     m.tiles_n = (int32_t)ceil_div(s->rows, kGemmBN);
-    m.tile_begin = tiles;
-    tiles += (int64_t)m.tiles_m * m.tiles_n;
   }
   p.count = count;
-  p.total_tiles = tiles;
+  gemm_tiles(p, kGemmBM);
   return Q4_OK;
+}
+
+// The tile height of a launch (kGemmBM or kGemmHalfM) and its plan; p's
+// tiles are set for that height and, with `lists`, its item lists written.
+static GemmPlan gemm_choose_uncached(GemmParams &p, int count, int sms, size_t max_split_bytes, bool lists) {
+  int tile_m = kGemmBM;
+  if (p.mat[0].M <= kGemmHalfM) {
+    tile_m = kGemmHalfM;  // one half per tile either way: two accumulators overlap the epilogue
+  } else {
+    gemm_tiles(p, kGemmBM);
+    const GemmPlan tall = gemm_plan(p, count, sms, max_split_bytes, nullptr);
+    if (tall.max_load > 0) {  // listed: compare with the half-height tiles
+      gemm_tiles(p, kGemmHalfM);
+      const GemmPlan low = gemm_plan(p, count, sms, max_split_bytes, nullptr);
+      if (low.max_load > 0 && low.max_load < tall.max_load) tile_m = kGemmHalfM;
+    }
+  }
+  gemm_tiles(p, tile_m);
+  return gemm_plan(p, count, sms, max_split_bytes, lists ? &p : nullptr);
+}
+
+// Planning a listed launch takes up to nine list-scheduling passes (two
+// tile heights, three cut modes, the final lists): hundreds of
+// microseconds of host time for a decoder layer.  A plan depends only on
+// the shapes, M, the SM count and the workspace bound, so the last few
+// plans of each host thread are kept and reused.
+struct GemmPlanKey {
+  int32_t count, sms;
+  int64_t M;
+  size_t max_split_bytes;
+  int32_t N[16], K[16];
+  bool operator==(const GemmPlanKey &o) const {
+    if (count != o.count || sms != o.sms || M != o.M || max_split_bytes != o.max_split_bytes) return false;
+    for (int i = 0; i < count; ++i)
+      if (N[i] != o.N[i] || K[i] != o.K[i]) return false;
+    return true;
+  }
+};
+struct GemmPlanEntry {
+  bool used = false;
+  GemmPlanKey key;
+  GemmPlan plan;
+  int32_t tile_m = 0;
+  uint16_t cta_off[kGemmListCtas + 1];
+  uint32_t tile_list[kGemmListTiles];
+};
+constexpr int kGemmPlanCache = 8;
+static GemmPlan gemm_choose(GemmParams &p, int count, int sms, size_t max_split_bytes, bool lists) {
+  static thread_local GemmPlanEntry cache[kGemmPlanCache];
+  static thread_local int next = 0;
+  GemmPlanKey key;
+  memset(&key, 0, sizeof(key));
+  key.count = count;
+  key.sms = sms;
+  key.M = p.mat[0].M;
+  key.max_split_bytes = max_split_bytes;
+  for (int i = 0; i < count; ++i) key.N[i] = p.mat[i].N, key.K[i] = p.mat[i].K;
+  for (GemmPlanEntry &e : cache) {
+    if (!e.used || !(e.key == key)) continue;
+    gemm_tiles(p, e.tile_m);
+    if (lists && e.plan.listed) {
+      memcpy(p.cta_off, e.cta_off, sizeof(uint16_t) * (size_t)(e.plan.grid + 1));
+      memcpy(p.tile_list, e.tile_list, sizeof(uint32_t) * e.cta_off[e.plan.grid]);
+    }
+    return e.plan;
+  }
+  const GemmPlan plan = gemm_choose_uncached(p, count, sms, max_split_bytes, true);
+  GemmPlanEntry &e = cache[next];
+  next = (next + 1) % kGemmPlanCache;
+  e.used = true;
+  e.key = key;
+  e.plan = plan;
+  e.tile_m = p.tile_m;
+  if (plan.listed) {
+    memcpy(e.cta_off, p.cta_off, sizeof(uint16_t) * (size_t)(plan.grid + 1));
+    memcpy(e.tile_list, p.tile_list, sizeof(uint32_t) * p.cta_off[plan.grid]);
+  }
+  return plan;
 }
 
 int q4_gemm_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes) {
@@ -760,7 +862,7 @@ int q4_gemm_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
   if (rc != Q4_OK) return rc;
   const DeviceInfo di = device_info();
   if (di.ok != Q4_OK) return di.ok;
-  const GemmPlan plan = gemm_plan(p, count, di.sms, (size_t)-1, nullptr);
+  const GemmPlan plan = gemm_choose(p, count, di.sms, (size_t)-1, false);
   *bytes = gemm_split_bytes(plan.slots);
   return Q4_OK;
 }
@@ -789,7 +891,7 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     const q4_state *s = Wq[i];
     GemmMat &m = p.mat[i];
     const CUtensorMapDataType adt = a_dtype == Q4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    if (!make_map(&m.tmA, adt, A[i], M, s->cols, 2, kGemmBK, kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_map(&m.tmA, adt, A[i], M, s->cols, 2, kGemmBK, kGemmHalfM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&m.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, s->packed, s->rows, s->cols / 2, 1, kGemmBK / 2,
                   kGemmBN, CU_TENSOR_MAP_SWIZZLE_NONE)) {
       rc = Q4_ERR_CUDA;
@@ -818,7 +920,7 @@ int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *
     }
     p.log2_bs = __builtin_ctz((unsigned)Wq[0]->blocksize);
     p.scale_f16 = Wq[0]->scale_f16;
-    const GemmPlan plan = gemm_plan(p, count, di.sms, workspace ? workspace_bytes : 0, &p);
+    const GemmPlan plan = gemm_choose(p, count, di.sms, workspace ? workspace_bytes : 0, true);
     p.listed = plan.listed;
     p.grid = (int32_t)plan.grid;
     if (plan.slots) {

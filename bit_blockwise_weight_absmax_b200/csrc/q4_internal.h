@@ -63,8 +63,9 @@ int run_double_quant(const float *absmax, int64_t nb, const float *mean, int8_t 
 int run_quantize_grouped(int dt, int qt, int bs, bool dq, const QuantGroupParams &p, int grid, cudaStream_t st);
 int run_double_quant_grouped(const DqGroupParams &p, cudaStream_t st);
 int run_dequantize(int qt, int dout, int bs, bool dq, const DequantGroupParams &p, int sms, cudaStream_t st);
+// the instance set follows split and p.tile_m (tall or half-height tiles)
 int run_gemm(int da, int mode, bool split, const GemmParams &p, cudaStream_t st);
-template <bool SPLIT>
+template <bool SPLIT, bool TALL>
 int run_gemm_t(int da, int mode, const GemmParams &p, cudaStream_t st);
 int run_gemv_small(int da, int bs, int M, bool asym, const GsParams &p, int sms, cudaStream_t st);
 template <bool AZ>

@@ -76,6 +76,55 @@ def test_gemm_split_k_few_tiles(q4, oracle):
     assert_matmul_close(y1[:, torch.from_numpy(rows).cuda()], ref)
 
 
+def _sampled_case(q4, oracle, M, N, K, seed, rows):
+    g = torch.Generator().manual_seed(seed)
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).bfloat16()
+    st = q4.quantize(W.cuda(), 64, "nf4", True)
+    ost = oracle_state(oracle, W, 64, 0, True)
+    w16 = oracle.dequantize(ost, True).reshape(N, K)[rows]
+    ref = oracle.matmul(bits(A), True, w16, True, M, len(rows), K)
+    return A.cuda(), st, ref
+
+
+def test_gemm_tall_tiles_ragged_half(q4, oracle):
+    """512-token tiles whose last tile's second half lies wholly past M:
+    M = 700, N = 10240, K = 512.  The planner takes the tall tiles here (160
+    tall tiles, the busiest CTA at 272 weighted units, against 320 for 240
+    half-height tiles), so tokens 512 .. 699 run as a lone first half and
+    the second half is neither loaded nor multiplied."""
+    M, N, K = 700, 10240, 512
+    rows = np.concatenate([np.arange(0, N, 37), np.arange(N - 40, N)])
+    a, st, ref = _sampled_case(q4, oracle, M, N, K, 21, rows)
+    y = q4.gemm(a, st)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+
+
+def test_gemm_tall_tiles_split_k(q4, oracle):
+    """512-token tiles cut into k halves: M = 1000, N = 2560, K = 16384.  40
+    tall tiles of 256 k-blocks leave most SMs idle; cut, their 80 halves
+    (busiest CTA 4896 weighted units) beat both the uncut tall tiles (8704)
+    and the 80 half-height tiles (5120; cut, 160 halves overflow the SMs).
+    Against the oracle, bit-identical on repeat, counters left zeroed."""
+    import ctypes
+    M, N, K = 1000, 2560, 16384
+    rows = np.concatenate([np.arange(0, N, 29), np.arange(N - 16, N)])
+    a, st, ref = _sampled_case(q4, oracle, M, N, K, 22, rows)
+    arr = (ctypes.POINTER(q4._CState) * 1)(ctypes.pointer(st.c_struct()))
+    wsz = ctypes.c_size_t(0)
+    assert q4.library().q4_gemm_workspace_size(1, arr, M, ctypes.byref(wsz)) == 0
+    assert wsz.value > 0  # the plan cuts tiles
+    ys = [q4.gemm(a, st) for _ in range(2)]
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    assert torch.equal(ys[0], ys[1])
+    assert_matmul_close(ys[0][:, torch.from_numpy(rows).cuda()], ref)
+    ws = q4._workspace(a.device, "gemm", wsz.value)
+    assert int(ws[:65536].count_nonzero()) == 0
+
+
 def test_gemm_exact_small_integers(q4, oracle):
     """A in {-1, 0, 1}, every block's maximum 1 (so w^ is the bf16 level),
     K = 64, fp32 output: each partial sum of the tensor cores is exactly
