@@ -10,26 +10,32 @@
 // into shared memory and consumed there by the tensor cores, so the 16-bit
 // weight matrix never exists in HBM.
 //
-// Design (one CTA per SM, persistent over output tiles of 256 x 128, m-tiles
-// fastest so that neighbouring CTAs share a weight tile in L2):
-//   warp 0      TMA producer: the A tile [256 x 64] (128B-swizzled, K-major)
-//               and the raw packed tile [128 rows x 32 bytes] per k-block,
-//               into a ring of 4 stages.
-//   warp 1      TMEM allocator and MMA issuer: per k-block 4
-//               tcgen05.mma kind::f16 (M=128 weight rows, N=256 tokens,
-//               K=16) into one fp32 accumulator of 256 columns (a TMEM lane
-//               per weight row, a column per token); two accumulators
-//               alternate between tiles (512 TMEM columns), so the epilogue
-//               of one tile overlaps the MMAs of the next.  With the weight
+// Design (one CTA per SM, persistent over output tiles of 128 weight rows
+// by 512 tokens -- or 256 tokens for launches of few tiles, a template
+// parameter the host picks -- m-tiles fastest so that neighbouring CTAs
+// share a weight tile in L2):
+//   warp 0      TMA producer: the raw packed tile [128 rows x 32 bytes] of
+//               each 64-k block into a ring of 4 dequant stages, and the
+//               activation tile in 256-token halves [256 x 64] (128B-
+//               swizzled, K-major) into a ring of 4 slots; the raw codes
+//               run two k-blocks ahead of the activations (tall tiles).
+//   warp 1      TMEM allocator and MMA issuer: per k-block and token half
+//               4 tcgen05.mma kind::f16 (M=128 weight rows, N=256 tokens,
+//               K=16), both halves reading the same dequantized weight
+//               stage, into a 512-column fp32 accumulator (a TMEM lane per
+//               weight row, a column per token).  256-token tiles use two
+//               256-column accumulators that alternate between tiles, so an
+//               epilogue overlaps the next tile's MMAs.  With the weight
 //               tile on the M side each MMA reads 12 KB of shared memory
-//               for 128 tensor cycles (two N=128 MMAs over the token halves
-//               read 16 KB), and shared-memory bandwidth is what the MMAs,
-//               the copies and the dequant stores share.
+//               for 128 tensor cycles (two N=128 MMAs over token halves
+//               would read 16 KB), and shared-memory bandwidth is what the
+//               MMAs, the copies and the dequant stores share; a tall tile
+//               also halves the dequant work per flop.
 //   warps 2..17 dequant: four threads per weight row, 16 codes each, scaled
 //               by the row's block scale into bf16/fp16 and written in the
 //               128B-swizzled K-major layout the UMMA descriptor reads; the
 //               block scales come 16 blocks per load.  Then the epilogue:
-//               tcgen05.ld of the accumulators (a lane per weight row, 16
+//               tcgen05.ld of the accumulator (a lane per weight row, 16
 //               tokens at a time), convert, store one token row's 32
 //               consecutive outputs per warp instruction.
 // Every mbarrier wait is bounded in time; a timeout sets Q4_STATUS_TIMEOUT,
