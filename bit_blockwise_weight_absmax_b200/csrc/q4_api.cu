@@ -867,6 +867,22 @@ int q4_gemm_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, 
   return Q4_OK;
 }
 
+int q4_gemm_plan_info(int32_t count, const q4_state *const *Wq, int64_t M, int32_t sms, size_t workspace_bytes,
+                      int32_t *tile_m, int32_t *grid, int64_t *cut_tiles) {
+  if (!tile_m || !grid || !cut_tiles || !Wq || count < 1 || count > kGsMaxGroup) return Q4_ERR_ARG;
+  if (sms < 1 || sms > 1024) return Q4_ERR_ARG;
+  if (M < 1 || M > INT32_MAX) return Q4_ERR_SHAPE;
+  static thread_local GemmParams p;
+  memset(&p, 0, sizeof(p));
+  const int rc = gemm_check(count, Wq, M, p);
+  if (rc != Q4_OK) return rc;
+  const GemmPlan plan = gemm_choose(p, count, sms, workspace_bytes, false);
+  *tile_m = p.tile_m;
+  *grid = (int32_t)plan.grid;
+  *cut_tiles = plan.slots;
+  return Q4_OK;
+}
+
 int q4_gemm_grouped(int32_t count, const void *const *A, const q4_state *const *Wq,
                     void *const *Y, int64_t M, int32_t a_dtype, int32_t y_dtype, void *workspace,
                     size_t workspace_bytes, void *stream) {

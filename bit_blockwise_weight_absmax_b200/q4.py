@@ -74,6 +74,8 @@ def library():
             "q4_gemv_grouped": ([i32, ctypes.POINTER(P), ctypes.POINTER(SP), ctypes.POINTER(P), i64,
                                  i32, i32, P, sz, P], i32),
             "q4_gemm_workspace_size": ([i32, ctypes.POINTER(SP), i64, ctypes.POINTER(ctypes.c_size_t)], i32),
+            "q4_gemm_plan_info": ([i32, ctypes.POINTER(SP), i64, i32, ctypes.c_size_t, ctypes.POINTER(i32),
+                                   ctypes.POINTER(i32), ctypes.POINTER(i64)], i32),
             "q4_gemm": ([P, i32, i64, SP, P, i32, P, ctypes.c_size_t, P], i32),
             "q4_gemm_grouped": ([i32, ctypes.POINTER(P), ctypes.POINTER(SP), ctypes.POINTER(P), i64,
                                  i32, i32, P, ctypes.c_size_t, P], i32),

@@ -285,6 +285,20 @@ Q4_API int q4_gemv_grouped(int32_t count, const void *const *A, const q4_state *
  * counters zeroed (after Q4_STATUS_TIMEOUT, zero-fill it again). */
 Q4_API int q4_gemm_workspace_size(int32_t count, const q4_state *const *Wq, int64_t M, size_t *bytes);
 
+/* How a q4_gemm_grouped launch over these matrices would run on a device of
+ * `sms` streaming multiprocessors with `workspace_bytes` of workspace
+ * (SIZE_MAX: as much as q4_gemm_workspace_size asks for): the tokens per
+ * output tile (*tile_m: 512, or 256 for launches of few tiles and for M <=
+ * 256), the CTAs of the grid (*grid) and the tiles cut in halves of their k
+ * range (*cut_tiles).  Host only: it reads the states' shapes and formats,
+ * touches no device and allocates nothing; the same shape and format
+ * checks as q4_gemm_workspace_size (Q4_ERR_ARG / Q4_ERR_SHAPE), and sms
+ * outside 1 .. 1024 is Q4_ERR_ARG.  The planning it reports: the host deals
+ * work items longest first onto the least-loaded CTA, for both tile
+ * heights, and keeps the height whose busiest CTA finishes first. */
+Q4_API int q4_gemm_plan_info(int32_t count, const q4_state *const *Wq, int64_t M, int32_t sms,
+                             size_t workspace_bytes, int32_t *tile_m, int32_t *grid, int64_t *cut_tiles);
+
 /*
  * q4_gemm -- the same product for any M >= 1, computed by dequantizing
  * weight tiles into shared memory (bit-exact w^ in a_dtype) and feeding

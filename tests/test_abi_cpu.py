@@ -263,6 +263,47 @@ def test_gemm_workspace_size_host_checks(lib):
     assert lib.q4_gemm_workspace_size(1, arr, 512, None) == -1
 
 
+def _plan(lib, shapes, M, sms=148, ws=2 ** 64 - 1):
+    """q4_gemm_plan_info over fake NF4 (B=64, double-quantized) states of
+    the given (N, K) shapes: (return code, tile_m, grid, cut tiles)."""
+    from bit_blockwise_weight_absmax_b200 import q4
+    P = ctypes.POINTER(q4._CState)
+    sts = [_fake_state(0, N, K, 64, True) for N, K in shapes]
+    arr = (P * len(sts))(*[ctypes.pointer(st) for st in sts])
+    tm, grid, cut = ctypes.c_int32(-7), ctypes.c_int32(-7), ctypes.c_int64(-7)
+    rc = lib.q4_gemm_plan_info(len(sts), arr, M, sms, ws, ctypes.byref(tm), ctypes.byref(grid), ctypes.byref(cut))
+    return rc, tm.value, grid.value, cut.value
+
+
+def test_gemm_plan_tile_height_and_cuts(lib):
+    """The GEMM's host planner (no device): 512-token tiles when there are
+    enough of them to fill the SMs, 256-token tiles for M <= 256 and for
+    launches of few tiles, k-cuts only with a workspace and only where they
+    take at least a tenth off the busiest CTA."""
+    from bit_blockwise_weight_absmax_b200 import workloads as wl
+    layer = [(N, K) for _, N, K in wl.LAYER_7B]
+    # the 7B layer at prefill sizes: 332 (1328) tall tiles, none cut
+    assert _plan(lib, layer, 512) == (0, 512, 148, 0)
+    assert _plan(lib, layer, 2048) == (0, 512, 148, 0)
+    # M <= 256: one token half per tile either way, so two accumulators
+    assert _plan(lib, layer, 64)[:2] == (0, 256)
+    assert _plan(lib, layer, 256)[:2] == (0, 256)
+    # one 4096 x 4096 matrix at M = 512: 32 tall tiles would leave 116 SMs
+    # idle; 64 half-height tiles cut in k give 128 items
+    assert _plan(lib, [(4096, 4096)], 512) == (0, 256, 128, 64)
+    assert _plan(lib, [(4096, 4096)], 512, ws=0) == (0, 256, 64, 0)  # no workspace, no cuts
+    # the GPU tests' shapes for the tall tiles' lone first half and cut tall tiles
+    assert _plan(lib, [(10240, 512)], 700) == (0, 512, 148, 0)
+    assert _plan(lib, [(2560, 16384)], 1000) == (0, 512, 80, 40)
+    # fewer SMs: the same layer still takes tall tiles, and the grid follows
+    assert _plan(lib, layer, 512, sms=74) == (0, 512, 74, 0)
+    # argument and shape checks, before any device is asked for
+    assert _plan(lib, layer, 512, sms=0)[0] == -1
+    assert _plan(lib, layer, 512, sms=1025)[0] == -1
+    assert _plan(lib, layer, 0)[0] == -2
+    assert _plan(lib, [(4096, 4000)], 512)[0] == -2  # K % 64
+
+
 def test_grouped_calls_reject_a_null_entry_before_any_use(lib):
     """A NULL state, activation or output pointer in any entry of a grouped
     call is Q4_ERR_ARG, found before the library reads any entry (a NULL
