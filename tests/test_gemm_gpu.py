@@ -102,6 +102,27 @@ def test_gemm_tall_tiles_ragged_half(q4, oracle):
     assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
 
 
+def test_gemm_tall_tiles_f16_fp32_out(q4, oracle):
+    """512-token tiles with fp16 activations and fp32 output (M = 600, N =
+    10240, K = 512: 160 tall tiles, the second of each column a lone first
+    half of 88 tokens); the fp32 output differs from the binary64 product
+    only by the fp32 accumulation order."""
+    M, N, K = 600, 10240, 512
+    g = torch.Generator().manual_seed(23)
+    W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
+    A = torch.randn(M, K, generator=g).half()
+    st = q4.quantize(W.cuda(), 64, "nf4", True)
+    ost = oracle_state(oracle, W, 64, 0, True)
+    rows = np.concatenate([np.arange(0, N, 41), np.arange(N - 24, N)])
+    w16 = oracle.dequantize(ost, False).reshape(N, K)[rows]
+    ref = oracle.matmul(bits(A), False, w16, False, M, len(rows), K)
+    y = q4.gemm(A.cuda(), st, torch.float32)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    fro, mx = assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+    assert fro < 1e-5
+
+
 def test_gemm_tall_tiles_split_k(q4, oracle):
     """512-token tiles cut into k halves: M = 1000, N = 2560, K = 16384.  40
     tall tiles of 256 k-blocks leave most SMs idle; cut, their 80 halves

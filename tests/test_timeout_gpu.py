@@ -75,16 +75,17 @@ def test_grouped_quantize_wait_limit_times_out_and_recovers(oracle, dq):
     assert q4.last_device_status() == 0
 
 
-def test_gemm_wait_limit_times_out_and_recovers(oracle):
+@pytest.mark.parametrize("M,N,K", [(512, 1024, 2048), (700, 10240, 512)])
+def test_gemm_wait_limit_times_out_and_recovers(oracle, M, N, K):
     """The GEMM's MMA and dequant warps wait for tiles that the stalled
     producer never copies: Q4_STATUS_TIMEOUT, the kernel returns (waiting
     for its issued MMAs before it frees the tensor memory), and a following
-    call is correct."""
+    call is correct.  The first shape runs 256-token tiles, the second
+    512-token tiles (two rings for the producer to drain)."""
     from bit_blockwise_weight_absmax_b200 import build
     build.build()
     from bit_blockwise_weight_absmax_b200 import q4
     g = torch.Generator().manual_seed(7)
-    M, N, K = 512, 1024, 2048
     W = torch.randn(N, K, generator=g).mul(0.02).bfloat16()
     A = torch.randn(M, K, generator=g).bfloat16()
     st = q4.quantize(W.cuda(), 64, "nf4", True)
