@@ -51,8 +51,8 @@ constexpr int kQgPieceBytes = kQgPiece * 2;          // 16 KB
 constexpr int kQgStages = 8;
 constexpr int kQgBufs = 16;                          // chunk buffers of block scales (reducer input)
 constexpr int kQgRing = kQgStages * kQgPieceBytes;
-constexpr uint32_t kQgSleepNs = 200;
-constexpr int64_t kQgMaxChunks = 65536;  // chunk sums one matrix's mean is formed from  // producer / reducer back-off between probes
+constexpr uint32_t kQgSleepNs = 200;      // producer / reducer back-off between probes
+constexpr int64_t kQgMaxChunks = 65536;  // chunk sums one matrix's mean is formed from
 static_assert(kQgBufs >= kQgStages, "the producer never waits on a chunk buffer whose chunk it has not reclaimed");
 constexpr int kQgSmem = kQgRing + 32 * 32 * 8 /*bin tables*/ + kQgBufs * kChunkBlocks * 4 +
                         (2 * kQgStages + 2 * kQgBufs) * 8 + 64;
