@@ -109,6 +109,7 @@ struct alignas(64) GemmMat {
 // writes Y.  Item encoding: bits 0-15 tile, 16-17 half (0 whole, 1 first,
 // 2 second), 18-31 split slot.
 constexpr int kGemmListTiles = 2048;
+constexpr int kGemmGroupM = 4;  // m-tiles per group of a round-robin launch
 constexpr int kGemmListCtas = 256;  // grid bound of a listed launch
 constexpr int kGemmSplitWarpFloats = kGemmBM / 4 * 32;  // one epilogue warp's partial: its columns x lanes
 constexpr size_t kGemmSplitSlotBytes = 2 * 16 * kGemmSplitWarpFloats * sizeof(float);  // two halves x 16 warps
@@ -299,8 +300,20 @@ __device__ __forceinline__ TileCoord gemm_tile(const GemmParams &p, int64_t v) {
   const int64_t local = t - p.mat[mi].tile_begin;
   const int tm_count = p.mat[mi].tiles_m;
   const int nk = p.mat[mi].K / kGemmBK;
-  // m-tiles fastest: consecutive CTAs share one weight tile (read once from HBM)
-  TileCoord tc{mi, (int)(local % tm_count), (int)(local / tm_count), 0, nk, -1, 0};
+  // m-tiles fastest: consecutive CTAs share one weight tile (read once from
+  // HBM).  Launches dealt round robin (too many tiles for a list: large M)
+  // go through the m-tiles kGemmGroupM at a time, so that the CTAs running
+  // at once share a few activation m-tiles in L2 instead of streaming all
+  // of them (at M = 8192 the down projection's activations are 180 MB).
+  int tm = (int)(local % tm_count), tn = (int)(local / tm_count);
+  if (!p.listed && tm_count > kGemmGroupM) {
+    const int64_t per_group = (int64_t)kGemmGroupM * p.mat[mi].tiles_n;
+    const int64_t g = local / per_group, r = local % per_group;
+    const int gm = min(kGemmGroupM, tm_count - (int)g * kGemmGroupM);
+    tm = (int)g * kGemmGroupM + (int)(r % gm);
+    tn = (int)(r / gm);
+  }
+  TileCoord tc{mi, tm, tn, 0, nk, -1, 0};
   if (hc != 0) {
     tc.half = hc - 1;
     tc.slot = (int)(v >> 18);

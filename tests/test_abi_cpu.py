@@ -296,6 +296,8 @@ def test_gemm_plan_tile_height_and_cuts(lib):
     assert _plan(lib, [(10240, 512)], 700) == (0, 512, 148, 0)
     assert _plan(lib, [(10240, 512)], 600)[:2] == (0, 512)
     assert _plan(lib, [(1024, 2048)], 512)[:2] == (0, 256)  # the timeout test's other shape
+    # more tiles than a list holds: whole tall tiles round robin
+    assert _plan(lib, [(27648, 256)], 5000) == (0, 512, 148, 0)
     assert _plan(lib, [(2560, 16384)], 1000) == (0, 512, 80, 40)
     # fewer SMs: the same layer still takes tall tiles, and the grid follows
     assert _plan(lib, layer, 512, sms=74) == (0, 512, 74, 0)

@@ -123,6 +123,22 @@ def test_gemm_tall_tiles_f16_fp32_out(q4, oracle):
     assert fro < 1e-5
 
 
+def test_gemm_round_robin_ragged_groups(q4, oracle):
+    """A launch of too many tiles for a list (M = 5000, N = 27648, K = 256:
+    10 x 216 tall tiles) is dealt round robin with the m-tiles taken four
+    at a time; 10 m-tiles leave a last group of two.  Sampled rows and
+    tokens, including the last of each, against the oracle."""
+    M, N, K = 5000, 27648, 256
+    rows = np.concatenate([np.arange(0, N, 211), np.arange(N - 8, N)])
+    a, st, ref = _sampled_case(q4, oracle, M, N, K, 24, rows)
+    y = q4.gemm(a, st)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    toks = np.concatenate([np.arange(0, M, 97), np.arange(M - 8, M)])
+    sel = y[torch.from_numpy(toks).cuda()][:, torch.from_numpy(rows).cuda()]
+    assert_matmul_close(sel, ref[toks])
+
+
 def test_gemm_tall_tiles_split_k(q4, oracle):
     """512-token tiles cut into k halves: M = 1000, N = 2560, K = 16384.  40
     tall tiles of 256 k-blocks leave most SMs idle; cut, their 80 halves
