@@ -473,6 +473,21 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
       prefetch_tensormap(&p.mat[lane].tmA);
     }
     if (lane == 0) {
+      // The weight boxes of the first ring's worth of stages into L2 before
+      // the wait, so that their DRAM latency overlaps the previous kernel's
+      // last CTAs (a prefetch consumes nothing: the copies below still come
+      // after the wait).
+      {
+        int pmi = 0, n = 0;
+        GsUnit v;
+        if (g0 < g1) v = gs_describe<B>(info, p.count, pmi, g0, g0, g1);
+        for (uint32_t gi = g0; gi < g1 && n < S;) {
+          if (gi != g0) v = gs_next<B>(info, p.count, v, gi, g0, g1);
+          for (int q = v.q0; q < v.q1 && n < S; ++q, ++n)
+            tma_prefetch_l2_2d(&p.mat[v.mi].tmW, q * (kGsStageK / 2), v.tile * kGsRows);
+          gi += (uint32_t)(v.q1 - v.q0);
+        }
+      }
       pdl_wait();
       const uint32_t tx = (uint32_t)kGsWTile + 2u * 128u * (uint32_t)M;
       int s = 0, mi = 0, issued = 0;
