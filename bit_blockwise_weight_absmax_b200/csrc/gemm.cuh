@@ -217,15 +217,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
-// Prefetch of one box of a tensor into L2 (no shared memory, no barrier).
-// L2 is where the GPU's memory is coherent, so a box prefetched while an
-// earlier kernel may still write it is read correctly by the copy that
-// follows the dependency wait.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
-               : "memory");
-}
-
 // Fetches a tensor map (a kernel parameter) into the descriptor cache ahead
 // of its first copy.
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *m) {

@@ -213,6 +213,15 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
 }
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Prefetch of one box of a tensor into L2 (no shared memory, no barrier).
+// L2 is where the GPU's memory is coherent, so a box prefetched while an
+// earlier kernel may still write it is read correctly by the copy that
+// follows the dependency wait.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
+
 // Address of the table entry of byte j of `word`: byte 1 of the address is
 // the packed byte; bytes 0, 2, 3 come from `lb` (table base + lane offset,
 // whose byte 1 is zero because the table is 64 KB aligned).
