@@ -49,7 +49,7 @@ NCU_TRAFFIC = {
     "gemm": ("bit_blockwise_weight_absmax_b200/csrc/gemm.cuh",
              "131690000b067cfa5b54292cd0fcbaaca0955854007702fa36d49b37172ba8dd", 142_834_176 + 19_374_592),
     "gemv": ("bit_blockwise_weight_absmax_b200/csrc/gemv_small.cuh",
-             "28253323ac707e25de95c3d126c95494539dda6da3298d757bae61973122a062", 109_082_624 + 5_255_680),
+             "6721fbd3bd7b25d31d2883e150619d5e9d6219e3ae024ce700d78fcb40b82906", 108_711_936 + 6_480_640),
 }
 
 
