@@ -295,6 +295,7 @@ def test_gemm_plan_tile_height_and_cuts(lib):
     # the GPU tests' shapes for the tall tiles' lone first half and cut tall tiles
     assert _plan(lib, [(10240, 512)], 700) == (0, 512, 148, 0)
     assert _plan(lib, [(10240, 512)], 600)[:2] == (0, 512)
+    assert _plan(lib, [(9440, 512)], 700) == (0, 512, 148, 0)  # a ragged last weight tile
     assert _plan(lib, [(1024, 2048)], 512)[:2] == (0, 256)  # the timeout test's other shape
     # more tiles than a list holds: whole tall tiles round robin
     assert _plan(lib, [(27648, 256)], 5000) == (0, 512, 148, 0)

@@ -102,6 +102,19 @@ def test_gemm_tall_tiles_ragged_half(q4, oracle):
     assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
 
 
+def test_gemm_tall_tiles_ragged_rows(q4, oracle):
+    """512-token tiles over a weight matrix whose last tile is ragged (M =
+    700, N = 9440 = 73 x 128 + 96, K = 512: 148 tall tiles, the planner's
+    pick); the rows past N are neither stored nor let into the result."""
+    M, N, K = 700, 9440, 512
+    rows = np.concatenate([np.arange(0, N, 53), np.arange(N - 112, N)])
+    a, st, ref = _sampled_case(q4, oracle, M, N, K, 25, rows)
+    y = q4.gemm(a, st)
+    torch.cuda.synchronize()
+    assert q4.last_device_status() == 0
+    assert_matmul_close(y[:, torch.from_numpy(rows).cuda()], ref)
+
+
 def test_gemm_tall_tiles_f16_fp32_out(q4, oracle):
     """512-token tiles with fp16 activations and fp32 output (M = 600, N =
     10240, K = 512: 160 tall tiles, the second of each column a lone first
