@@ -63,14 +63,25 @@ def _ncu_traffic(kernel):
 
 
 def _peaks():
+    """The roofline denominators: the measured copy bandwidth and bf16 GEMM
+    rates of MEASURED_PEAKS.json when it is present and readable, else the
+    recipe's fallback figures (the source says which, and why)."""
+    fallback = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        d = json.load(open(p))
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
-                "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-            "source": "fallback"}
+    if not os.path.exists(p):
+        return fallback
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        out = {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+               "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+               "source": "measured"}
+    except (OSError, ValueError, KeyError, TypeError) as e:
+        return dict(fallback, source=f"fallback (MEASURED_PEAKS.json unreadable: {type(e).__name__})")
+    if min(out["hbm_gbs"], out["bf16_tflops"], out["bf16_tflops_sustained"]) <= 0:
+        return dict(fallback, source="fallback (MEASURED_PEAKS.json holds a non-positive peak)")
+    return out
 
 
 def layer_state_bytes(shapes, blocksize=64):

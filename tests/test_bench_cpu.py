@@ -86,3 +86,24 @@ def test_reference_arm_json_line(capsys):
                            "d2h_bytes_per_step": 0}
     # ms_per_step is the step's measured wall time, not the whole-layer estimate
     assert 0 < line["ms_per_step"] < line["layer_gemv_ms_estimate"]
+
+
+def test_peaks_measured_fallback_and_unreadable(tmp_path, monkeypatch):
+    """The roofline denominators: MEASURED_PEAKS.json when present and
+    readable, else the recipe's fallback, with the reason in `source`."""
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._peaks() == {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                              "source": "fallback"}
+    f = tmp_path / "MEASURED_PEAKS.json"
+    f.write_text('{"hbm_gbs": 6542.1, "bf16_tflops": 1641.8, "bf16_tflops_sustained": 1367.1}')
+    p = bench._peaks()
+    assert p["source"] == "measured" and (p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"]) == (
+        6542.1, 1641.8, 1367.1)
+    f.write_text('{"hbm_gbs": 6542.1, "bf16_tflops": 1641.8}')  # no sustained figure: the burst one
+    assert bench._peaks()["bf16_tflops_sustained"] == 1641.8
+    for bad in ('{"hbm_gbs": 6542.1}', "not json", '{"hbm_gbs": "x", "bf16_tflops": 1}',
+                '{"hbm_gbs": 0, "bf16_tflops": 1641.8}'):
+        f.write_text(bad)
+        p = bench._peaks()
+        assert p["source"].startswith("fallback (") and p["hbm_gbs"] == 6650.0, bad
