@@ -318,6 +318,11 @@ Q4_API int q4_gemm_plan_info(int32_t count, const q4_state *const *Wq, int64_t M
  *       which half finishes first.
  * Same tolerance as q4_gemv.  A grouped call takes one format (qtype,
  * blocksize, double_quant) for all its matrices (Q4_ERR_ARG otherwise).
+ * Host cost: each launch is planned on the host (tile height, per-CTA
+ * tile lists, cuts; q4_gemm_plan_info reports the outcome).  Planning a
+ * decoder layer takes up to about a millisecond of host time; each host
+ * thread keeps its last 8 plans (keyed by shapes, M, SM count and
+ * workspace bytes), so repeated shapes plan once.
  */
 Q4_API int q4_gemm(const void *A, int32_t a_dtype, int64_t M, const q4_state *Wq, void *Y,
             int32_t y_dtype, void *workspace, size_t workspace_bytes, void *stream);
