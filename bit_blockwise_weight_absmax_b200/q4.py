@@ -393,8 +393,26 @@ def dequantize_grouped(states, dtype: torch.dtype | None = None, outs=None, stre
 _gemv_ws_need = {}  # (shapes and formats of the group, M) -> workspace bytes
 
 
-def _gemv_workspace(states, structs, M, device):
+_struct_arrays = {}
+
+
+def _struct_array(structs):
+    """The C array of pointers to these state structs, built once per tuple
+    of structs (c_struct() returns the same object while a state is
+    unchanged; the cache holds the structs, so their ids stay theirs)."""
+    key = tuple(id(s) for s in structs)
+    hit = _struct_arrays.get(key)
+    if hit is not None:
+        return hit[1]
     arr = (ctypes.POINTER(_CState) * len(structs))(*[ctypes.pointer(s) for s in structs])
+    if len(_struct_arrays) >= 256:
+        _struct_arrays.clear()
+    _struct_arrays[key] = (tuple(structs), arr)
+    return arr
+
+
+def _gemv_workspace(states, structs, M, device):
+    arr = _struct_array(structs)
     key = (tuple((s.rows, s.cols, s.blocksize, s.qtype, s.double_quant) for s in states), M)
     need = _gemv_ws_need.get(key)
     if need is None:
@@ -438,7 +456,7 @@ def gemm_grouped(As, states, out_dtype: torch.dtype | None = None, outs=None, st
     a_dtype = As[0].dtype
     out_dtype = out_dtype or a_dtype
     structs = [s.c_struct() for s in states]
-    arr = (ctypes.POINTER(_CState) * len(structs))(*[ctypes.pointer(s) for s in structs])
+    arr = _struct_array(structs)
     if outs is None:
         outs = [torch.empty(M, s.rows, dtype=out_dtype, device=As[0].device) for s in states]
     for a, s in zip(As, states):
