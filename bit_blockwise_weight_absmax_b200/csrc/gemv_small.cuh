@@ -562,9 +562,11 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
 
   const uint32_t lb = lut + ES * (uint32_t)lane;
   uint32_t sb = 0;  // c~ buffer parity
-  // partial tiles of this CTA awaiting their count: [0] the one holding the
-  // CTA's first stage, [1] the one holding its last
-  int pend_mi0 = -1, pend_tile0 = 0, pend_len0 = 0;
+  // partial tiles: the one holding this CTA's first stage is counted when
+  // done (done0: its row groups this warp completed, summed at the end); the
+  // one holding its last stage is counted at the end
+  int pend_mi0 = -1, pend_tile0 = 0;
+  uint32_t done0 = 0u;
   int pend_mi1 = -1, pend_tile1 = 0, pend_len1 = 0;
   float acc[R][NT][4];
   int qstart = 0;
@@ -594,6 +596,93 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
     zst[rt] = zbase + (uint32_t)(warp * R + rt) * 512u + (uint32_t)((blk0 * 8 + (r & 7)) * 2 + (r >> 3));
     zrd0[rt] = zbase + (uint32_t)(warp * R + rt) * 512u + (uint32_t)g * 2u;
   }
+
+  // A partial tile's rows (this warp's 16-row groups) are counted, and the
+  // warp that completes a group's count sums the slots of all contributors
+  // in CTA order, writes Y and leaves slots and count zeroed.  A CTA counts
+  // its first partial tile as soon as it is done (its partner, the CTA
+  // before, finishes that tile only at its own end) and its last one at its
+  // end; the sums run at the end, so the end of a launch counts one tile per
+  // CTA.  count_piece returns the row groups this warp completed.
+  auto count_piece = [&](int pmi, int tile, unsigned len) -> uint32_t {
+    fence_acq_rel_gpu();  // this thread's slot stores are visible before its count
+    __syncwarp();
+    const GsInfo &mt = info[pmi];
+    // lane 0 counts every row group of the warp at once (the atomics are in
+    // flight together), then each one is checked for completion
+    unsigned olds[R];
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) {
+      olds[rt] = 0u;
+      const int r_base = tile * kGsRows + warp * 16 * R + rt * 16;
+      if (lane == 0 && r_base < mt.N) olds[rt] = atomicAdd(mt.cnt + (r_base >> 4), len);
+    }
+    uint32_t done = 0u;
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) {
+      const int r_base = tile * kGsRows + warp * 16 * R + rt * 16;
+      const unsigned old = __shfl_sync(0xffffffffu, olds[rt], 0);
+      if (r_base < mt.N && old + len == (unsigned)mt.n_stages) done |= 1u << rt;
+    }
+    return done;
+  };
+  auto sum_piece = [&](int pmi, int tile, uint32_t done) {
+    const GsInfo &mt = info[pmi];
+    const int N = mt.N, Q = mt.n_stages;
+    const uint32_t x0 = mt.stage_begin + (uint32_t)(tile * Q);  // the tile's first stage
+#pragma unroll
+    for (int rt = 0; rt < R; ++rt) {
+      if (!(done & (1u << rt))) continue;
+      const int r_base = tile * kGsRows + warp * 16 * R + rt * 16;
+      // every contributor has counted: sum their slots in CTA order
+      __syncwarp();
+      fence_acq_rel_gpu();
+      const int c0 = gs_cta_of(x0, T, G), c1 = gs_cta_of(x0 + Q - 1, T, G);
+      float sum[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sum[nt][j] = 0.0f;
+      for (int cb = c0; cb <= c1; cb += 4) {
+        // up to four contributors' rows in flight at once, added in CTA order
+        float2 v[4][NT][2];
+        float *slot[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c = min(cb + k, c1);
+          const int role = (gs_range_begin(c, T, G) >= x0) ? 0 : 1;  // c starts inside the tile
+          slot[k] = p.slots + ((int64_t)(c * 2 + role) * kGsRows + warp * 16 * R + rt * 16 + g) * MW + 2 * tig;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              v[k][nt][h] = __ldcg(reinterpret_cast<const float2 *>(slot[k] + (h * 8) * MW + nt * 8));
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (cb + k > c1) break;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // the workspace is left zeroed
+              __stcg(reinterpret_cast<float2 *>(slot[k] + (h * 8) * MW + nt * 8), make_float2(0.0f, 0.0f));
+              sum[nt][2 * h] += v[k][nt][h].x;
+              sum[nt][2 * h + 1] += v[k][nt][h].y;
+            }
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = r_base + (j >> 1) * 8 + g;
+          const int m = nt * 8 + 2 * tig + (j & 1);
+          if (m < M && row < N) gs_store(mt.Y, p.y_dtype, (int64_t)m * N + row, sum[nt][j]);
+        }
+      if (lane == 0) mt.cnt[r_base >> 4] = 0u;
+    }
+  };
 
   bool ok = true;
 #pragma unroll 1
@@ -826,7 +915,9 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
               __stcg(reinterpret_cast<float2 *>(slot + (rt * 16 + h * 8) * MW + nt * 8),
                      make_float2(acc[rt][nt][2 * h], acc[rt][nt][2 * h + 1]));
         if (role0) {
-          pend_mi0 = cu.mi; pend_tile0 = cu.tile; pend_len0 = cu.q1 - qstart;
+          pend_mi0 = cu.mi;
+          pend_tile0 = cu.tile;
+          done0 = count_piece(cu.mi, cu.tile, (unsigned)(cu.q1 - qstart));
         } else {
           pend_mi1 = cu.mi; pend_tile1 = cu.tile; pend_len1 = cu.q1 - qstart;
         }
@@ -834,89 +925,9 @@ __global__ void __launch_bounds__(GsShape<R>::kThreads, 1) gemv_small_kernel(con
     }
     gi = gn;
   }
-  if (!ok || (pend_mi0 < 0 && pend_mi1 < 0)) return;
-
-  // ---- count this CTA's partial tiles; finish every 16-row group it completes
-  fence_acq_rel_gpu();  // this thread's slot stores are visible before its count
-  __syncwarp();
-  // lane 0 counts every partial row group of the warp at once (the atomics
-  // are in flight together), then each one is checked for completion
-  unsigned olds[2][R];
-#pragma unroll
-  for (int rl = 0; rl < 2; ++rl)
-#pragma unroll
-    for (int rt = 0; rt < R; ++rt) {
-      olds[rl][rt] = 0u;
-      const int pmi = rl ? pend_mi1 : pend_mi0;
-      if (pmi < 0 || lane != 0) continue;
-      const GsInfo &mt = info[pmi];
-      const int r_base = (rl ? pend_tile1 : pend_tile0) * kGsRows + warp * 16 * R + rt * 16;
-      if (r_base < mt.N) olds[rl][rt] = atomicAdd(mt.cnt + (r_base >> 4), (unsigned)(rl ? pend_len1 : pend_len0));
-    }
-#pragma unroll
-  for (int rl = 0; rl < 2; ++rl) {
-    const int pmi = rl ? pend_mi1 : pend_mi0;
-    if (pmi < 0) continue;
-    const GsInfo &mt = info[pmi];
-    const int N = mt.N, Q = mt.n_stages;
-    const int tile = rl ? pend_tile1 : pend_tile0;
-    const unsigned len = (unsigned)(rl ? pend_len1 : pend_len0);
-    const uint32_t x0 = mt.stage_begin + (uint32_t)(tile * Q);  // the tile's first stage
-#pragma unroll
-    for (int rt = 0; rt < R; ++rt) {
-      const int r_base = tile * kGsRows + warp * 16 * R + rt * 16;
-      if (r_base >= N) continue;
-      const unsigned old = __shfl_sync(0xffffffffu, olds[rl][rt], 0);
-      if (old + len != (unsigned)Q) continue;
-      // every contributor has counted: sum their slots in CTA order
-      __syncwarp();
-      fence_acq_rel_gpu();
-      const int c0 = gs_cta_of(x0, T, G), c1 = gs_cta_of(x0 + Q - 1, T, G);
-      float sum[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) sum[nt][j] = 0.0f;
-      for (int cb = c0; cb <= c1; cb += 4) {
-        // up to four contributors' rows in flight at once, added in CTA order
-        float2 v[4][NT][2];
-        float *slot[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int c = min(cb + k, c1);
-          const int role = (gs_range_begin(c, T, G) >= x0) ? 0 : 1;  // c starts inside the tile
-          slot[k] = p.slots + ((int64_t)(c * 2 + role) * kGsRows + warp * 16 * R + rt * 16 + g) * MW + 2 * tig;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              v[k][nt][h] = __ldcg(reinterpret_cast<const float2 *>(slot[k] + (h * 8) * MW + nt * 8));
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (cb + k > c1) break;
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              // the workspace is left zeroed
-              __stcg(reinterpret_cast<float2 *>(slot[k] + (h * 8) * MW + nt * 8), make_float2(0.0f, 0.0f));
-              sum[nt][2 * h] += v[k][nt][h].x;
-              sum[nt][2 * h + 1] += v[k][nt][h].y;
-            }
-        }
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = r_base + (j >> 1) * 8 + g;
-          const int m = nt * 8 + 2 * tig + (j & 1);
-          if (m < M && row < N) gs_store(mt.Y, p.y_dtype, (int64_t)m * N + row, sum[nt][j]);
-        }
-      if (lane == 0) mt.cnt[r_base >> 4] = 0u;
-    }
-  }
+  if (!ok) return;
+  if (pend_mi1 >= 0) sum_piece(pend_mi1, pend_tile1, count_piece(pend_mi1, pend_tile1, (unsigned)pend_len1));
+  if (pend_mi0 >= 0 && done0) sum_piece(pend_mi0, pend_tile0, done0);
 }
 
 }  // namespace q4
