@@ -49,7 +49,7 @@ NCU_TRAFFIC = {
     "gemm": ("bit_blockwise_weight_absmax_b200/csrc/gemm.cuh",
              "131690000b067cfa5b54292cd0fcbaaca0955854007702fa36d49b37172ba8dd", 142_834_176 + 19_374_592),
     "gemv": ("bit_blockwise_weight_absmax_b200/csrc/gemv_small.cuh",
-             "6721fbd3bd7b25d31d2883e150619d5e9d6219e3ae024ce700d78fcb40b82906", 108_711_936 + 6_480_640),
+             "e1c37f32b32c6306cbcee77f09a0121d152d14267279be05e5e7aa0ea42ff327", 108_468_224 + 3_651_840),
 }
 
 
