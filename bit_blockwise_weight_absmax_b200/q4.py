@@ -356,7 +356,7 @@ def quantize_grouped(Ws, blocksize: int = 64, qtype="nf4", double_quant: bool = 
                                                          ctypes.byref(wsz)), "q4_quantize_grouped_workspace_size")
     ws = _workspace(dev, "quantize", wsz.value)
     structs = [st.c_struct() for st in outs]
-    arr = (ctypes.POINTER(_CState) * n)(*[ctypes.pointer(c) for c in structs])
+    arr = _struct_array(structs)
     wp = (ctypes.c_void_p * n)(*[W.data_ptr() for W in Ws])
     _check(library().q4_quantize_grouped(n, wp, _DT[dtype], rows, cols, blocksize, qt_arg, int(double_quant), arr,
                                          _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
@@ -384,7 +384,7 @@ def dequantize_grouped(states, dtype: torch.dtype | None = None, outs=None, stre
         outs = [torch.empty(st.rows, st.cols, dtype=dtype, device=st.device) for st in states]
     structs = [st.c_struct() for st in states]
     n = len(states)
-    arr = (ctypes.POINTER(_CState) * n)(*[ctypes.pointer(c) for c in structs])
+    arr = _struct_array(structs)
     op = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
     _check(library().q4_dequantize_grouped(n, arr, op, _DT[dtype], _stream(stream)), "q4_dequantize_grouped")
     return outs
