@@ -302,6 +302,11 @@ def test_gemm_plan_tile_height_and_cuts(lib):
     assert _plan(lib, [(2560, 16384)], 1000) == (0, 512, 80, 40)
     # fewer SMs: the same layer still takes tall tiles, and the grid follows
     assert _plan(lib, layer, 512, sms=74) == (0, 512, 74, 0)
+    # cuts only within the workspace: 64 KB of counters, then one 512 KB
+    # fp32 slot per cut tile (128 weight rows x 512 tokens x two halves)
+    need = 65536 + 64 * 524288
+    assert _plan(lib, [(4096, 4096)], 512, ws=need) == (0, 256, 128, 64)
+    assert _plan(lib, [(4096, 4096)], 512, ws=need - 1) == (0, 256, 64, 0)
     # argument and shape checks, before any device is asked for
     assert _plan(lib, layer, 512, sms=0)[0] == -1
     assert _plan(lib, layer, 512, sms=1025)[0] == -1
