@@ -103,9 +103,12 @@ DeviceInfo device_info() {
   if (filled[dev]) return cache[dev];
   DeviceInfo d;
   int major = 0, minor = 0;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || d.sms < 1) {
+    cudaGetLastError();
+    return DeviceInfo{Q4_ERR_CUDA, 0, nullptr};  // not cached: a later call asks again
+  }
   d.ok = (major == 10 && minor == 0) ? Q4_OK : Q4_ERR_ARCH;
   if (d.ok == Q4_OK) {
     void *ptr = nullptr;
